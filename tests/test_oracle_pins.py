@@ -1,0 +1,396 @@
+"""Pins of the CPU oracle against things other than itself.
+
+Hand-worked fixtures, closed forms, brute force on tiny inputs, an
+independently written dense attention (plus torch's SDPA in fp64), torch's
+bf16 conversion, and the structural invariants the page implies (split read
+plus combine equals the unsplit read; replicated selector; one cache group;
+synthetic tokens write nothing).
+"""
+
+import itertools
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from synth import make_custom, make_workload
+from synth.workloads import Dims
+from tests.helpers import bits, exact_bf16, golden
+
+pytestmark = pytest.mark.filterwarnings("ignore")
+
+
+# ------------------------------------------------------------ bf16 helpers
+
+def test_bf16_rounding_matches_torch():
+    g = torch.Generator().manual_seed(7)
+    x = torch.randn(200000, generator=g) * torch.exp(torch.randn(200000, generator=g) * 8)
+    special = torch.tensor([0.0, -0.0, 1.0, -1.0, 1.00390625, 1.01171875, 3.3895314e38,
+                            float("inf"), float("-inf"), 1e-40, -1e-40, 65504.0],
+                           dtype=torch.float32)
+    x = torch.cat([x, special])
+    ref = bits(x.to(torch.bfloat16))
+    got = oracle.f32_to_bf16(x.numpy())
+    assert np.array_equal(got, ref)
+    back = oracle.bf16_to_f32(ref)
+    assert np.array_equal(back, x.to(torch.bfloat16).to(torch.float32).numpy())
+
+
+# ---------------------------------------------------- micro-block keys
+
+def test_compress_hand_cases():
+    d = golden("compress_rounding_hand.json")
+    for case in d["cases"] + d["partial_cases"]:
+        keys = exact_bf16(case["keys"]).reshape(len(case["keys"]), 1)
+        got = int(oracle.compress_keys(keys)[0])
+        assert got == int(case["bf16"], 16), case["derivation"]
+
+
+def test_compress_within_one_ulp_of_exact_mean():
+    g = np.random.default_rng(3)
+    keys = oracle.f32_to_bf16(g.standard_normal((4096, 4, 64)).astype(np.float32))
+    kc = oracle.bf16_to_f32(oracle.compress_keys(keys)).astype(np.float64)
+    exact = oracle.bf16_to_f32(keys).astype(np.float64).mean(axis=1)
+    ulp = np.ldexp(1.0, np.floor(np.log2(np.maximum(np.abs(exact), 1e-30))).astype(int) - 7)
+    assert np.all(np.abs(kc - exact) <= ulp)
+
+
+def test_side_cache_equals_blockwise_compress():
+    g = np.random.default_rng(4)
+    kidx = oracle.f32_to_bf16(g.standard_normal((403, 16)).astype(np.float32))
+    side = oracle.side_cache(kidx, 403)
+    assert side.shape == (100, 16)
+    for j in (0, 1, 57, 99):
+        assert np.array_equal(side[j], oracle.compress_keys(kidx[4 * j:4 * j + 4]))
+    kc = oracle.block_keys(kidx, 403)
+    assert kc.shape == (101, 16)
+    tail = oracle.bf16_to_f32(oracle.compress_keys(kidx[400:403]))
+    assert np.array_equal(kc[100], tail.astype(np.float64))
+
+
+# ------------------------------------------------------------- scoring
+
+def test_score_and_topk_hand():
+    d = golden("score_topk_hand.json")
+    kidx = exact_bf16(d["kidx"])
+    q = exact_bf16(d["q_idx"])
+    w = np.asarray(d["w"], dtype=np.float32)
+    kc = oracle.block_keys(kidx, d["L"])
+    assert np.array_equal(kc, np.asarray(d["kc"], dtype=np.float64))
+    s = oracle.index_scores(kc, q, w)
+    assert np.array_equal(s, np.asarray(d["scores"]))
+    for k, sel in d["topk"].items():
+        assert oracle.topk_blocks(s, int(k)).tolist() == sel
+    full = oracle.decode_sequence(kidx, np.zeros((10, 1, 4), np.uint16),
+                                  np.zeros((10, 1, 4), np.uint16), np.zeros((1, 4), np.uint16),
+                                  q, w, d["L"], 2, 1, 1.0)
+    assert full["sel"].tolist() == d["topk"]["2"]
+
+
+def test_score_closed_form_single_head():
+    # One head, w = 1: s_b = max(0, q . kc_b), checked with scalar loops.
+    g = np.random.default_rng(5)
+    kidx = oracle.f32_to_bf16(g.standard_normal((64, 8)).astype(np.float32))
+    q = oracle.f32_to_bf16(g.standard_normal((1, 8)).astype(np.float32))
+    kc = oracle.block_keys(kidx, 64)
+    s = oracle.index_scores(kc, q, np.ones(1, np.float32))
+    qf = oracle.bf16_to_f32(q)[0].astype(np.float64)
+    for b in range(16):
+        dot = sum(float(qf[i]) * float(kc[b, i]) for i in range(8))
+        assert abs(s[b] - max(0.0, dot)) <= 1e-12 * (1 + abs(dot))
+
+
+# ----------------------------------------------------------- selection
+
+def _topk_by_beat_count(scores, k):
+    """Brute force: block i is kept iff fewer than k blocks beat it, where j
+    beats i if s_j > s_i, or s_j == s_i and j < i."""
+    n = len(scores)
+    keep = [i for i in range(n)
+            if sum(1 for j in range(n) if scores[j] > scores[i]
+                   or (scores[j] == scores[i] and j < i)) < k]
+    return keep + [-1] * (k - len(keep))
+
+
+def test_topk_ties_hand():
+    for case in golden("topk_ties_hand.json")["cases"]:
+        got = oracle.topk_blocks(np.asarray(case["scores"], dtype=np.float64), case["k"])
+        assert got.tolist() == case["sel"], case["derivation"]
+
+
+def test_topk_exhaustive_tiny():
+    for nb in range(1, 8):
+        for combo in itertools.product((0.0, 1.0, 2.0), repeat=nb):
+            for k in range(1, nb + 2):
+                assert oracle.topk_blocks(np.asarray(combo), k).tolist() == \
+                    _topk_by_beat_count(list(combo), k)
+
+
+def test_topk_random_with_ties():
+    g = np.random.default_rng(6)
+    for _ in range(300):
+        nb = int(g.integers(1, 60))
+        s = g.integers(0, 6, nb).astype(np.float64) * 0.5
+        k = int(g.integers(1, 70))
+        assert oracle.topk_blocks(s, k).tolist() == _topk_by_beat_count(s.tolist(), k)
+
+
+def test_all_zero_index_keys_select_first_blocks():
+    kidx = np.zeros((4099, 64), dtype=np.uint16)
+    q = oracle.f32_to_bf16(np.random.default_rng(1).standard_normal((4, 64)).astype(np.float32))
+    s = oracle.index_scores(oracle.block_keys(kidx, 4099), q, np.ones(4, np.float32))
+    assert np.all(s == 0.0)
+    assert oracle.topk_blocks(s, 512).tolist() == list(range(512))
+
+
+def test_planted_needles_always_selected_tiny_config():
+    wl = make_workload(1, device="cpu")
+    for b in range(wl.B):
+        K, V, X = wl.seq_tokens(b)
+        res = oracle.decode_sequence(bits(X), bits(K), bits(V), bits(wl.q[b]), bits(wl.q_idx[b]),
+                                     wl.w[b].numpy(), wl.seq_lens[b], wl.k, wl.R, wl.dims.scale)
+        sel = set(res["sel"].tolist())
+        assert set(wl.needles[b]) <= sel
+        s = res["scores"]
+        assert min(s[j] for j in wl.needles[b]) > np.sort(s)[::-1][min(wl.k, len(s)) - 1]
+
+
+def test_planted_needles_always_selected_mixture():
+    d = Dims(Hq=8, Hkv=1, D=32, Hi=16, di=128, P=64, scale=1 / math.sqrt(32))
+    wl = make_custom(d, [16384], k=512, R=4, seed=11, needles=8, mixture=True)
+    K, V, X = wl.seq_tokens(0)
+    kc = oracle.block_keys(bits(X), 16384)
+    s = oracle.index_scores(kc, bits(wl.q_idx[0]), wl.w[0].numpy())
+    sel = set(oracle.topk_blocks(s, 512).tolist())
+    assert set(wl.needles[0]) <= sel
+
+
+# ----------------------------------------------------------- attention
+
+def _expr(e):
+    return float(eval(e, {"e": math.e, "ln": math.log}))
+
+
+def test_attention_hand():
+    d = golden("attention_hand.json")
+    q = exact_bf16(d["q"])
+    K = exact_bf16(d["K"])
+    V = exact_bf16(d["V"])
+    sel = np.array([0, 1, -1])
+    O1, L1 = oracle.attend_slices(q, K, V, sel, d["L"], d["scale"], 1)
+    for h in range(2):
+        assert abs(L1[0, h] - _expr(d["expr"]["R1"]["LSE"][h])) < 1e-12
+        for c in range(2):
+            assert abs(O1[0, h, c] - _expr(d["expr"]["R1"]["O"][h][c])) < 1e-12
+    O2, L2 = oracle.attend_slices(q, K, V, sel, d["L"], d["scale"], 2)
+    for r in range(2):
+        for h in range(2):
+            assert abs(L2[r, h] - _expr(d["expr"]["R2"]["LSE"][r][h])) < 1e-12
+            for c in range(2):
+                assert abs(O2[r, h, c] - _expr(d["expr"]["R2"]["O"][r][h][c])) < 1e-12
+    Om, Lm = oracle.merge_partials(O2, L2)
+    assert np.allclose(Om, O1[0], atol=1e-12) and np.allclose(Lm, L1[0], atol=1e-12)
+    # selecting only the partial block: one token, LSE = z_4
+    O3, L3 = oracle.attend_slices(q, K, V, np.array([1]), d["L"], d["scale"], 1)
+    assert L3[0].tolist() == [2.0, 0.0] and O3[0].tolist() == [[4.0, -4.0], [4.0, -4.0]]
+
+
+def _dense_loops(q, K, V, L, scale, G):
+    """Textbook softmax attention with scalar loops (independent of the oracle)."""
+    Hq, D = len(q), len(q[0])
+    out, lses = [], []
+    for h in range(Hq):
+        g = h // G
+        z = [scale * sum(q[h][d] * K[t][g][d] for d in range(D)) for t in range(L)]
+        m = max(z)
+        ex = [math.exp(v - m) for v in z]
+        s = sum(ex)
+        out.append([sum(ex[t] * V[t][g][d] for t in range(L)) / s for d in range(D)])
+        lses.append(m + math.log(s))
+    return np.array(out), np.array(lses)
+
+
+def test_full_selection_equals_dense_attention_loops():
+    d = Dims(Hq=4, Hkv=2, D=8, Hi=2, di=8, P=8, scale=0.35)
+    wl = make_custom(d, [37], k=16, R=3, seed=12, paged=False)
+    K, V, X = wl.seq_tokens(0)
+    res = oracle.decode_sequence(bits(X), bits(K), bits(V), bits(wl.q[0]), bits(wl.q_idx[0]),
+                                 wl.w[0].numpy(), 37, 16, 3, d.scale)
+    assert res["sel"][:10].tolist() == list(range(10)) and np.all(res["sel"][10:] == -1)
+    f = lambda t: t.to(torch.float64).tolist()
+    O, LSE = _dense_loops(f(wl.q[0]), f(K), f(V), 37, d.scale, d.G)
+    assert np.allclose(res["O"], O, atol=1e-12, rtol=0)
+    assert np.allclose(res["LSE"], LSE, atol=1e-12, rtol=0)
+
+
+def test_full_selection_equals_sdpa_fp64():
+    # the tiny preset's 1500-token sequence has 375 < 512 blocks: all selected
+    wl = make_workload(1, device="cpu")
+    b, L = 1, wl.seq_lens[1]
+    K, V, X = wl.seq_tokens(b)
+    res = oracle.decode_sequence(bits(X), bits(K), bits(V), bits(wl.q[b]), bits(wl.q_idx[b]),
+                                 wl.w[b].numpy(), L, wl.k, wl.R, wl.dims.scale)
+    assert res["sel"][:375].tolist() == list(range(375))
+    G = wl.dims.G
+    qh = wl.q[b].to(torch.float64)[None, :, None, :]                   # [1, Hq, 1, D]
+    Kh = K.to(torch.float64).repeat_interleave(G, dim=1).permute(1, 0, 2)[None]
+    Vh = V.to(torch.float64).repeat_interleave(G, dim=1).permute(1, 0, 2)[None]
+    ref = torch.nn.functional.scaled_dot_product_attention(qh, Kh, Vh, scale=wl.dims.scale)
+    assert np.allclose(res["O"], ref[0, :, 0].numpy(), atol=1e-10, rtol=0)
+    z = (qh @ Kh.transpose(-1, -2))[0, :, 0] * wl.dims.scale
+    assert np.allclose(res["LSE"], torch.logsumexp(z, dim=-1).numpy(), atol=1e-10, rtol=0)
+
+
+def test_split_merge_equals_unsplit():
+    d = Dims(Hq=8, Hkv=2, D=32, Hi=4, di=32, P=16, scale=0.2)
+    wl = make_custom(d, [997], k=40, R=1, seed=13, paged=False)
+    K, V, X = wl.seq_tokens(0)
+    args = (bits(wl.q[0]), bits(K), bits(V))
+    sel = oracle.topk_blocks(oracle.index_scores(oracle.block_keys(bits(X), 997),
+                                                 bits(wl.q_idx[0]), wl.w[0].numpy()), 40)
+    O1, L1 = oracle.attend_slices(*args, sel, 997, d.scale, 1)
+    for R in (2, 3, 4, 7, 8, 64):
+        O, Ls = oracle.attend_slices(*args, sel, 997, d.scale, R)
+        Om, Lm = oracle.merge_partials(O, Ls)
+        assert np.abs(Om - O1[0]).max() <= 1e-12 and np.abs(Lm - L1[0]).max() <= 1e-12
+
+
+def test_slice_bounds_hand():
+    assert oracle.slice_bounds(10, 4) == [(0, 2), (2, 5), (5, 7), (7, 10)]
+    assert oracle.slice_bounds(3, 4) == [(0, 0), (0, 1), (1, 2), (2, 3)]
+    assert oracle.slice_bounds(7, 1) == [(0, 7)]
+
+
+def test_q_zero_closed_form_per_slice():
+    # q = 0: every z_t = 0, so LSE_r = ln(#valid tokens of slice r) and O_r is the
+    # plain mean of those V rows. L = 41 -> nb = 11, R = 4 -> slices
+    # [0,2) [2,5) [5,8) [8,11); block 10 holds only token 40.
+    d = Dims(Hq=4, Hkv=2, D=16, Hi=2, di=16, P=16, scale=0.3)
+    wl = make_custom(d, [41], k=11, R=4, seed=14, paged=False)
+    K, V, _ = wl.seq_tokens(0)
+    q0 = np.zeros((4, 16), np.uint16)
+    sel = np.array([0, 3, 4, 5, 9, 10, -1])
+    O, LSE = oracle.attend_slices(q0, bits(K), bits(V), sel, 41, d.scale, 4)
+    counts = [4, 8, 4, 5]             # slice 0: block 0; 1: 3,4; 2: 5; 3: 9 + token 40
+    toks = [[0, 1, 2, 3], list(range(12, 20)), list(range(20, 24)), [36, 37, 38, 39, 40]]
+    Vf = V.to(torch.float64).numpy()
+    for r in range(4):
+        for h in range(4):
+            assert abs(LSE[r, h] - math.log(counts[r])) < 1e-12
+            assert np.allclose(O[r, h], Vf[toks[r], h // 2].mean(axis=0), atol=1e-12)
+
+
+def test_constant_v_per_kv_head_gives_that_constant():
+    d = Dims(Hq=8, Hkv=4, D=16, Hi=2, di=16, P=16, scale=0.3)
+    wl = make_custom(d, [50], k=13, R=2, seed=15, paged=False)
+    K, _, _ = wl.seq_tokens(0)
+    consts = [1.5, -2.0, 0.25, 3.0]
+    Vc = np.stack([exact_bf16([[c] * 16 for c in consts])] * 50)   # [50, Hkv, D]
+    O, LSE = oracle.attend_slices(bits(wl.q[0]), bits(K), Vc, np.arange(13), 50, d.scale, 1)
+    for h in range(8):
+        assert np.allclose(O[0, h], consts[h // 2], atol=1e-12)
+
+
+def test_single_token_closed_form():
+    d = Dims(Hq=4, Hkv=1, D=16, Hi=2, di=16, P=16, scale=0.25)
+    wl = make_custom(d, [1], k=4, R=2, seed=16, paged=False)
+    K, V, X = wl.seq_tokens(0)
+    res = oracle.decode_sequence(bits(X), bits(K), bits(V), bits(wl.q[0]), bits(wl.q_idx[0]),
+                                 wl.w[0].numpy(), 1, 4, 2, d.scale)
+    assert res["sel"].tolist() == [0, -1, -1, -1]
+    q = wl.q[0].to(torch.float64).numpy()
+    k0 = K[0, 0].to(torch.float64).numpy()
+    for h in range(4):
+        assert abs(res["LSE"][h] - d.scale * float(q[h] @ k0)) < 1e-12
+        assert np.allclose(res["O"][h], V[0, 0].to(torch.float64).numpy(), atol=1e-12)
+    # nb = 1 with R = 2: slice 0 owns no block, slice 1 owns block 0
+    assert np.all(np.isneginf(res["LSE_part"][0])) and np.all(res["O_part"][0] == 0)
+
+
+def test_merge_ignores_empty_slices():
+    g = np.random.default_rng(8)
+    O = g.standard_normal((3, 5, 4))
+    LSE = g.standard_normal((3, 5))
+    LSE[1, :] = -np.inf
+    O[1] = 123.0
+    Om, Lm = oracle.merge_partials(O, LSE)
+    Om2, Lm2 = oracle.merge_partials(O[[0, 2]], LSE[[0, 2]])
+    assert np.allclose(Om, Om2, atol=1e-14) and np.allclose(Lm, Lm2, atol=1e-14)
+    Os, Ls = oracle.merge_partials(O[:1], LSE[:1])
+    assert np.allclose(Os, O[0]) and np.allclose(Ls, LSE[0])
+    # two equal-weight slices average; LSE grows by ln 2
+    Oe, Le = oracle.merge_partials(np.stack([O[0], O[2]]), np.stack([LSE[0], LSE[0]]))
+    assert np.allclose(Oe, (O[0] + O[2]) / 2) and np.allclose(Le, LSE[0] + math.log(2))
+
+
+# ------------------------------------------------------------ paged append
+
+def _pools(wl):
+    d = wl.dims
+    n = wl.num_pages
+    rng = np.random.default_rng(99)   # stale garbage, so untouched bytes are visible
+    mk = lambda *s: rng.integers(0, 1 << 16, size=s, dtype=np.uint16)
+    return (mk(n, d.P, d.Hkv, d.D), mk(n, d.P, d.Hkv, d.D), mk(n, d.P, d.di),
+            mk(n, d.P // 4, d.di))
+
+
+def test_append_token_by_token_equals_one_shot():
+    d = Dims(Hq=4, Hkv=2, D=8, Hi=2, di=8, P=16, scale=0.3)
+    lens = [259, 64, 3, 100]
+    wl = make_custom(d, lens, k=8, R=1, seed=17, paged=True)
+    bt = wl.block_table.numpy()
+    kp, vp, xp, sp = _pools(wl)
+    kp2, vp2, xp2, sp2 = (a.copy() for a in (kp, vp, xp, sp))
+    Kb, Vb, Xb = bits(wl.k_tok), bits(wl.v_tok), bits(wl.kidx_tok)
+    # incremental: one call per decode step, one token per sequence
+    for t in range(max(lens)):
+        seqs = [b for b in range(4) if t < lens[b]]
+        rows = [wl.tok_off[b] + t for b in seqs]
+        oracle.append_paged(kp, vp, xp, sp, bt, d.P, seqs, [t] * len(seqs),
+                            Kb[rows], Vb[rows], Xb[rows])
+    # bulk: every token in one call, in a shuffled order
+    order = np.random.default_rng(5).permutation(sum(lens))
+    seq_of = np.concatenate([[b] * n for b, n in enumerate(lens)])
+    pos_of = np.concatenate([np.arange(n) for n in lens])
+    oracle.append_paged(kp2, vp2, xp2, sp2, bt, d.P, seq_of[order], pos_of[order],
+                        Kb[order], Vb[order], Xb[order])
+    for a, b in zip((kp, vp, xp, sp), (kp2, vp2, xp2, sp2)):
+        assert np.array_equal(a, b)
+    # side slots of every complete block equal the one-shot side cache
+    for b, L in enumerate(lens):
+        one_shot = oracle.side_cache(Xb[wl.tok_off[b]:wl.tok_off[b] + L], L)
+        for j in range(L // 4):
+            page = bt[b, (4 * j) // d.P]
+            assert np.array_equal(sp[page, (4 * j % d.P) // 4], one_shot[j])
+            assert np.array_equal(kp[page, 4 * j % d.P], Kb[wl.tok_off[b] + 4 * j])
+
+
+def test_append_placement_by_hand():
+    d = Dims(Hq=2, Hkv=1, D=8, Hi=1, di=8, P=8, scale=1.0)
+    bt = np.array([[5, 2, -1], [0, 4, 1]])
+    n = 6
+    kp = np.zeros((n, 8, 1, 8), np.uint16)
+    vp, xp, sp = kp.copy(), np.zeros((n, 8, 8), np.uint16), np.zeros((n, 2, 8), np.uint16)
+    kv = np.arange(8, dtype=np.uint16).reshape(1, 1, 8) + 1
+    # seq 1, position 13 -> page bt[1][1] = 4, slot 5
+    oracle.append_paged(kp, vp, xp, sp, bt, d.P, [1], [13], kv, kv, kv[0])
+    assert np.array_equal(kp[4, 5], kv[0]) and kp.sum() == kv.sum()
+    # positions 4..7 of seq 0 close block 1 -> side page 5, slot 1
+    x = exact_bf16([[1.0] * 8, [2.0] * 8, [2.0] * 8, [3.0] * 8])
+    oracle.append_paged(kp, vp, xp, sp, bt, d.P, [0] * 4, [4, 5, 6, 7],
+                        np.zeros((4, 1, 8), np.uint16), np.zeros((4, 1, 8), np.uint16), x)
+    assert np.all(sp[5, 1] == 0x4000) and sp.sum() == 8 * 0x4000   # mean 2.0
+
+
+def test_padding_tokens_write_nothing():
+    d = Dims(Hq=4, Hkv=2, D=8, Hi=2, di=8, P=16, scale=0.3)
+    wl = make_custom(d, [40, 40], k=8, R=1, seed=18, paged=True)
+    bt = wl.block_table.numpy()
+    pools = _pools(wl)
+    before = [a.copy() for a in pools]
+    K, V, X = bits(wl.k_tok[:4]), bits(wl.v_tok[:4]), bits(wl.kidx_tok[:4])
+    oracle.append_paged(*pools, bt, d.P, [-1, 0, -1, 1], [3, -1, 7, -5], K, V, X)
+    for a, b in zip(pools, before):
+        assert np.array_equal(a, b)
