@@ -1,0 +1,442 @@
+#!/usr/bin/env python
+"""Benchmark of the QSA decode step on B200.
+
+One step = the whole hot path on one batch: qsa_append (the current token of
+every sequence) -> qsa_index_score -> qsa_topk_select -> qsa_sparse_decode
+(R-way split) -> qsa_merge, on seeded synthetic inputs already resident in
+HBM. Default workload: B=8 sequences x 262,144 tokens, 32 query / 4 KV heads,
+head dim 128, indexer 16 x 128, top-512 blocks, R=4, paged (P=64, shuffled).
+
+The step is captured once in a CUDA graph and replayed; L2 is flushed (a
+write larger than L2) before every timed step, outside the step's events.
+Prints one JSON line (rank 0). ``--impl reference`` times the CPU oracle on
+the same workload instead (a bounded sample per step).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 3]
+    torchrun --nproc-per-node N bench.py --gpus N ...   (replicas, weak scaling)
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "QSA decode seqs/s & attended tokens/s at 256K ctx; HBM GB/s as % of roofline"
+L2_FLUSH_BYTES = 512 << 20
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", type=int, default=3, choices=[2, 3, 4, 5])
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the batch size (smaller profiling case)")
+    ap.add_argument("--k", type=int, default=None)
+    ap.add_argument("--R", type=int, default=None)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------- helpers
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def profile_traffic(kernel_src: str, summary: str):
+    """Per-launch DRAM bytes of a kernel from a committed ncu summary, if the
+    summary was taken on the current source of that kernel (else None)."""
+    path = os.path.join(ROOT, "profiles", summary)
+    src = os.path.join(ROOT, "block_sparse_decode_b200", "csrc", kernel_src)
+    if not (os.path.exists(path) and os.path.exists(src)):
+        return None
+    text = open(path).read()
+    m_sha = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
+    m_b = re.search(r"dram_bytes_per_full_launch:\s*([0-9.eE+]+)", text)
+    if not (m_sha and m_b):
+        return None
+    if hashlib.sha256(open(src, "rb").read()).hexdigest() != m_sha.group(1):
+        return None
+    return float(m_b.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.06)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        rows = []
+        for line in (self.out or "").strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), parts[4:8]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({n for _, _, flags in rows for n, f in zip(names, flags)
+                          if f.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows)}
+
+
+def algorithmic_bytes(seq_lens, dims, k):
+    side = sum(((L + 3) // 4) * dims.di * 2 for L in seq_lens)
+    kv = sum(min(4 * k, L) * dims.Hkv * dims.D * 2 * 2 for L in seq_lens)
+    return side, kv
+
+
+# ------------------------------------------------------------ our arm
+
+def run_ours(args, rank, world, local_rank):
+    from block_sparse_decode_b200 import qsa
+    from synth import make_custom, config_spec, seed_for
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    spec = config_spec(args.config)
+    k = args.k or spec["k"]
+    R = args.R or spec["R"]
+    lens = list(spec["seq_lens"])
+    if args.batch:
+        lens = (lens * ((args.batch + len(lens) - 1) // len(lens)))[:args.batch]
+    if args.config == 5:
+        lens = [spec["prefill"] + 1] * len(lens)
+    seed = seed_for(args.config) + 7919 * rank
+    wl = make_custom(spec["dims"], lens, k=k, R=R, seed=seed, device=dev,
+                     paged=spec["paged"], needles=spec["needles"], mixture=spec["mixture"],
+                     name=f"config{args.config}", config_id=args.config)
+    dims = qsa.QsaDims.of(wl.dims)
+    B = wl.B
+
+    # cache: prefill L-1 tokens in bulk; the step appends token L-1
+    cache = qsa.alloc_cache(dims, wl.num_pages, wl.block_table, device=dev)
+    T = sum(wl.cap_lens)
+    tok_seq = torch.empty(T, dtype=torch.int32, device=dev)
+    tok_pos = torch.empty(T, dtype=torch.int32, device=dev)
+    for b, L in enumerate(wl.cap_lens):
+        o = wl.tok_off[b]
+        tok_seq[o:o + L] = b
+        tok_pos[o:o + L] = torch.arange(L, dtype=torch.int32, device=dev)
+        tok_seq[o + wl.seq_lens[b] - 1:o + L] = -1
+    qsa.qsa_append(dims, cache, tok_seq, tok_pos, wl.k_tok, wl.v_tok, wl.kidx_tok)
+    del tok_seq, tok_pos
+    rows = torch.tensor([wl.tok_off[b] + L - 1 for b, L in enumerate(wl.seq_lens)], device=dev)
+    step_in = dict(
+        tok_seq=torch.arange(B, dtype=torch.int32, device=dev),
+        tok_pos=torch.tensor([L - 1 for L in wl.seq_lens], dtype=torch.int32, device=dev),
+        k_new=wl.k_tok[rows].contiguous(), v_new=wl.v_tok[rows].contiguous(),
+        kidx_new=wl.kidx_tok[rows].contiguous(),
+        seq_lens=torch.tensor(wl.seq_lens, dtype=torch.int32, device=dev),
+        q=wl.q.contiguous(), q_idx=wl.q_idx.contiguous(), w=wl.w.contiguous())
+    ld = qsa.ld_for(wl.seq_lens)
+    buf = qsa.alloc_step(dims, B, ld, k, R, device=dev)
+    qsa.qsa_check_device_errors()
+
+    # host-side copies for the oracle baseline (seq 0), then free the token arrays
+    cpu_sample = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        K0, V0, X0 = wl.seq_tokens(0)
+        cpu_sample = dict(K=K0.cpu(), V=V0.cpu(), X=X0.cpu(), q=wl.q[0].cpu(),
+                          q_idx=wl.q_idx[0].cpu(), w=wl.w[0].cpu(), L=wl.seq_lens[0])
+    del wl.k_tok, wl.v_tok, wl.kidx_tok
+    torch.cuda.empty_cache()
+
+    stream = torch.cuda.Stream(device=dev)
+    ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(6)]
+
+    def step(record):
+        si = step_in
+        if record:
+            ev[0].record()
+        qsa.qsa_append(dims, cache, si["tok_seq"], si["tok_pos"], si["k_new"], si["v_new"],
+                       si["kidx_new"])
+        if record:
+            ev[1].record()
+        qsa.qsa_index_score(dims, cache, si["seq_lens"], si["q_idx"], si["w"], buf.scores)
+        if record:
+            ev[2].record()
+        qsa.qsa_topk_select(si["seq_lens"], buf.scores, k, buf.sel)
+        if record:
+            ev[3].record()
+        qsa.qsa_sparse_decode(dims, cache, si["seq_lens"], si["q"], buf.sel, k, R, buf.o_part,
+                              buf.lse_part, buf.ws)
+        if record:
+            ev[4].record()
+        qsa.qsa_merge(buf.o_part, buf.lse_part, buf.out, buf.lse)
+        if record:
+            ev[5].record()
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):  # eager warm-up (module load, attributes)
+            step(False)
+    torch.cuda.synchronize(dev)
+    qsa.qsa_check_device_errors()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        step(True)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def timed_iter():
+        with torch.cuda.stream(stream):
+            flush.zero_()
+            s0.record()
+            graph.replay()
+            s1.record()
+        s1.synchronize()
+        parts = [ev[i].elapsed_time(ev[i + 1]) for i in range(5)]
+        return s0.elapsed_time(s1), parts
+
+    for _ in range(max(3, args.warmup)):
+        timed_iter()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    step_ms, part_ms = [], []
+    with ClockSampler(local_rank) as clk:
+        for _ in range(args.steps):
+            t, p = timed_iter()
+            step_ms.append(t)
+            part_ms.append(p)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    qsa.qsa_check_device_errors()
+
+    tot = torch.tensor([sum(step_ms)], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(tot, op=torch.distributed.ReduceOp.MAX)
+    ms_per_step = float(tot.item()) / args.steps
+
+    # e2e: host buffers in pinned memory, copies inside the timed region,
+    # calls made eagerly through the binding (the user's API)
+    e2e = None
+    if not args.no_e2e:
+        host_in = {n: t.cpu().pin_memory() for n, t in step_in.items()}
+        host_out = torch.empty(buf.out.shape, dtype=buf.out.dtype).pin_memory()
+        host_lse = torch.empty(buf.lse.shape, dtype=torch.float32).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+        d2h = host_out.numel() * host_out.element_size() + host_lse.numel() * 4
+        e_ms = []
+        for i in range(max(3, args.warmup) + args.steps):
+            with torch.cuda.stream(stream):
+                flush.zero_()
+                s0.record()
+                for n, t in host_in.items():
+                    step_in[n].copy_(t, non_blocking=True)
+                step(False)
+                host_out.copy_(buf.out, non_blocking=True)
+                host_lse.copy_(buf.lse, non_blocking=True)
+                s1.record()
+            s1.synchronize()
+            if i >= max(3, args.warmup):
+                e_ms.append(s0.elapsed_time(s1))
+        et = torch.tensor([sum(e_ms)], dtype=torch.float64, device=dev)
+        if world > 1:
+            torch.distributed.all_reduce(et, op=torch.distributed.ReduceOp.MAX)
+        e_step = float(et.item()) / args.steps
+        e2e = {"value": world * B / (e_step / 1e3), "unit": "seqs/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": e_step, "api": "eager qsa_* calls through the ctypes binding"}
+
+    side_b, kv_b = algorithmic_bytes(wl.seq_lens, dims, k)
+    mean_parts = [statistics.mean(p[i] for p in part_ms) for i in range(5)]
+    names = ["append", "index_score", "topk_select", "sparse_decode", "merge"]
+    peak, peak_kind = load_peaks()
+    score_ms = mean_parts[1]
+    achieved = side_b / (score_ms / 1e3) / 1e9
+    traffic = profile_traffic("index_score.cu", "index_score_config3.md")
+    attended = sum(min(4 * k, L) for L in wl.seq_lens)
+    res = {
+        "metric": METRIC,
+        "value": world * B / (ms_per_step / 1e3),
+        "unit": "seqs/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": f"config{args.config}: B={B} x L={max(wl.seq_lens)} tokens, "
+                               f"32q/4kv heads x 128, indexer 16x128, top-{k} blocks of 4, "
+                               f"R={R}, paged P=64 (shuffled)",
+                   "batch": B, "context": max(wl.seq_lens), "k": k, "R": R,
+                   "l2": "flushed before every timed step (512 MiB write)",
+                   "step": "CUDA graph of append+score+topk+decode+merge",
+                   "parallelism": f"replicas x{world}"},
+        "attended_tokens_per_s": world * attended / (ms_per_step / 1e3),
+        "roofline": {"bound": "hbm", "kernel": "qsa_index_score", "achieved": achieved,
+                     "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "peak_source": peak_kind,
+                     "traffic": None if traffic is None else traffic * B / 8.0,
+                     "algorithmic_bytes": side_b},
+        "kernels_us": {n: 1e3 * m for n, m in zip(names, mean_parts)},
+        "score_plus_decode": {
+            "bytes": side_b + kv_b,
+            "us": 1e3 * (mean_parts[1] + mean_parts[3]),
+            "gbs": (side_b + kv_b) / ((mean_parts[1] + mean_parts[3]) / 1e3) / 1e9,
+            "frac": (side_b + kv_b) / ((mean_parts[1] + mean_parts[3]) / 1e3) / 1e9 / peak},
+        "step_roofline_frac": (side_b + kv_b) / (ms_per_step / 1e3) / 1e9 / peak,
+        "gpu_launches": 7 * args.steps,
+        "clocks": clk.summary(),
+        "e2e": e2e,
+    }
+    graph.reset()
+    if cpu_sample is not None:
+        res["cpu_baseline"] = cpu_baseline(cpu_sample, dims, k, R)
+    return res
+
+
+def _threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info()]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def _oracle_one(sample, dims, k, R):
+    import oracle
+    to_bits = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)
+    return oracle.decode_sequence(to_bits(sample["X"]), to_bits(sample["K"]),
+                                  to_bits(sample["V"]), to_bits(sample["q"]),
+                                  to_bits(sample["q_idx"]), sample["w"].numpy(), sample["L"],
+                                  k, R, dims.scale)
+
+
+def cpu_baseline(sample, dims, k, R, budget_s=12.0):
+    """The oracle, as it stands, on whole sequences of the same workload."""
+    n, t0 = 0, time.perf_counter()
+    while True:
+        _oracle_one(sample, dims, k, R)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or n >= 20:
+            break
+    return {"value": n / el, "unit": "seqs/s", "cores": _threads(), "kind": "oracle",
+            "sample": f"{n} full decode(s) of one {sample['L']}-token sequence of the same "
+                      f"workload (score, top-{k}, R={R} attention, merge), numpy fp64"}
+
+
+# ------------------------------------------------------------ reference arm
+
+def run_reference(args):
+    from synth import make_custom, config_spec, seed_for
+    from block_sparse_decode_b200.qsa import QsaDims
+
+    spec = config_spec(args.config)
+    k = args.k or spec["k"]
+    R = args.R or spec["R"]
+    L = max(spec["seq_lens"]) if args.config != 5 else spec["prefill"] + 1
+    B = len(spec["seq_lens"]) if not args.batch else args.batch
+    wl = make_custom(spec["dims"], [L], k=k, R=R, seed=seed_for(args.config), device="cpu",
+                     paged=spec["paged"], needles=spec["needles"], mixture=spec["mixture"])
+    K, V, X = wl.seq_tokens(0)
+    sample = dict(K=K, V=V, X=X, q=wl.q[0], q_idx=wl.q_idx[0], w=wl.w[0], L=L)
+    dims = QsaDims.of(wl.dims)
+    for _ in range(max(0, min(args.warmup, 3))):
+        _oracle_one(sample, dims, k, R)
+    t = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        _oracle_one(sample, dims, k, R)
+        t.append(time.perf_counter() - t0)
+    ms = 1e3 * statistics.mean(t)
+    v = 1.0 / (ms / 1e3)
+    return {"impl": "reference", "metric": METRIC, "value": v, "unit": "seqs/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": f"config{args.config}: one {L}-token sequence per step "
+                                   f"(B={B} workload sampled), top-{k}, R={R}",
+                       "batch": 1, "context": L, "k": k, "R": R},
+            "cpu_baseline": {"value": v, "unit": "seqs/s", "cores": _threads(),
+                             "kind": "oracle",
+                             "sample": f"one sequence of {L} tokens per step"},
+            "e2e": {"value": v, "unit": "seqs/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+    if world > 1:
+        torch.distributed.init_process_group(
+            "nccl", timeout=datetime.timedelta(seconds=120),
+            device_id=torch.device("cuda", local_rank))
+    res = run_ours(args, rank, world, local_rank)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,298 @@
+// C ABI of libqsa.so: argument checks, the device error word and dispatch to
+// the kernel launchers. See include/qsa.h for the contract of every call.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "common.cuh"
+#include "launch.h"
+
+#define QSA_VERSION_NUM 100  // 0.1.0
+
+namespace qsa {
+
+// One error word per device (module-scope device variable, no allocation).
+__device__ unsigned g_err_word;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+unsigned *g_err_ptr[kMaxDevices] = {};
+int g_sm_count[kMaxDevices] = {};
+
+thread_local std::string t_last_error;
+
+int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  return dev;
+}
+
+}  // namespace
+
+unsigned *device_error_word(cudaError_t *status) {
+  *status = cudaSuccess;
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) {
+    *status = cudaErrorInvalidDevice;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_err_ptr[dev] == nullptr) {
+    void *p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_err_word);
+    if (e != cudaSuccess) {
+      *status = e;
+      return nullptr;
+    }
+    g_err_ptr[dev] = static_cast<unsigned *>(p);
+    int sms = 0;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    g_sm_count[dev] = sms > 0 ? sms : 148;
+  }
+  return g_err_ptr[dev];
+}
+
+int device_sm_count() {
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return 148;
+  std::lock_guard<std::mutex> lk(g_mu);
+  return g_sm_count[dev] > 0 ? g_sm_count[dev] : 148;
+}
+
+}  // namespace qsa
+
+using namespace qsa;
+
+namespace {
+
+qsa_status fail(qsa_status s, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  t_last_error = buf;
+  return s;
+}
+
+qsa_status ok() {
+  t_last_error.clear();
+  return QSA_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+qsa_status check_dims(const qsa_dims *d) {
+  if (d == nullptr) return fail(QSA_ERR_INVALID_ARG, "dims is NULL");
+  if (d->Hq <= 0 || d->Hkv <= 0 || d->D <= 0 || d->Hi <= 0 || d->di <= 0 || d->P <= 0)
+    return fail(QSA_ERR_INVALID_ARG, "dims must be positive");
+  if (d->Hq % d->Hkv != 0)
+    return fail(QSA_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hkv (%d)", d->Hq, d->Hkv);
+  if (d->D != 128) return fail(QSA_ERR_UNSUPPORTED, "head dim D=%d unsupported (128)", d->D);
+  if (d->di != 64 && d->di != 128)
+    return fail(QSA_ERR_UNSUPPORTED, "indexer dim di=%d unsupported (64, 128)", d->di);
+  if (d->Hi > 32) return fail(QSA_ERR_UNSUPPORTED, "indexer heads Hi=%d > 32", d->Hi);
+  if (d->Hq / d->Hkv > 8)
+    return fail(QSA_ERR_UNSUPPORTED, "GQA group %d > 8", d->Hq / d->Hkv);
+  if (d->P % 4 != 0 || d->P > 1024)
+    return fail(QSA_ERR_UNSUPPORTED, "page size P=%d must be a multiple of 4, <= 1024", d->P);
+  if (!(d->scale == d->scale)) return fail(QSA_ERR_INVALID_ARG, "scale is NaN");
+  return QSA_OK;
+}
+
+qsa_status check_cache(const qsa_cache *c, bool need_kv, bool need_side) {
+  if (c == nullptr) return fail(QSA_ERR_INVALID_ARG, "cache is NULL");
+  if (c->block_table == nullptr) return fail(QSA_ERR_INVALID_ARG, "block_table is NULL");
+  if (c->num_seqs < 0 || c->max_pages_per_seq <= 0 || c->num_pages <= 0)
+    return fail(QSA_ERR_INVALID_ARG, "cache sizes must be positive");
+  if (need_kv && (c->k_pool == nullptr || c->v_pool == nullptr || !aligned16(c->k_pool) ||
+                  !aligned16(c->v_pool)))
+    return fail(QSA_ERR_INVALID_ARG, "k_pool / v_pool NULL or not 16-byte aligned");
+  if (need_side && (c->kidx_pool == nullptr || c->side_pool == nullptr ||
+                    !aligned16(c->kidx_pool) || !aligned16(c->side_pool)))
+    return fail(QSA_ERR_INVALID_ARG, "kidx_pool / side_pool NULL or not 16-byte aligned");
+  return QSA_OK;
+}
+
+qsa_status cuda_status(cudaError_t e, const char *what) {
+  if (e == cudaSuccess) return ok();
+  return fail(QSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+#define QSA_TRY(x)                      \
+  do {                                  \
+    qsa_status _s = (x);                \
+    if (_s != QSA_OK) return _s;        \
+  } while (0)
+
+#define QSA_ERRWORD(var)                                        \
+  cudaError_t _ee;                                              \
+  unsigned *var = device_error_word(&_ee);                      \
+  if (var == nullptr) return cuda_status(_ee, "device error word")
+
+}  // namespace
+
+extern "C" {
+
+int32_t qsa_version(void) { return QSA_VERSION_NUM; }
+
+const char *qsa_last_error(void) { return t_last_error.c_str(); }
+
+qsa_status qsa_append(const qsa_dims *dims, const qsa_cache *cache, int32_t N,
+                      const int32_t *tok_seq, const int32_t *tok_pos, const void *k_new,
+                      const void *v_new, const void *kidx_new, qsa_stream_t stream) {
+  try {
+    QSA_TRY(check_dims(dims));
+    QSA_TRY(check_cache(cache, true, true));
+    if (N < 0) return fail(QSA_ERR_INVALID_ARG, "N < 0");
+    if (N > 0 && (tok_seq == nullptr || tok_pos == nullptr || k_new == nullptr ||
+                  v_new == nullptr || kidx_new == nullptr))
+      return fail(QSA_ERR_INVALID_ARG, "a token array is NULL");
+    if (N > 0 && (!aligned16(k_new) || !aligned16(v_new) || !aligned16(kidx_new)))
+      return fail(QSA_ERR_INVALID_ARG, "k_new / v_new / kidx_new not 16-byte aligned");
+    QSA_ERRWORD(err);
+    return cuda_status(launch_append(*dims, *cache, N, tok_seq, tok_pos, k_new, v_new, kidx_new,
+                                     err, reinterpret_cast<cudaStream_t>(stream)),
+                       "qsa_append launch");
+  } catch (...) {
+    return fail(QSA_ERR_CUDA, "qsa_append: internal exception");
+  }
+}
+
+qsa_status qsa_index_score(const qsa_dims *dims, const qsa_cache *cache, int32_t B,
+                           const int32_t *seq_lens, const void *q_idx, const float *w,
+                           float *scores, int32_t ld_scores, qsa_stream_t stream) {
+  try {
+    QSA_TRY(check_dims(dims));
+    QSA_TRY(check_cache(cache, false, true));
+    if (B < 0 || B > 16384) return fail(QSA_ERR_INVALID_ARG, "B=%d outside [0, 16384]", B);
+    if (B > cache->num_seqs)
+      return fail(QSA_ERR_INVALID_ARG, "B=%d exceeds block_table rows %d", B, cache->num_seqs);
+    if (ld_scores <= 0) return fail(QSA_ERR_INVALID_ARG, "ld_scores must be positive");
+    if (B > 0 && (seq_lens == nullptr || q_idx == nullptr || w == nullptr || scores == nullptr))
+      return fail(QSA_ERR_INVALID_ARG, "an argument array is NULL");
+    if (B > 0 && ((reinterpret_cast<uintptr_t>(q_idx) & 3u) != 0))
+      return fail(QSA_ERR_INVALID_ARG, "q_idx not 4-byte aligned");
+    QSA_ERRWORD(err);
+    return cuda_status(launch_index_score(*dims, *cache, B, seq_lens, q_idx, w, scores, ld_scores,
+                                          err, reinterpret_cast<cudaStream_t>(stream)),
+                       "qsa_index_score launch");
+  } catch (...) {
+    return fail(QSA_ERR_CUDA, "qsa_index_score: internal exception");
+  }
+}
+
+size_t qsa_topk_workspace_size(int32_t B, int32_t ld_scores, int32_t k) {
+  (void)B;
+  (void)ld_scores;
+  (void)k;
+  return 0;
+}
+
+qsa_status qsa_topk_select(int32_t B, const int32_t *seq_lens, const float *scores,
+                           int32_t ld_scores, int32_t k, int32_t *sel, void *ws, size_t ws_bytes,
+                           qsa_stream_t stream) {
+  (void)ws;
+  (void)ws_bytes;
+  try {
+    if (B < 0 || B > 65535) return fail(QSA_ERR_INVALID_ARG, "B=%d outside [0, 65535]", B);
+    if (k < 1 || k > 4096) return fail(QSA_ERR_UNSUPPORTED, "k=%d outside [1, 4096]", k);
+    if (ld_scores <= 0 || ld_scores > TOPK_CLUSTER * TOPK_MAX_KEYS_PER_CTA)
+      return fail(QSA_ERR_UNSUPPORTED, "ld_scores=%d outside [1, %d]", ld_scores,
+                  TOPK_CLUSTER * TOPK_MAX_KEYS_PER_CTA);
+    if (B > 0 && (seq_lens == nullptr || scores == nullptr || sel == nullptr))
+      return fail(QSA_ERR_INVALID_ARG, "an argument array is NULL");
+    QSA_ERRWORD(err);
+    return cuda_status(launch_topk(B, seq_lens, scores, ld_scores, k, sel, err,
+                                   reinterpret_cast<cudaStream_t>(stream)),
+                       "qsa_topk_select launch");
+  } catch (...) {
+    return fail(QSA_ERR_CUDA, "qsa_topk_select: internal exception");
+  }
+}
+
+size_t qsa_sparse_decode_workspace_size(const qsa_dims *dims, int32_t B, int32_t k, int32_t R) {
+  if (dims == nullptr || B <= 0 || k <= 0 || R <= 0 || dims->Hkv <= 0 || dims->Hq <= 0)
+    return 0;
+  return decode_ws_bytes(*dims, B, k, R);
+}
+
+qsa_status qsa_sparse_decode(const qsa_dims *dims, const qsa_cache *cache, int32_t B,
+                             const int32_t *seq_lens, const void *q, const int32_t *sel,
+                             int32_t k, int32_t R, float *o_part, float *lse_part, void *ws,
+                             size_t ws_bytes, qsa_stream_t stream) {
+  try {
+    QSA_TRY(check_dims(dims));
+    QSA_TRY(check_cache(cache, true, false));
+    if (B < 0 || B > 65535) return fail(QSA_ERR_INVALID_ARG, "B=%d outside [0, 65535]", B);
+    if (B > cache->num_seqs)
+      return fail(QSA_ERR_INVALID_ARG, "B=%d exceeds block_table rows %d", B, cache->num_seqs);
+    if (k < 1 || k > 4096) return fail(QSA_ERR_UNSUPPORTED, "k=%d outside [1, 4096]", k);
+    if (R < 1 || R > 64) return fail(QSA_ERR_UNSUPPORTED, "R=%d outside [1, 64]", R);
+    if (B == 0) return ok();
+    if (seq_lens == nullptr || q == nullptr || sel == nullptr || o_part == nullptr ||
+        lse_part == nullptr || ws == nullptr)
+      return fail(QSA_ERR_INVALID_ARG, "an argument array is NULL");
+    if (!aligned16(q) || !aligned16(o_part) || !aligned16(ws))
+      return fail(QSA_ERR_INVALID_ARG, "q / o_part / ws not 16-byte aligned");
+    const size_t need = decode_ws_bytes(*dims, B, k, R);
+    if (ws_bytes < need)
+      return fail(QSA_ERR_INVALID_ARG, "workspace %zu bytes < %zu needed", ws_bytes, need);
+    QSA_ERRWORD(err);
+    return cuda_status(launch_sparse_decode(*dims, *cache, B, seq_lens, q, sel, k, R, o_part,
+                                            lse_part, ws, err,
+                                            reinterpret_cast<cudaStream_t>(stream)),
+                       "qsa_sparse_decode launch");
+  } catch (...) {
+    return fail(QSA_ERR_CUDA, "qsa_sparse_decode: internal exception");
+  }
+}
+
+qsa_status qsa_merge(int32_t R, int32_t B, int32_t Hq, int32_t D, const float *o_part,
+                     const float *lse_part, void *out, int32_t out_is_bf16, float *lse_out,
+                     qsa_stream_t stream) {
+  try {
+    if (R < 1 || R > 64) return fail(QSA_ERR_UNSUPPORTED, "R=%d outside [1, 64]", R);
+    if (B < 0 || Hq <= 0 || D <= 0 || D % 4 != 0)
+      return fail(QSA_ERR_INVALID_ARG, "bad B / Hq / D (D must be a positive multiple of 4)");
+    if ((long long)B * Hq > (1LL << 30)) return fail(QSA_ERR_INVALID_ARG, "B*Hq too large");
+    if (B == 0) return ok();
+    if (o_part == nullptr || lse_part == nullptr || out == nullptr)
+      return fail(QSA_ERR_INVALID_ARG, "an argument array is NULL");
+    if (!aligned16(o_part) || (reinterpret_cast<uintptr_t>(out) & 7u) != 0)
+      return fail(QSA_ERR_INVALID_ARG, "o_part not 16-byte / out not 8-byte aligned");
+    return cuda_status(launch_merge(R, B, Hq, D, o_part, lse_part, out, out_is_bf16, lse_out,
+                                    reinterpret_cast<cudaStream_t>(stream)),
+                       "qsa_merge launch");
+  } catch (...) {
+    return fail(QSA_ERR_CUDA, "qsa_merge: internal exception");
+  }
+}
+
+qsa_status qsa_check_device_errors(qsa_stream_t stream, int32_t *flags) {
+  try {
+    if (flags) *flags = 0;
+    cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_status(e, "stream synchronize");
+    QSA_ERRWORD(err);
+    (void)err;
+    unsigned v = 0;
+    e = cudaMemcpyFromSymbol(&v, g_err_word, sizeof v);
+    if (e != cudaSuccess) return cuda_status(e, "read error word");
+    const unsigned zero = 0;
+    e = cudaMemcpyToSymbol(g_err_word, &zero, sizeof zero);
+    if (e != cudaSuccess) return cuda_status(e, "clear error word");
+    if (flags) *flags = (int32_t)v;
+    if (v & ~ERR_TIMEOUT) return fail(QSA_ERR_BOUNDS, "device index check failed (flags 0x%x)", v);
+    if (v & ERR_TIMEOUT) return fail(QSA_ERR_TIMEOUT, "device wait timed out (flags 0x%x)", v);
+    return ok();
+  } catch (...) {
+    return fail(QSA_ERR_CUDA, "qsa_check_device_errors: internal exception");
+  }
+}
+
+}  // extern "C"

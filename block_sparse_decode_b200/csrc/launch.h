@@ -1,0 +1,41 @@
+// Internal host-side launchers of the QSA kernels (not part of the C ABI).
+// Each returns the cudaError_t of its launch(es); argument checks happen in
+// abi.cu before any of these is called.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/qsa.h"
+
+namespace qsa {
+
+// Device address of this device's error word (set up once per device).
+unsigned *device_error_word(cudaError_t *status);
+int device_sm_count();
+
+cudaError_t launch_append(const qsa_dims &d, const qsa_cache &c, int N, const int32_t *tok_seq,
+                          const int32_t *tok_pos, const void *k_new, const void *v_new,
+                          const void *kidx_new, unsigned *err, cudaStream_t st);
+
+cudaError_t launch_index_score(const qsa_dims &d, const qsa_cache &c, int B,
+                               const int32_t *seq_lens, const void *q_idx, const float *w,
+                               float *scores, int ld, unsigned *err, cudaStream_t st);
+
+constexpr int TOPK_CLUSTER = 8;
+constexpr int TOPK_MAX_KEYS_PER_CTA = 53248;  // 208 KiB of keys per CTA
+cudaError_t launch_topk(int B, const int32_t *seq_lens, const float *scores, int ld, int k,
+                        int32_t *sel, unsigned *err, cudaStream_t st);
+
+int decode_num_slots(int k, int R);
+size_t decode_ws_bytes(const qsa_dims &d, int B, int k, int R);
+cudaError_t launch_sparse_decode(const qsa_dims &d, const qsa_cache &c, int B,
+                                 const int32_t *seq_lens, const void *q, const int32_t *sel,
+                                 int k, int R, float *o_part, float *lse_part, void *ws,
+                                 unsigned *err, cudaStream_t st);
+
+cudaError_t launch_merge(int R, int B, int Hq, int D, const float *o_part, const float *lse_part,
+                         void *out, int out_is_bf16, float *lse_out, cudaStream_t st);
+
+}  // namespace qsa

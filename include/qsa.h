@@ -1,0 +1,211 @@
+/*
+ * qsa.h -- C ABI of the QSA sparse-decode library (libqsa.so), sm_100a.
+ *
+ * The library computes one decode step of Qwen Sparse Attention (QSA) as
+ * described on the page "Qwen 4 QSA gets decode context parallelism: inside
+ * vLLM's draft PR for Qwen3.8-Flash-Next" (orcarouter.ai), section "What the
+ * pull request actually changes": a lightweight indexer compresses keys
+ * into micro-blocks at ratio 4, scores the blocks and keeps the best 512
+ * (about 2,048 token positions); the final softmax and value aggregation run
+ * on the uncompressed K and V. The decode-context-parallel split read of the
+ * same section (each slice of the main KV cache read on its own, the
+ * selector replicated, partial results combined afterwards; also "Questions
+ * worth answering directly", DCP vs TP) is done inside one GPU as an R-way
+ * split with a log-sum-exp merge.
+ *
+ * The page gives no formulas; this library fixes these readings:
+ *   micro-block key   kc = bf16_rne(fp32 sum of its n keys in token order / n)
+ *                     (n = 4, or L mod 4 for the trailing partial block)
+ *   block score       s_b = sum_h w_h * max(0, q_idx_h . kc_b)
+ *   selection         k_b = min(k, nb) blocks by (score desc, index asc),
+ *                     listed in ascending block order, padded with -1
+ *   slice r of R      blocks [floor(r*nb/R), floor((r+1)*nb/R))
+ *   partial r         z_t = scale * q_h . K_t over tokens t < L of the
+ *                     selected blocks of slice r; LSE_r = ln sum exp z_t;
+ *                     O_r = sum softmax(z)_t V_t; empty slice: O_r = 0,
+ *                     LSE_r = -inf
+ *   merge             O = sum_r e^(LSE_r-m) O_r / sum_r e^(LSE_r-m),
+ *                     LSE = m + ln sum_r e^(LSE_r-m), m = max_r LSE_r
+ *
+ * Conventions for every call:
+ *   - All array pointers are DEVICE pointers owned by the caller. The library
+ *     allocates no device memory and keeps no pointer after a call returns
+ *     (the caller owns every cache view; nothing is kept alive behind its
+ *     back).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream). A returned QSA_OK means the launch was accepted.
+ *   - Arrays are dense row-major with the shapes given below; bf16 arrays and
+ *     pools must be 16-byte aligned.
+ *   - Indices are int32. K, V, queries and indexer keys are bf16; weights,
+ *     scores, partial outputs and LSEs are fp32 (LSE in natural log).
+ *   - Data-dependent indices (block-table entries, sequence lengths, token
+ *     positions, selected block ids) are bounds-checked on the device. A
+ *     failed check skips the access and sets a bit in the device error word,
+ *     which qsa_check_device_errors() reads and clears (QSA_ERR_BOUNDS).
+ *     No kernel traps or asserts.
+ *   - No C++ exception crosses this boundary. On a non-OK status,
+ *     qsa_last_error() gives a message (thread-local).
+ */
+#ifndef QSA_H
+#define QSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t qsa_status;
+#define QSA_OK 0
+#define QSA_ERR_INVALID_ARG 1 /* null pointer, bad size or alignment          */
+#define QSA_ERR_UNSUPPORTED 2 /* dims outside the supported set               */
+#define QSA_ERR_CUDA 3        /* a CUDA runtime call or a launch failed       */
+#define QSA_ERR_BOUNDS 4      /* a device-side index check failed             */
+#define QSA_ERR_TIMEOUT 5     /* a bounded device-side wait gave up           */
+
+/* Same object as cudaStream_t. */
+typedef struct CUstream_st *qsa_stream_t;
+
+/* Head geometry.
+ *   Hq query heads share Hkv KV heads; query head h reads KV head h / (Hq/Hkv).
+ *   D   head dim of q, K and V            supported: 128
+ *   Hi  indexer heads                     supported: 1..32
+ *   di  indexer key width                 supported: 64, 128
+ *   P   tokens per cache page             supported: multiple of 4, 4..1024
+ *   G = Hq/Hkv                            supported: 1..8
+ *   scale  softmax scale applied to q.K (e.g. 1/sqrt(D)). */
+typedef struct qsa_dims {
+  int32_t Hq, Hkv, D, Hi, di, P;
+  float scale;
+} qsa_dims;
+
+/* The paged cache. ONE block table indexes all four pools, so the selector
+ * state and the main KV cache can never disagree about where a token lives
+ * (the page's "selector and the main KV cache are kept in one cache group").
+ *   k_pool, v_pool  bf16 [num_pages, P, Hkv, D]   token (page, slot), head g
+ *   kidx_pool       bf16 [num_pages, P, di]       per-token indexer key
+ *   side_pool       bf16 [num_pages, P/4, di]     compressed key of each
+ *                                                 complete micro-block
+ *   block_table     int32 [num_seqs, max_pages_per_seq]: physical page of
+ *                   tokens [j*P, (j+1)*P) of sequence b is block_table[b][j].
+ * A contiguous cache is the same structure with an identity block table. */
+typedef struct qsa_cache {
+  void *k_pool;
+  void *v_pool;
+  void *kidx_pool;
+  void *side_pool;
+  const int32_t *block_table;
+  int32_t num_seqs;
+  int32_t max_pages_per_seq;
+  int32_t num_pages;
+} qsa_cache;
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int32_t qsa_version(void);
+
+/* Message of the last non-OK status returned on this thread ("" if none). */
+const char *qsa_last_error(void);
+
+/* Write N new tokens into the cache (page section "What the pull request
+ * actually changes": QSA keeps the main cache plus the indexer's side
+ * caches; the fourth bullet: synthetic batches must not write the side
+ * caches).
+ *   tok_seq, tok_pos  int32 [N]: sequence row and position of each token;
+ *                     an entry with tok_seq < 0 or tok_pos < 0 is padding and
+ *                     writes nothing at all.
+ *   k_new, v_new      bf16 [N, Hkv, D];  kidx_new  bf16 [N, di].
+ * Token i goes to page block_table[seq][pos / P], slot pos % P of k/v/kidx
+ * pools. After all N tokens are written (a second launch on the same
+ * stream), every token with pos % 4 == 3 stores the compressed key of its
+ * micro-block (positions pos-3..pos, read back from kidx_pool) at side slot
+ * (pos % P) / 4 of the same page. So a bulk prefill in any token order gives
+ * the same side cache as one token per call. Two entries with the same
+ * (seq, pos) in one call race (undefined which one lands). */
+qsa_status qsa_append(const qsa_dims *dims, const qsa_cache *cache, int32_t N,
+                      const int32_t *tok_seq, const int32_t *tok_pos,
+                      const void *k_new, const void *v_new,
+                      const void *kidx_new, qsa_stream_t stream);
+
+/* Block scores of B sequences (page section "What the pull request actually
+ * changes": the indexer "scores them").
+ *   seq_lens  int32 [B]: L_b, context length after the current token was
+ *             appended; nb_b = ceil(L_b / 4) blocks are scored. Reads
+ *             block_table rows 0..B-1.
+ *   q_idx     bf16 [B, Hi, di];  w  fp32 [B, Hi]
+ *   scores    fp32 [B, ld_scores], ld_scores >= max_b nb_b (a longer
+ *             sequence sets QSA_ERR_BOUNDS and is skipped). Entries
+ *             j >= nb_b are not written.
+ * Complete blocks read the side pool; the trailing partial block's key is
+ * built from its L mod 4 tokens in kidx_pool by the same rule. */
+qsa_status qsa_index_score(const qsa_dims *dims, const qsa_cache *cache,
+                           int32_t B, const int32_t *seq_lens,
+                           const void *q_idx, const float *w, float *scores,
+                           int32_t ld_scores, qsa_stream_t stream);
+
+/* Scratch bytes qsa_topk_select needs (0 for this implementation). */
+size_t qsa_topk_workspace_size(int32_t B, int32_t ld_scores, int32_t k);
+
+/* Per-sequence top-k blocks (page section "What the pull request actually
+ * changes": "keeps the best 512 blocks").
+ *   scores  fp32 [B, ld_scores] (first nb_b = ceil(seq_lens[b]/4) entries
+ *           used; NaN scores are not supported)
+ *   sel     int32 [B, k]: the k_b = min(k, nb_b) best blocks by (score
+ *           desc, block index asc), in ascending block order, then -1.
+ * -0.0 ranks equal to +0.0. Supported: 1 <= k <= 4096,
+ * ld_scores <= 425,984. ws may be NULL when its size is 0. */
+qsa_status qsa_topk_select(int32_t B, const int32_t *seq_lens,
+                           const float *scores, int32_t ld_scores, int32_t k,
+                           int32_t *sel, void *ws, size_t ws_bytes,
+                           qsa_stream_t stream);
+
+/* Scratch bytes qsa_sparse_decode needs for B sequences, top-k k, R slices.
+ * The scratch holds per-chunk partial results; it needs no initialisation
+ * and is fully rewritten by every call (calls sharing one scratch buffer
+ * must be ordered on the GPU). */
+size_t qsa_sparse_decode_workspace_size(const qsa_dims *dims, int32_t B,
+                                        int32_t k, int32_t R);
+
+/* Split-read sparse attention over the selected blocks (page section "What
+ * the pull request actually changes": exact softmax and value aggregation on
+ * the uncompressed K/V; each slice of the main cache read separately with
+ * the selector replicated, results combined afterwards).
+ *   q         bf16 [B, Hq, D]
+ *   sel       int32 [B, k] as produced by qsa_topk_select (ascending, -1
+ *             padded); the same selection serves all R slices
+ *   o_part    fp32 [R, B, Hq, D];  lse_part  fp32 [R, B, Hq]
+ * Slice r holds the attention of each query head over the tokens t < L_b of
+ * the selected blocks in [floor(r*nb/R), floor((r+1)*nb/R)); an empty slice
+ * gives zeros and LSE = -inf. Supported: 1 <= R <= 64, 1 <= k <= 4096. */
+qsa_status qsa_sparse_decode(const qsa_dims *dims, const qsa_cache *cache,
+                             int32_t B, const int32_t *seq_lens,
+                             const void *q, const int32_t *sel, int32_t k,
+                             int32_t R, float *o_part, float *lse_part,
+                             void *ws, size_t ws_bytes, qsa_stream_t stream);
+
+/* LSE-weighted combine of R partial results (page sections "What the pull
+ * request actually changes", second bullet, and "Questions worth answering
+ * directly": partial attention results are merged afterwards).
+ *   o_part fp32 [R, B, Hq, D], lse_part fp32 [R, B, Hq]
+ *   out    [B, Hq, D], bf16 if out_is_bf16 else fp32;  lse_out fp32 [B, Hq]
+ *          (lse_out may be NULL). Slices with LSE = -inf are ignored; if
+ *          every slice is empty the row is 0 with LSE = -inf. */
+qsa_status qsa_merge(int32_t R, int32_t B, int32_t Hq, int32_t D,
+                     const float *o_part, const float *lse_part, void *out,
+                     int32_t out_is_bf16, float *lse_out, qsa_stream_t stream);
+
+/* Wait for `stream`, then read and clear the device error word of the
+ * current device. *flags receives the bits that were set (0 if none):
+ *   1 sequence row out of range    2 page id out of range
+ *   4 block-table column out of range   8 selected block id out of range
+ *   16 sequence length out of range (negative, or nb > ld_scores)
+ *   32 a bounded wait gave up
+ * Returns QSA_ERR_BOUNDS if any bit below 32 was set, QSA_ERR_TIMEOUT if only
+ * bit 32 was, QSA_OK otherwise. flags may be NULL. */
+qsa_status qsa_check_device_errors(qsa_stream_t stream, int32_t *flags);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QSA_H */

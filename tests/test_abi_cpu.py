@@ -1,0 +1,82 @@
+"""The C-ABI library loads, exports every symbol include/qsa.h declares, and
+rejects bad arguments on the host (no GPU needed: none of these calls reaches
+a CUDA call)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from block_sparse_decode_b200 import build, qsa
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                      "include", "qsa.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return qsa.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(qsa_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_exports():
+    assert declared_functions() == sorted(qsa.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+    out = os.popen(f"nm -D --defined-only {qsa.LIB_PATH}").read()
+    for name in declared_functions():
+        assert re.search(rf"\bT {name}\b", out), f"{name} not exported"
+
+
+def test_version_and_workspace_sizes(L):
+    assert qsa.qsa_version() == 100
+    assert qsa.qsa_topk_workspace_size(8, 65536, 512) == 0
+    d = qsa.QsaDims(32, 4, 128, 16, 128, 64, 0.088)
+    # (ceil(512/32) + 4) slots x 4 kv heads x 8 heads x (128 + 1) floats per sequence
+    assert qsa.qsa_sparse_decode_workspace_size(d, 8, 512, 4) == 8 * 20 * 4 * 8 * 129 * 4
+
+
+def _status(fn, *args):
+    return fn(*args)
+
+
+def test_host_side_argument_checks(L):
+    D = qsa._Dims
+    bad = [
+        D(32, 4, 64, 16, 128, 64, 0.1),    # D != 128
+        D(32, 5, 128, 16, 128, 64, 0.1),   # Hq % Hkv
+        D(32, 4, 128, 16, 96, 64, 0.1),    # di
+        D(32, 4, 128, 33, 128, 64, 0.1),   # Hi > 32
+        D(32, 2, 128, 16, 128, 64, 0.1),   # G = 16 > 8
+        D(32, 4, 128, 16, 128, 62, 0.1),   # P % 4
+    ]
+    c = qsa._Cache(16, 16, 16, 16, 16, 1, 1, 1)
+    for d in bad:
+        st = L.qsa_index_score(ctypes.byref(d), ctypes.byref(c), 1, 16, 16, 16, 16, 4, None)
+        assert st in (qsa.QSA_ERR_UNSUPPORTED, qsa.QSA_ERR_INVALID_ARG)
+        assert L.qsa_last_error().decode()
+    ok = D(32, 4, 128, 16, 128, 64, 0.1)
+    assert L.qsa_index_score(None, ctypes.byref(c), 1, 16, 16, 16, 16, 4, None) == \
+        qsa.QSA_ERR_INVALID_ARG
+    assert L.qsa_topk_select(1, 16, 16, 100, 0, 16, None, 0, None) == qsa.QSA_ERR_UNSUPPORTED
+    assert L.qsa_topk_select(1, 16, 16, 1 << 30, 8, 16, None, 0, None) == \
+        qsa.QSA_ERR_UNSUPPORTED
+    assert L.qsa_merge(0, 1, 1, 128, 16, 16, 16, 1, None, None) == qsa.QSA_ERR_UNSUPPORTED
+    assert L.qsa_merge(2, 1, 1, 126, 16, 16, 16, 1, None, None) == qsa.QSA_ERR_INVALID_ARG
+    assert L.qsa_sparse_decode(ctypes.byref(ok), ctypes.byref(c), 1, 16, 16, 16, 8, 0, 16, 16,
+                               16, 1 << 20, None) == qsa.QSA_ERR_UNSUPPORTED
+    assert L.qsa_append(ctypes.byref(ok), ctypes.byref(c), -1, 16, 16, 16, 16, 16, None) == \
+        qsa.QSA_ERR_INVALID_ARG
+    unaligned = qsa._Cache(17, 16, 16, 16, 16, 1, 1, 1)
+    assert L.qsa_append(ctypes.byref(ok), ctypes.byref(unaligned), 1, 16, 16, 16, 16, 16,
+                        None) == qsa.QSA_ERR_INVALID_ARG

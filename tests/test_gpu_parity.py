@@ -1,0 +1,355 @@
+"""Parity of the CUDA library (through its C ABI) with the CPU oracle.
+
+Bars: side cache, pool bytes and top-k indices bit-exact (top-k compared on
+the GPU's own fp32 scores, so both sides decide in the same precision);
+scores within the bound of tests/gpu_harness.score_tolerance; selection equal
+to the oracle's up to the near-tie band; attention, recomputed by the oracle
+over the GPU's own selection, within max abs 1e-2 and rel-L2 5e-3, LSE within
+1e-3.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from block_sparse_decode_b200 import qsa
+from synth import make_custom, make_workload, step_queries
+from synth.workloads import DIMS_FULL, Dims
+from tests.gpu_harness import GpuRun, oracle_sequence, score_tolerance, token_index
+from tests.helpers import bits, check_attention, check_selection
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def _check_seq(run, b, L=None, q=None, q_idx=None, w=None, full=True):
+    wl, k, R = run.wl, run.k, run.R
+    L = wl.seq_lens[b] if L is None else L
+    nb = (L + 3) // 4
+    ref = oracle_sequence(wl, b, L, q, q_idx, w, k=k, R=R)
+    K, V, X = wl.seq_tokens(b, L)
+    # side cache: bit-exact against the one-shot build
+    assert np.array_equal(run.side_rows(b, L), oracle.side_cache(bits(X), L)), f"side b={b}"
+    # scores
+    s_gpu = run.buf.scores[b, :nb].double().cpu().numpy()
+    tol = score_tolerance(wl, b, L, q_idx, w)
+    err = np.abs(s_gpu - ref["scores"])
+    assert np.all(err <= tol), f"scores b={b}: worst {err.max():.3e} at {int(err.argmax())}"
+    # top-k: exact on the GPU's scores; oracle's own selection up to ties
+    sel_gpu = run.buf.sel[b].cpu().numpy()
+    assert np.array_equal(sel_gpu, oracle.topk_blocks(s_gpu, k)), f"top-k b={b}"
+    check_selection(sel_gpu, ref["sel"], ref["scores"], k, what=f"sel b={b}")
+    if not full:
+        return
+    # attention over the GPU's own selection
+    ref2 = oracle_sequence(wl, b, L, q, q_idx, w, k=k, R=R, sel=sel_gpu)
+    check_attention(run.buf.o_part[:, b].cpu().numpy(), run.buf.lse_part[:, b].cpu().numpy(),
+                    ref2["O_part"], ref2["LSE_part"], what=f"partials b={b}")
+    check_attention(run.buf.out[b].float().cpu().numpy(), run.buf.lse[b].cpu().numpy(),
+                    ref2["O"], ref2["LSE"], what=f"merged b={b}")
+
+
+# ------------------------------------------------------------ small cases
+
+@pytest.mark.parametrize("R", [2, 1, 3, 8])
+def test_tiny_preset_end_to_end(R):
+    wl = make_workload(1, device=DEV)
+    run = GpuRun(wl, R=R)
+    run.step()
+    for b in range(wl.B):
+        _check_seq(run, b)
+        assert set(wl.needles[b]) <= set(run.buf.sel[b].tolist())
+
+
+@pytest.mark.parametrize("R", [1, 2, 4, 8])
+def test_ragged_paged_full_heads(R):
+    lens = [1, 2, 3, 4, 5, 63, 64, 65, 2047, 2048, 2049, 2051, 4099, 9001, 20000]
+    wl = make_custom(DIMS_FULL, lens, k=512, R=R, seed=101, device=DEV, paged=True)
+    run = GpuRun(wl)
+    run.step()
+    for b in range(wl.B):
+        _check_seq(run, b)
+
+
+@pytest.mark.parametrize("dims,lens,k", [
+    (Dims(Hq=4, Hkv=4, D=128, Hi=5, di=64, P=16, scale=0.11), [77, 1030, 3], 40),
+    (Dims(Hq=12, Hkv=2, D=128, Hi=24, di=128, P=128, scale=0.09), [4096, 515, 6000], 100),
+    (Dims(Hq=2, Hkv=1, D=128, Hi=1, di=128, P=4, scale=0.2), [33, 257], 7),
+    (Dims(Hq=16, Hkv=2, D=128, Hi=32, di=64, P=64, scale=0.088), [1500, 2600], 1),
+])
+def test_other_dims(dims, lens, k):
+    for R in (1, 3):
+        wl = make_custom(dims, lens, k=k, R=R, seed=102, device=DEV, paged=True)
+        run = GpuRun(wl)
+        run.step()
+        for b in range(wl.B):
+            _check_seq(run, b)
+
+
+def test_clustered_selection_leaves_empty_slices():
+    # needles + k small: the selection sits in a few slices, most slices empty
+    d = DIMS_FULL
+    wl = make_custom(d, [8192, 3000], k=4, R=16, seed=103, device=DEV, needles=4)
+    run = GpuRun(wl)
+    run.step()
+    for b in range(wl.B):
+        _check_seq(run, b)
+        assert np.isneginf(run.buf.lse_part[:, b].cpu().numpy()).any()
+
+
+# ------------------------------------------------------------ top-k alone
+
+def _topk_gpu(scores_np, k, lens=None):
+    B, ld = scores_np.shape
+    lens = [4 * ld] * B if lens is None else lens
+    sl = torch.tensor(lens, dtype=torch.int32, device=DEV)
+    sc = torch.from_numpy(np.ascontiguousarray(scores_np, dtype=np.float32)).to(DEV)
+    sel = torch.full((B, k), -7, dtype=torch.int32, device=DEV)
+    qsa.qsa_topk_select(sl, sc, k, sel)
+    assert qsa.qsa_check_device_errors() == 0
+    return sel.cpu().numpy()
+
+
+@pytest.mark.parametrize("case", ["random", "ties", "allzero", "negzero", "negative", "few",
+                                  "heavy"])
+def test_topk_exact(case):
+    g = np.random.default_rng(sum(map(ord, case)))
+    B, ld, k = 6, 70001, 512
+    if case == "random":
+        s = g.standard_normal((B, ld)).astype(np.float32) ** 2
+    elif case == "ties":
+        s = g.integers(0, 40, (B, ld)).astype(np.float32)
+    elif case == "allzero":
+        s = np.zeros((B, ld), np.float32)
+    elif case == "negzero":
+        s = np.where(g.random((B, ld)) < 0.5, -0.0, 0.0).astype(np.float32)
+        s[:, ::97] = 1.0
+    elif case == "negative":
+        s = g.standard_normal((B, ld)).astype(np.float32)
+    elif case == "few":
+        s = g.standard_normal((B, ld)).astype(np.float32)
+    else:  # heavy tail with a block of exact ties at the threshold
+        s = np.exp(3 * g.standard_normal((B, ld))).astype(np.float32)
+        s[:, 1000:3000] = np.float32(np.sort(s[0])[-400])
+    lens = [4 * ld - 3, 4 * ld, 2049, 2048, 4 * 513, 1]
+    if case == "few":
+        lens = [5, 4 * 511 + 1, 4 * 512, 4 * 512 + 1, 4 * 65536, 4 * 70001]
+    got = _topk_gpu(s, k, lens)
+    for b in range(B):
+        nb = (lens[b] + 3) // 4
+        ref = oracle.topk_blocks(s[b, :nb].astype(np.float64), k)
+        assert np.array_equal(got[b], ref), f"{case} b={b} nb={nb}"
+
+
+@pytest.mark.parametrize("k", [1, 2, 255, 256, 1024, 4096])
+def test_topk_k_sweep(k):
+    g = np.random.default_rng(k)
+    s = (g.integers(0, 1000, (3, 30000)) * 0.25).astype(np.float32)
+    lens = [4 * 30000, 4 * 4097 - 2, 4 * k + 4]
+    got = _topk_gpu(s, k, lens)
+    for b in range(3):
+        nb = (lens[b] + 3) // 4
+        assert np.array_equal(got[b], oracle.topk_blocks(s[b, :nb].astype(np.float64), k))
+
+
+# ------------------------------------------------------------ merge alone
+
+@pytest.mark.parametrize("R,out_bf16", [(1, True), (2, False), (5, True), (64, False)])
+def test_merge_matches_oracle(R, out_bf16):
+    g = np.random.default_rng(R)
+    B, Hq, D = 3, 32, 128
+    O = g.standard_normal((R, B, Hq, D)).astype(np.float32)
+    LSE = (3 * g.standard_normal((R, B, Hq))).astype(np.float32)
+    LSE[R // 2, 1, :5] = -np.inf
+    if R > 1:
+        LSE[:, 2, 7] = -np.inf  # a row with every slice empty
+    o_t, l_t = torch.from_numpy(O).to(DEV), torch.from_numpy(LSE).to(DEV)
+    out = torch.empty((B, Hq, D), dtype=torch.bfloat16 if out_bf16 else torch.float32,
+                      device=DEV)
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=DEV)
+    qsa.qsa_merge(o_t, l_t, out, lse)
+    out_np, lse_np = out.float().cpu().numpy(), lse.cpu().numpy()
+    for b in range(B):
+        Om, Lm = oracle.merge_partials(O[:, b].astype(np.float64), LSE[:, b].astype(np.float64))
+        check_attention(out_np[b], lse_np[b], Om, Lm, what=f"merge b={b}")
+
+
+# ------------------------------------------------------------ append alone
+
+def test_append_pools_bit_exact():
+    d = Dims(Hq=8, Hkv=4, D=128, Hi=4, di=128, P=16, scale=0.1)
+    lens = [259, 64, 3, 100]
+    wl = make_custom(d, lens, k=8, R=1, seed=104, device=DEV, paged=True, pool_slack_pages=3)
+    cache = qsa.alloc_cache(qsa.QsaDims.of(d), wl.num_pages, wl.block_table, device=DEV)
+    for t in (cache.k_pool, cache.v_pool, cache.kidx_pool, cache.side_pool):
+        t.view(torch.int16).random_(-32768, 32767)
+    host = [bits(t).copy() for t in (cache.k_pool, cache.v_pool, cache.kidx_pool,
+                                     cache.side_pool)]
+    seq, pos = token_index(wl)
+    perm = np.random.default_rng(0).permutation(len(seq))
+    seq, pos = seq[perm], pos[perm]
+    pos[::17] = -1  # padding entries
+    seq[5::23] = -1
+    rows = torch.from_numpy(perm).to(DEV)
+    kn, vn, xn = wl.k_tok[rows].contiguous(), wl.v_tok[rows].contiguous(), \
+        wl.kidx_tok[rows].contiguous()
+    qsa.qsa_append(qsa.QsaDims.of(d), cache, torch.from_numpy(seq).to(DEV),
+                   torch.from_numpy(pos).to(DEV), kn, vn, xn)
+    assert qsa.qsa_check_device_errors() == 0
+    oracle.append_paged(*host, wl.block_table.cpu().numpy(), d.P, seq, pos, bits(kn), bits(vn),
+                        bits(xn))
+    for got, want, name in zip((cache.k_pool, cache.v_pool, cache.kidx_pool, cache.side_pool),
+                               host, ("k", "v", "kidx", "side")):
+        assert np.array_equal(bits(got), want), f"{name} pool differs"
+
+
+def test_append_incremental_equals_bulk_side_cache():
+    d = DIMS_FULL
+    lens = [515, 64, 7]
+    wl = make_custom(d, lens, k=8, R=1, seed=105, device=DEV, paged=True)
+    run = GpuRun(wl, prefill=[0] * 3)  # nothing written in bulk
+    for t in range(max(lens)):
+        live = [b for b in range(3) if t < lens[b]]
+        rows = torch.tensor([wl.tok_off[b] + t for b in live], device=DEV)
+        qsa.qsa_append(run.dims, run.cache, torch.tensor(live, dtype=torch.int32, device=DEV),
+                       torch.full((len(live),), t, dtype=torch.int32, device=DEV),
+                       wl.k_tok[rows].contiguous(), wl.v_tok[rows].contiguous(),
+                       wl.kidx_tok[rows].contiguous())
+    assert qsa.qsa_check_device_errors() == 0
+    for b, L in enumerate(lens):
+        _, _, X = wl.seq_tokens(b, L)
+        assert np.array_equal(run.side_rows(b, L), oracle.side_cache(bits(X), L))
+
+
+# ------------------------------------------------------------ error paths
+
+def test_bad_page_ids_are_flagged_not_faulted():
+    wl = make_custom(DIMS_FULL, [3000, 900], k=64, R=2, seed=106, device=DEV)
+    run = GpuRun(wl)
+    bad = run.cache.block_table.clone()
+    run.cache.block_table[0, 3] = wl.num_pages + 1000   # out-of-range page id
+    run.cache.block_table[1, 1] = -5
+    with pytest.raises(qsa.QsaError) as ei:
+        run.step(append=False)
+    assert ei.value.status == qsa.QSA_ERR_BOUNDS
+    run.cache.block_table.copy_(bad)
+    run.step()  # the context is still healthy
+    _check_seq(run, 0)
+
+
+def test_seq_len_beyond_score_row_is_flagged():
+    wl = make_custom(DIMS_FULL, [3000, 900], k=64, R=1, seed=107, device=DEV)
+    run = GpuRun(wl)
+    sc = torch.zeros((2, 100), dtype=torch.float32, device=DEV)  # ld too short for seq 0
+    qsa.qsa_index_score(run.dims, run.cache, run.seq_lens, wl.q_idx, wl.w, sc)
+    with pytest.raises(qsa.QsaError) as ei:
+        qsa.qsa_check_device_errors()
+    assert ei.value.status == qsa.QSA_ERR_BOUNDS
+
+
+def test_invalid_arguments_rejected_on_host():
+    wl = make_custom(DIMS_FULL, [100], k=8, R=1, seed=108, device=DEV)
+    run = GpuRun(wl)
+    with pytest.raises(qsa.QsaError) as ei:
+        qsa.qsa_sparse_decode(run.dims, run.cache, run.seq_lens, wl.q, run.buf.sel, 8, 65,
+                              run.buf.o_part, run.buf.lse_part, run.buf.ws)
+    assert ei.value.status == qsa.QSA_ERR_UNSUPPORTED
+    small_ws = torch.empty(16, dtype=torch.uint8, device=DEV)
+    with pytest.raises(qsa.QsaError) as ei:
+        qsa.qsa_sparse_decode(run.dims, run.cache, run.seq_lens, wl.q, run.buf.sel, 8, 1,
+                              run.buf.o_part, run.buf.lse_part, small_ws)
+    assert ei.value.status == qsa.QSA_ERR_INVALID_ARG
+
+
+def test_empty_batch_is_a_no_op():
+    d = qsa.QsaDims.of(DIMS_FULL)
+    bt = torch.zeros((1, 1), dtype=torch.int32, device=DEV)
+    cache = qsa.alloc_cache(d, 1, bt, device=DEV)
+    buf = qsa.alloc_step(d, 1, 4, 8, 1, device=DEV)
+    e = torch.empty(0, dtype=torch.int32, device=DEV)
+    qsa.qsa_index_score(d, cache, e, buf.out[:0], buf.lse[:0], buf.scores[:0])
+    qsa.qsa_topk_select(e, buf.scores[:0], 8, buf.sel[:0])
+    qsa.qsa_merge(buf.o_part[:, :0], buf.lse_part[:, :0], buf.out[:0], buf.lse[:0])
+    assert qsa.qsa_check_device_errors() == 0
+
+
+# ------------------------------------------------------------ full-size presets
+
+def _sampled(wl, n):
+    B = wl.B
+    idx = sorted({0, B - 1, *np.random.default_rng(wl.seed).choice(B, size=min(n, B),
+                                                                   replace=False).tolist()})
+    return idx
+
+
+def test_preset2_full_size():
+    wl = make_workload(2, device=DEV)
+    run = GpuRun(wl)
+    run.step()
+    for b in _sampled(wl, 3):
+        _check_seq(run, b)
+    del run, wl
+    torch.cuda.empty_cache()
+
+
+def test_preset3_full_size_split_equals_unsplit():
+    wl = make_workload(3, device=DEV)
+    run = GpuRun(wl)
+    run.step()
+    for b in _sampled(wl, 2):
+        _check_seq(run, b)
+        assert set(wl.needles[b]) <= set(run.buf.sel[b].tolist())
+    out4, lse4 = run.buf.out.float().clone(), run.buf.lse.clone()
+    sel4 = run.buf.sel.clone()
+    run.R = 1
+    run.buf = qsa.alloc_step(run.dims, wl.B, run.ld, run.k, 1, device=DEV)
+    run.step(append=False)
+    assert torch.equal(run.buf.sel, sel4)
+    d = (run.buf.out.float() - out4).abs().max().item()
+    assert d <= 1e-2 and (run.buf.lse - lse4).abs().max().item() <= 1e-3
+    del run, wl
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("R", [1, 2, 4, 8])
+def test_preset4_ragged_full_size(R):
+    wl = make_workload(4, device=DEV)
+    run = GpuRun(wl, R=R)
+    run.step()
+    lens = np.array(wl.seq_lens)
+    pick = {int(lens.argmin()), int(lens.argmax())}
+    for res in (1, 2, 3):
+        pick.add(int(np.nonzero(lens % 4 == res)[0][0]))
+    pick.add(int(np.nonzero(lens < 2048)[0][0]))
+    for b in sorted(pick):
+        _check_seq(run, b, full=(R in (1, 8)) or b == min(pick))
+    del run, wl
+    torch.cuda.empty_cache()
+
+
+def test_preset5_append_steps():
+    wl = make_workload(5, device=DEV)
+    spec_prefill, steps = wl.extra["prefill"], wl.extra["steps"]
+    for k in (256, 512, 1024):
+        run = GpuRun(wl, k=k, prefill=[spec_prefill] * wl.B)
+        for t in range(steps):
+            lens = [spec_prefill + t + 1] * wl.B
+            q, q_idx, w = step_queries(wl, t)
+            run.step(q=q, q_idx=q_idx, w=w, lens=lens)
+            if t in (0, 3, steps - 1):
+                for b in (0, 77):
+                    _check_seq(run, b, L=lens[0], q=q[b], q_idx=q_idx[b], w=w[b],
+                               full=(k == 512 or t == steps - 1))
+        if k != 1024:
+            del run
+            torch.cuda.empty_cache()
+    # after the 64 incremental steps, every sequence's side cache equals the
+    # oracle's one-shot rebuild from its tokens
+    L = spec_prefill + steps
+    for b in range(wl.B):
+        _, _, X = wl.seq_tokens(b, L)
+        assert np.array_equal(run.side_rows(b, L), oracle.side_cache(bits(X), L)), b
