@@ -46,6 +46,16 @@ def exact_bf16(values) -> np.ndarray:
     return bits(b)
 
 
+def bf16_same(a, b) -> bool:
+    """Bit-equal bf16 arrays, except that any two NaNs count as equal (a NaN's
+    payload depends on the hardware's NaN propagation, not on the method)."""
+    a = np.asarray(a, dtype=np.uint16)
+    b = np.asarray(b, dtype=np.uint16)
+    nan_a = (a & 0x7FFF) > 0x7F80
+    nan_b = (b & 0x7FFF) > 0x7F80
+    return bool(np.array_equal(nan_a, nan_b) and np.array_equal(a[~nan_a], b[~nan_b]))
+
+
 def rel_l2(a, b) -> float:
     a = np.asarray(a, dtype=np.float64)
     b = np.asarray(b, dtype=np.float64)

@@ -19,7 +19,7 @@ from block_sparse_decode_b200 import qsa
 from synth import make_custom, make_workload, step_queries
 from synth.workloads import DIMS_FULL, Dims
 from tests.gpu_harness import GpuRun, oracle_sequence, score_tolerance, token_index
-from tests.helpers import bits, check_attention, check_selection
+from tests.helpers import bf16_same, bits, check_attention, check_selection
 
 pytestmark = pytest.mark.gpu
 
@@ -204,7 +204,9 @@ def test_append_pools_bit_exact():
                         bits(xn))
     for got, want, name in zip((cache.k_pool, cache.v_pool, cache.kidx_pool, cache.side_pool),
                                host, ("k", "v", "kidx", "side")):
-        assert np.array_equal(bits(got), want), f"{name} pool differs"
+        # the poisoned pools hold NaN patterns; sums over them give NaN whose
+        # payload is hardware-specific
+        assert bf16_same(bits(got), want), f"{name} pool differs"
 
 
 def test_append_incremental_equals_bulk_side_cache():
