@@ -337,7 +337,7 @@ def run_ours(args, rank, world, local_rank):
             "gbs": (side_b + kv_b) / ((mean_parts[1] + mean_parts[3]) / 1e3) / 1e9,
             "frac": (side_b + kv_b) / ((mean_parts[1] + mean_parts[3]) / 1e3) / 1e9 / peak},
         "step_roofline_frac": (side_b + kv_b) / (ms_per_step / 1e3) / 1e9 / peak,
-        "gpu_launches": 7 * args.steps,
+        "gpu_launches": 5 * args.steps,
         "clocks": clk.summary(),
         "e2e": e2e,
     }

@@ -7,13 +7,15 @@
 // at ratio 4; synthetic batches must not write the side caches (padding
 // entries here write nothing at all).
 //
-// Two launches on one stream: the first writes K, V and the per-token indexer
-// key of every token (one warp per token, 16-byte stores); the second, for
-// every token with pos % 4 == 3, reads the block's 4 indexer keys back from
-// the pool and writes their mean. The split makes a bulk prefill (tokens of
-// a block written by the same call, in any order) give the same side cache
-// as one token per call. Traffic is a few KiB per token; these kernels are
-// launch-bound in decode.
+// Two phases: the first writes K, V and the per-token indexer key of every
+// token (one warp per token, 16-byte stores); the second, for every token
+// with pos % 4 == 3, reads the block's 4 indexer keys back from the pool and
+// writes their mean. Ordering the phases makes a bulk prefill (tokens of a
+// block written by the same call, in any order) give the same side cache as
+// one token per call. Up to 128 tokens (decode: one per sequence) both phases
+// run in one CTA separated by a barrier, one launch; larger calls use two
+// launches on the stream. Traffic is a few KiB per token; decode appends are
+// latency-bound.
 #include "common.cuh"
 #include "launch.h"
 
@@ -52,10 +54,8 @@ __device__ __forceinline__ int locate(const AppendArgs &a, int s, int p, int lan
   return page;
 }
 
-__global__ void __launch_bounds__(256) append_tokens_kernel(AppendArgs a) {
-  const int tok = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (tok >= a.N) return;
+// Phase 1 for one token (one warp): K, V and indexer key into the pools.
+__device__ __forceinline__ void write_token(const AppendArgs &a, int tok, int lane) {
   const int s = a.tok_seq[tok], p = a.tok_pos[tok];
   if (s < 0 || p < 0) return;  // padding / synthetic entry: no write anywhere
   const int page = locate(a, s, p, lane);
@@ -74,10 +74,9 @@ __global__ void __launch_bounds__(256) append_tokens_kernel(AppendArgs a) {
   for (int i = lane; i < a.x_vec; i += 32) xd[i] = xs[i];
 }
 
-__global__ void __launch_bounds__(256) append_compress_kernel(AppendArgs a) {
-  const int tok = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (tok >= a.N) return;
+// Phase 2 for one token (one warp): if it closes a micro-block, store the
+// block's compressed key in the side pool.
+__device__ __forceinline__ void compress_block(const AppendArgs &a, int tok, int lane) {
   const int s = a.tok_seq[tok], p = a.tok_pos[tok];
   if (s < 0 || p < 0 || (p & 3) != 3) return;
   const int page = locate(a, s, p, 32);  // errors were flagged by the first launch
@@ -95,6 +94,27 @@ __global__ void __launch_bounds__(256) append_compress_kernel(AppendArgs a) {
     float hi = __fadd_rn(__fadd_rn(__fadd_rn(bf16hi(v0), bf16hi(v1)), bf16hi(v2)), bf16hi(v3));
     out[e] = pack_bf16x2(__fdiv_rn(lo, 4.0f), __fdiv_rn(hi, 4.0f));
   }
+}
+
+__global__ void __launch_bounds__(256) append_tokens_kernel(AppendArgs a) {
+  const int tok = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (tok < a.N) write_token(a, tok, threadIdx.x & 31);
+}
+
+__global__ void __launch_bounds__(256) append_compress_kernel(AppendArgs a) {
+  const int tok = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (tok < a.N) compress_block(a, tok, threadIdx.x & 31);
+}
+
+// Both phases in one CTA (small N, e.g. one token per sequence in decode):
+// the barrier orders every phase-1 write before any phase-2 read.
+constexpr int SMALL_WARPS = 32;
+constexpr int SMALL_MAX_N = 4 * SMALL_WARPS;
+__global__ void __launch_bounds__(SMALL_WARPS * 32) append_small_kernel(AppendArgs a) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int tok = warp; tok < a.N; tok += SMALL_WARPS) write_token(a, tok, lane);
+  __syncthreads();
+  for (int tok = warp; tok < a.N; tok += SMALL_WARPS) compress_block(a, tok, lane);
 }
 
 }  // namespace
@@ -123,6 +143,10 @@ cudaError_t launch_append(const qsa_dims &d, const qsa_cache &c, int N, const in
   a.x_vec = d.di / 8;
   a.di = d.di;
   a.err = err;
+  if (N <= SMALL_MAX_N) {
+    append_small_kernel<<<1, SMALL_WARPS * 32, 0, st>>>(a);
+    return cudaGetLastError();
+  }
   const int threads = 256, per_block = threads / 32;
   const int blocks = (N + per_block - 1) / per_block;
   append_tokens_kernel<<<blocks, threads, 0, st>>>(a);

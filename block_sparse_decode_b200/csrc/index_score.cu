@@ -56,12 +56,14 @@ __global__ void __launch_bounds__(SC_WARPS * 32, 2) index_score_kernel(ScoreArgs
   constexpr int TILEB = SC_ROWS * ROWB;   // bytes per warp tile
   constexpr int KS = DI / 16;             // mma k-steps
   extern __shared__ __align__(128) unsigned char smem[];
-  int *prefix = reinterpret_cast<int *>(smem);                          // [B + 1]
-  unsigned char *tiles = smem + (((a.B + 1) * 4 + 127) & ~127);
+  int *prefix = reinterpret_cast<int *>(smem);  // [B + 1] tiles before sequence b
+  int *lens = prefix + (a.B + 1);               // [B] sequence lengths
+  unsigned char *tiles = smem + (((2 * a.B + 1) * 4 + 127) & ~127);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   // ---- per-CTA prefix of tiles per sequence
   __shared__ int carry;
+  __shared__ int wsum[SC_WARPS];
   if (threadIdx.x == 0) { carry = 0; prefix[0] = 0; }
   __syncthreads();
   for (int base = 0; base < a.B; base += blockDim.x) {
@@ -72,7 +74,9 @@ __global__ void __launch_bounds__(SC_WARPS * 32, 2) index_score_kernel(ScoreArgs
       if (L < 0 || nb > a.ld) {
         if (blockIdx.x == 0) raise_err(a.err, ERR_LEN);
         nb = 0;
+        L = 0;
       }
+      lens[b] = L;
       n = (nb + SC_ROWS - 1) / SC_ROWS;
     }
     int x = n;  // inclusive warp scan
@@ -81,7 +85,6 @@ __global__ void __launch_bounds__(SC_WARPS * 32, 2) index_score_kernel(ScoreArgs
       int y = __shfl_up_sync(0xffffffffu, x, o);
       if (lane >= o) x += y;
     }
-    __shared__ int wsum[SC_WARPS];
     if (lane == 31) wsum[warp] = x;
     __syncthreads();
     int off = carry;
@@ -95,63 +98,74 @@ __global__ void __launch_bounds__(SC_WARPS * 32, 2) index_score_kernel(ScoreArgs
 
   unsigned char *ring = tiles + warp * (SC_STAGES * TILEB);
   const uint32_t ring_s = smem_u32(ring);
-  const int gwarp = blockIdx.x * SC_WARPS + warp, nwarps = gridDim.x * SC_WARPS;
+  // contiguous tile range per warp: consecutive tiles stay in one sequence
+  const int nwarps = gridDim.x * SC_WARPS, gwarp = blockIdx.x * SC_WARPS + warp;
+  const int t_begin = (int)(((long long)gwarp * total) / nwarps);
+  const int t_end = (int)(((long long)(gwarp + 1) * total) / nwarps);
   const int rows_per_page = a.P >> 2;
+  const int32_t *bt_all = a.block_table;
 
-  // Issue the cp.async copies of tile t into ring stage st (complete blocks only).
-  auto issue = [&](int t, int st) {
+  // Page of row (lane & 15) of tile t: one independent load per lane, issued a
+  // tile ahead of its use. -1: no complete block there; -2: bounds error.
+  auto lookup = [&](int t) -> int {
+    if (t >= t_end) return -1;
     const int b = find_seq(prefix, a.B, t);
-    const int j0 = (t - prefix[b]) * SC_ROWS;
-    const int nfull = a.seq_lens[b] >> 2;
-    const int32_t *bt = a.block_table + (size_t)b * a.max_pages;
+    const int j = (t - prefix[b]) * SC_ROWS + (lane & 15);
+    if (j >= (lens[b] >> 2)) return -1;
+    const int col = j / rows_per_page;
+    if (col >= a.max_pages) return -2;
+    const int page = __ldg(bt_all + (size_t)b * a.max_pages + col);
+    return (page >= 0 && page < a.num_pages) ? page : -3;
+  };
+  // cp.async of tile t into stage st, given each row's page (from lookup()).
+  auto issue = [&](int t, int st, int pg) {
+    if (t >= t_end) return;
+    const int j0 = (t - prefix[find_seq(prefix, a.B, t)]) * SC_ROWS;
+    if (lane < 16 && pg < -1) raise_err(a.err, pg == -2 ? ERR_BT : ERR_PAGE);
 #pragma unroll
     for (int i = 0; i < SC_ROWS * CH / 32; ++i) {
       const int q = lane + 32 * i, r = q / CH, c = q % CH;
+      const int page = __shfl_sync(0xffffffffu, pg, r);
+      if (page == -1) continue;
       const int j = j0 + r;
-      if (j >= nfull) continue;
-      const int col = j / rows_per_page;
       const __nv_bfloat16 *src = a.side_pool;
       int bytes = 0;
-      if (col < a.max_pages) {
-        const int page = bt[col];
-        if (page >= 0 && page < a.num_pages) {
-          src = a.side_pool + ((size_t)page * rows_per_page + (j - col * rows_per_page)) * DI + c * 8;
-          bytes = 16;
-        } else if (c == 0) {
-          raise_err(a.err, ERR_PAGE);
-        }
-      } else if (c == 0) {
-        raise_err(a.err, ERR_BT);
+      if (page >= 0) {
+        src = a.side_pool + ((size_t)page * rows_per_page + (j % rows_per_page)) * DI + c * 8;
+        bytes = 16;
       }
       cp_async16(ring_s + st * TILEB + swz(r, c, ROWB), src, bytes);
     }
   };
 
+  // prologue: pages of the first STAGES tiles, copies of the first STAGES-1
+  int pg_next[SC_STAGES];
+#pragma unroll
+  for (int i = 0; i < SC_STAGES; ++i) pg_next[i] = lookup(t_begin + i);
+#pragma unroll
   for (int i = 0; i < SC_STAGES - 1; ++i) {
-    const int t = gwarp + i * nwarps;
-    if (t < total) issue(t, i);
+    issue(t_begin + i, i, pg_next[i]);
     cp_async_commit();
   }
+  int pg_ahead = pg_next[SC_STAGES - 1];  // pages of tile it + STAGES - 1
 
   uint32_t qf[NT][KS][2];
   float wv[NT][2];
   int qb = -1;
 
   for (int it = 0;; ++it) {
-    const int t = gwarp + it * nwarps;
-    if (t >= total) break;
-    {
-      const int tn = gwarp + (it + SC_STAGES - 1) * nwarps;
-      if (tn < total) issue(tn, (it + SC_STAGES - 1) % SC_STAGES);
-      cp_async_commit();
-    }
+    const int t = t_begin + it;
+    if (t >= t_end) break;
+    issue(t + SC_STAGES - 1, (it + SC_STAGES - 1) % SC_STAGES, pg_ahead);
+    cp_async_commit();
+    pg_ahead = lookup(t + SC_STAGES);  // consumed by the next iteration
     cp_async_wait<SC_STAGES - 1>();
     __syncwarp();
 
     const int st = it % SC_STAGES;
     const int b = find_seq(prefix, a.B, t);
     const int j0 = (t - prefix[b]) * SC_ROWS;
-    const int L = a.seq_lens[b];
+    const int L = lens[b];
     const int nfull = L >> 2, nb = (L + 3) >> 2;
     unsigned char *tile = ring + st * TILEB;
 
@@ -181,7 +195,7 @@ __global__ void __launch_bounds__(SC_WARPS * 32, 2) index_score_kernel(ScoreArgs
       const int n = L - 4 * nfull, pos = 4 * nfull;
       const int col = pos / a.P;
       int page = -1;
-      if (col < a.max_pages) page = a.block_table[(size_t)b * a.max_pages + col];
+      if (col < a.max_pages) page = bt_all[(size_t)b * a.max_pages + col];
       const bool ok = page >= 0 && page < a.num_pages;
       if (!ok && lane == 0) raise_err(a.err, col < a.max_pages ? ERR_PAGE : ERR_BT);
       const uint32_t *x = reinterpret_cast<const uint32_t *>(a.kidx_pool) +
@@ -243,7 +257,7 @@ __global__ void __launch_bounds__(SC_WARPS * 32, 2) index_score_kernel(ScoreArgs
 
 template <int DI, int NT>
 cudaError_t launch_t(const ScoreArgs &a, cudaStream_t st) {
-  const size_t smem = (((size_t)(a.B + 1) * 4 + 127) & ~(size_t)127) +
+  const size_t smem = (((size_t)(2 * a.B + 1) * 4 + 127) & ~(size_t)127) +
                       (size_t)SC_WARPS * SC_STAGES * SC_ROWS * DI * 2;
   auto kern = index_score_kernel<DI, NT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -260,6 +274,8 @@ cudaError_t launch_index_score(const qsa_dims &d, const qsa_cache &c, int B,
                                const int32_t *seq_lens, const void *q_idx, const float *w,
                                float *scores, int ld, unsigned *err, cudaStream_t st) {
   if (B == 0) return cudaSuccess;
+  if (index_score_tc_supported(d))
+    return launch_index_score_tc(d, c, B, seq_lens, q_idx, w, scores, ld, err, st);
   ScoreArgs a;
   a.side_pool = static_cast<const __nv_bfloat16 *>(c.side_pool);
   a.kidx_pool = static_cast<const __nv_bfloat16 *>(c.kidx_pool);

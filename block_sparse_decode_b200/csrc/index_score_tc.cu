@@ -1,0 +1,550 @@
+// qsa_index_score on 5th-generation tensor cores: TMA-staged side-cache
+// tiles, tcgen05.mma into TMEM, and an epilogue that reads the accumulators
+// back with tcgen05.ld.
+//
+// Page "Qwen 4 QSA gets decode context parallelism" (orcarouter.ai), section
+// "What the pull request actually changes": the indexer scores the
+// micro-blocks. Score of block b: s_b = sum_h w_h * max(0, q_idx_h . kc_b)
+// (this library's reading; the page prints no formula).
+//
+// Why this shape: the contraction is [blocks x di] . [di x Hi], 8 MAC per
+// side-cache byte at di = 128, Hi = 16. At HBM speed that is ~50 TMAC/s,
+// past fp32 CUDA cores, and a warp-level MMA loop spends hundreds of
+// instructions per 4 KiB on address math and copies. Here one thread issues
+// the copies (TMA, 2 KiB per page half) and one thread issues the MMAs, so
+// the instruction cost per byte is tiny and the kernel runs at copy speed.
+//
+// Tile = 128 consecutive blocks of one sequence (MMA M = 128), K = di, N = 16
+// (or 32) indexer heads. The side pool is addressed through a 3-D tensor map
+// (di, rows of a page, page): each page's rows land in shared memory in the
+// 128-byte-swizzled K-major layout the MMA descriptors expect; the block
+// table supplies the page coordinates. The indexer query of the tile's
+// sequence is a second TMA load (2-D map over [B*Hi, di]).
+//
+// CTA = 6 warps, persistent over the flattened (sequence, tile) list:
+//   warp 0     producer: page lookups, expect-tx, TMA loads into a ring of
+//              stages (full/empty mbarriers)
+//   warp 1     TMEM owner; lane 0 issues tcgen05.mma (K/16 per tile) into one
+//              of two TMEM accumulators and commits to the stage's empty
+//              barrier and the accumulator's full barrier
+//   warps 2-5  epilogue: tcgen05.ld of 32 rows x N columns each, ReLU, head
+//              weights, one coalesced fp32 store per block; the trailing
+//              partial block (key built from its L mod 4 indexer keys) is
+//              scored on CUDA cores by the warp that owns its row.
+// Every mbarrier wait is bounded: on timeout the kernel sets the TIMEOUT bit,
+// stops all roles, drains what it issued (bounded) and frees TMEM.
+//
+// Supported here: P a power of two in [32, 1024], so a page's P/4 rows are a
+// multiple of 8 (every TMA box starts on a 1 KiB swizzle atom) and pages
+// tile the 128-row tile exactly; di in {64, 128}; Hi <= 32.
+// Roofline: HBM-bound; algorithmic bytes = nb * di * 2 per sequence.
+#include <cuda.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "launch.h"
+#include "umma_desc.h"
+
+namespace qsa {
+namespace {
+
+constexpr int TC_M = 128;                 // blocks per tile (MMA M)
+constexpr int TC_MAX_STAGES = 8;
+constexpr int TC_EPI_WARPS = 4;
+constexpr int TC_THREADS = 32 * (2 + TC_EPI_WARPS);
+constexpr uint32_t TC_SPIN_LIMIT = 1u << 22;  // try_wait rounds before giving up
+constexpr uint32_t TC_DRAIN_LIMIT = 1u << 20;
+
+struct TcArgs {
+  const __nv_bfloat16 *kidx_pool, *q_idx;
+  const float *w;
+  const int32_t *block_table, *seq_lens;
+  float *scores;
+  int B, ld, P, rpp, box_rows, max_pages, num_pages, Hi, stages;
+  unsigned *err;
+};
+
+struct TcCtrl {
+  uint64_t full[TC_MAX_STAGES];
+  uint64_t empty[TC_MAX_STAGES];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint32_t tmem_base;
+  int abort_flag;
+  int issued;    // tiles the producer issued
+  int consumed;  // tiles the MMA warp consumed
+  int mma_done;  // tiles the epilogue finished
+};
+
+// ------------------------------------------------------------ PTX helpers
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.b32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait; on timeout (or if another role already gave up) returns false.
+// The drain after an abort passes honor_abort = false: it must wait for its
+// own copies and MMAs even though the flag is already up.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                          unsigned *err, uint32_t limit = TC_SPIN_LIMIT,
+                                          bool honor_abort = true) {
+  for (uint32_t i = 0; i < limit; ++i) {
+    if (mbar_try(bar, parity)) return true;
+    if (honor_abort && (i & 255u) == 255u && *abort_flag) return false;
+  }
+  *abort_flag = 1;
+  raise_err(err, ERR_TIMEOUT);
+  return false;
+}
+__device__ __forceinline__ void mbar_arrive_expect(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, uint32_t bar,
+                                            int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(map), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar,
+                                            int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(map), "r"(bar), "r"(c0), "r"(c1)
+      : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(tmem_d),
+      "l"(da), "l"(db), "r"(idesc), "r"(accumulate));
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+__device__ __forceinline__ void tc_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ int tc_find_seq(const int *prefix, int B, int t) {
+  int lo = 0, hi = B - 1;
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (prefix[mid] <= t) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// Score of the trailing partial block of sequence b (whole warp; lane 0 gets it).
+template <int DI>
+__device__ float partial_block_score(const TcArgs &a, int b, int L, bool *ok_out) {
+  const int lane = threadIdx.x & 31;
+  const int nfull = L >> 2, n = L - 4 * nfull, pos = 4 * nfull;
+  const int col = pos / a.P;
+  int page = -1;
+  if (col < a.max_pages) page = a.block_table[(size_t)b * a.max_pages + col];
+  const bool ok = page >= 0 && page < a.num_pages;
+  *ok_out = ok;
+  if (!ok) {
+    if (lane == 0) raise_err(a.err, col < a.max_pages ? ERR_PAGE : ERR_BT);
+    return 0.f;
+  }
+  const uint32_t *x = reinterpret_cast<const uint32_t *>(a.kidx_pool) +
+                      ((size_t)page * a.P + pos % a.P) * (DI / 2);
+  float klo[DI / 64], khi[DI / 64];
+#pragma unroll
+  for (int i = 0; i < DI / 64; ++i) {
+    const int e = lane + 32 * i;
+    uint32_t v = x[e];
+    float lo = bf16lo(v), hi = bf16hi(v);
+    for (int u = 1; u < n; ++u) {
+      v = x[u * (DI / 2) + e];
+      lo = __fadd_rn(lo, bf16lo(v));
+      hi = __fadd_rn(hi, bf16hi(v));
+    }
+    // the block key is the bf16-rounded mean, exactly as the side cache holds it
+    const uint32_t kc = pack_bf16x2(__fdiv_rn(lo, (float)n), __fdiv_rn(hi, (float)n));
+    klo[i] = bf16lo(kc);
+    khi[i] = bf16hi(kc);
+  }
+  float score = 0.f;
+  for (int h = 0; h < a.Hi; ++h) {
+    const uint32_t *qrow = reinterpret_cast<const uint32_t *>(a.q_idx + ((size_t)b * a.Hi + h) * DI);
+    float part = 0.f;
+#pragma unroll
+    for (int i = 0; i < DI / 64; ++i) {
+      const uint32_t q = qrow[lane + 32 * i];
+      part = fmaf(klo[i], bf16lo(q), part);
+      part = fmaf(khi[i], bf16hi(q), part);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    score = fmaf(a.w[(size_t)b * a.Hi + h], fmaxf(part, 0.f), score);
+  }
+  return score;
+}
+
+template <int DI, int N>
+__global__ void __launch_bounds__(TC_THREADS, 1)
+    index_score_tc_kernel(const __grid_constant__ CUtensorMap side_map,
+                          const __grid_constant__ CUtensorMap q_map, TcArgs a) {
+  constexpr int KH = DI / 64;                 // 128-byte K halves
+  constexpr int A_HALF = TC_M * 128;          // bytes of one A half (128 rows)
+  constexpr int B_HALF = N * 128;             // bytes of one B half (N rows)
+  constexpr int STAGE = KH * (A_HALF + B_HALF);
+  constexpr int KSTEPS = DI / 16;
+  constexpr uint32_t IDESC = f16_idesc(TC_M, N);
+
+  extern __shared__ unsigned char smem_raw[];
+  __shared__ TcCtrl ctl;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int S = a.stages;
+
+  // dynamic smem: [pad to 1024][stages][prefix B+1][lens B]
+  const uint32_t raw_s = smem_u32(smem_raw);
+  const uint32_t pad = (1024u - (raw_s & 1023u)) & 1023u;
+  const uint32_t ring_s = raw_s + pad;
+  int *prefix = reinterpret_cast<int *>(smem_raw + pad + (size_t)S * STAGE);
+  int *lens = prefix + (a.B + 1);
+
+  // ---- per-CTA tile prefix over sequences
+  __shared__ int carry;
+  __shared__ int wsum[TC_THREADS / 32];
+  if (threadIdx.x == 0) {
+    carry = 0;
+    prefix[0] = 0;
+    ctl.abort_flag = 0;
+    ctl.issued = ctl.consumed = ctl.mma_done = 0;
+  }
+  __syncthreads();
+  for (int base = 0; base < a.B; base += TC_THREADS) {
+    const int b = base + threadIdx.x;
+    int n = 0;
+    if (b < a.B) {
+      int L = a.seq_lens[b];
+      int nb = L < 0 ? 0 : (L + 3) >> 2;
+      if (L < 0 || nb > a.ld) {
+        if (blockIdx.x == 0) raise_err(a.err, ERR_LEN);
+        nb = 0;
+        L = 0;
+      }
+      lens[b] = L;
+      n = (nb + TC_M - 1) / TC_M;
+    }
+    int x = n;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) wsum[warp] = x;
+    __syncthreads();
+    int off = carry;
+    for (int i = 0; i < warp; ++i) off += wsum[i];
+    if (b < a.B) prefix[b + 1] = off + x;
+    __syncthreads();
+    if (threadIdx.x == TC_THREADS - 1) carry = off + x;
+    __syncthreads();
+  }
+  const int total = prefix[a.B];
+
+  const uint32_t full0 = smem_u32(&ctl.full[0]), empty0 = smem_u32(&ctl.empty[0]);
+  const uint32_t tfull0 = smem_u32(&ctl.tfull[0]), tempty0 = smem_u32(&ctl.tempty[0]);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(tfull0 + 8 * i, 1);
+      mbar_init(tempty0 + 8 * i, TC_EPI_WARPS * 32);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {  // TMEM: two accumulators of N fp32 columns (64 columns allocated)
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&ctl.tmem_base)),
+                 "r"(64)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl.tmem_base;
+  volatile int *abort_flag = &ctl.abort_flag;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    int s = 0;
+    uint32_t ph = 0;
+    int issued = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+      if (!mbar_wait(empty0 + 8 * s, ph ^ 1u, abort_flag, a.err)) break;
+      const int b = tc_find_seq(prefix, a.B, t);
+      const int j0 = (t - prefix[b]) * TC_M;
+      const int nfull = lens[b] >> 2;
+      const int rows = max(0, min(TC_M, nfull - j0));        // complete blocks in the tile
+      const int nbox = (rows + a.box_rows - 1) / a.box_rows;  // page boxes to load
+      int page = -1, rip = 0;
+      bool ok = false;
+      if (lane < nbox) {
+        const int j = j0 + lane * a.box_rows;
+        const int col = j / a.rpp;
+        rip = j - col * a.rpp;
+        if (col < a.max_pages) {
+          page = __ldg(a.block_table + (size_t)b * a.max_pages + col);
+          ok = page >= 0 && page < a.num_pages;
+          if (!ok) raise_err(a.err, ERR_PAGE);
+        } else {
+          raise_err(a.err, ERR_BT);
+        }
+      }
+      const unsigned okmask = __ballot_sync(0xffffffffu, ok);
+      const uint32_t stage_s = ring_s + (uint32_t)s * STAGE;
+      const uint32_t bar = full0 + 8 * s;
+      if (lane == 0)
+        mbar_arrive_expect(bar, (uint32_t)(__popc(okmask) * a.box_rows * 128 * KH + B_HALF * KH));
+      __syncwarp();
+      if (ok) {
+#pragma unroll
+        for (int h = 0; h < KH; ++h)
+          tma_load_3d(stage_s + h * A_HALF + lane * a.box_rows * 128, &side_map, bar, h * 64, rip,
+                      page);
+      }
+      if (lane == 0) {
+#pragma unroll
+        for (int h = 0; h < KH; ++h)
+          tma_load_2d(stage_s + KH * A_HALF + h * B_HALF, &q_map, bar, h * 64, b * a.Hi);
+      }
+      ++issued;
+      if (++s == S) { s = 0; ph ^= 1u; }
+    }
+    if (lane == 0) ctl.issued = issued;
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int s = 0, acc = 0;
+      uint32_t ph = 0, aph = 0;
+      int consumed = 0;
+      for (int t = blockIdx.x; t < total; t += gridDim.x) {
+        if (!mbar_wait(tempty0 + 8 * acc, aph ^ 1u, abort_flag, a.err)) break;
+        if (!mbar_wait(full0 + 8 * s, ph, abort_flag, a.err)) break;
+        tc_fence_after();
+        const uint32_t stage_s = ring_s + (uint32_t)s * STAGE;
+        const uint32_t d = tmem + (uint32_t)(acc * 32);
+#pragma unroll
+        for (int ks = 0; ks < KSTEPS; ++ks) {
+          const int h = ks >> 2, kk = (ks & 3) * 32;
+          const uint64_t da = sw128_desc(stage_s + h * A_HALF + kk);
+          const uint64_t db = sw128_desc(stage_s + KH * A_HALF + h * B_HALF + kk);
+          tc_mma(d, da, db, IDESC, ks > 0 ? 1u : 0u);
+        }
+        tc_commit(empty0 + 8 * s);
+        tc_commit(tfull0 + 8 * acc);
+        ++consumed;
+        if (++s == S) { s = 0; ph ^= 1u; }
+        if (++acc == 2) { acc = 0; aph ^= 1u; }
+      }
+      ctl.consumed = consumed;
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    int acc = 0;
+    uint32_t aph = 0;
+    int done = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+      const int b = tc_find_seq(prefix, a.B, t);
+      const int j0 = (t - prefix[b]) * TC_M;
+      const int L = lens[b];
+      const int nfull = L >> 2, nb = (L + 3) >> 2;
+      if (!mbar_wait(tfull0 + 8 * acc, aph, abort_flag, a.err)) break;
+      tc_fence_after();
+      float v[16];
+      float score = 0.f;
+      const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * 32);
+      tc_ld16(taddr, v);
+#pragma unroll
+      for (int h = 0; h < 16; ++h)
+        if (h < a.Hi) score = fmaf(__ldg(a.w + (size_t)b * a.Hi + h), fmaxf(v[h], 0.f), score);
+      if (N == 32) {
+        tc_ld16(taddr + 16, v);
+#pragma unroll
+        for (int h = 0; h < 16; ++h)
+          if (h + 16 < a.Hi)
+            score = fmaf(__ldg(a.w + (size_t)b * a.Hi + 16 + h), fmaxf(v[h], 0.f), score);
+      }
+      tc_fence_before();
+      mbar_arrive(tempty0 + 8 * acc);  // accumulator may be overwritten
+      const int j = j0 + q * 32 + lane;
+      if (j < nfull) a.scores[(size_t)b * a.ld + j] = score;
+      if (nfull < nb && nfull >= j0 + q * 32 && nfull < j0 + q * 32 + 32) {
+        bool ok;
+        const float sp = partial_block_score<DI>(a, b, L, &ok);
+        if (lane == 0 && ok) a.scores[(size_t)b * a.ld + nfull] = sp;
+      }
+      ++done;
+      if (++acc == 2) { acc = 0; aph ^= 1u; }
+    }
+    if (threadIdx.x == 64) ctl.mma_done = done;
+  }
+
+  __syncthreads();
+  if (ctl.abort_flag) {
+    // drain: TMA loads issued but never consumed, MMAs issued but never read
+    if (threadIdx.x == 0) {
+      for (int i = ctl.consumed; i < ctl.issued; ++i)
+        mbar_wait(full0 + 8 * (i % S), (uint32_t)((i / S) & 1), abort_flag, a.err,
+                  TC_DRAIN_LIMIT, false);
+    }
+    if (threadIdx.x == 32) {
+      for (int i = ctl.mma_done; i < ctl.consumed; ++i)
+        mbar_wait(tfull0 + 8 * (i & 1), (uint32_t)((i >> 1) & 1), abort_flag, a.err,
+                  TC_DRAIN_LIMIT, false);
+    }
+    __syncthreads();
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(64)
+                 : "memory");
+  }
+}
+
+// ------------------------------------------------------------ host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn(cudaError_t *status) {
+  static EncodeTiledFn fn = nullptr;
+  static cudaError_t st = cudaSuccess;
+  static bool done = false;
+  if (!done) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    st = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+    if (st == cudaSuccess && q != cudaDriverEntryPointSuccess) st = cudaErrorNotSupported;
+    fn = reinterpret_cast<EncodeTiledFn>(p);
+    done = true;
+  }
+  *status = st;
+  return fn;
+}
+
+template <int DI, int N>
+cudaError_t launch_tc_t(const qsa_dims &d, const qsa_cache &c, const TcArgs &a0, cudaStream_t st) {
+  cudaError_t e;
+  EncodeTiledFn enc = encode_fn(&e);
+  if (e != cudaSuccess || enc == nullptr) return e != cudaSuccess ? e : cudaErrorNotSupported;
+  TcArgs a = a0;
+  CUtensorMap side_map, q_map;
+  {
+    const cuuint64_t dims[3] = {(cuuint64_t)DI, (cuuint64_t)a.rpp, (cuuint64_t)c.num_pages};
+    const cuuint64_t strides[2] = {(cuuint64_t)DI * 2, (cuuint64_t)a.rpp * DI * 2};
+    const cuuint32_t box[3] = {64u, (cuuint32_t)a.box_rows, 1u};
+    const cuuint32_t estr[3] = {1u, 1u, 1u};
+    if (enc(&side_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, c.side_pool, dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)DI, (cuuint64_t)a.B * d.Hi};
+    const cuuint64_t strides[1] = {(cuuint64_t)DI * 2};
+    const cuuint32_t box[2] = {64u, (cuuint32_t)N};
+    const cuuint32_t estr[2] = {1u, 1u};
+    if (enc(&q_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<__nv_bfloat16 *>(a.q_idx),
+            dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  constexpr int KH = DI / 64;
+  constexpr size_t STAGE = (size_t)KH * (TC_M * 128 + N * 128);
+  const size_t meta = (size_t)(2 * a.B + 1) * 4;
+  const size_t budget = 227 * 1024 - 1024 - meta - 1024;  // dynamic smem limit, pad, slack
+  int stages = (int)std::min<size_t>(6, budget / STAGE);
+  if (stages < 2) return cudaErrorInvalidValue;
+  a.stages = stages;
+  const size_t smem = 1024 + (size_t)stages * STAGE + meta;
+  auto kern = index_score_tc_kernel<DI, N>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const long long tiles_bound = (long long)a.B * ((a.ld + TC_M - 1) / TC_M);
+  const int grid = (int)std::max<long long>(1, std::min<long long>(device_sm_count(), tiles_bound));
+  kern<<<grid, TC_THREADS, smem, st>>>(side_map, q_map, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool index_score_tc_supported(const qsa_dims &d) {
+  const bool pow2 = d.P >= 32 && d.P <= 1024 && (d.P & (d.P - 1)) == 0;
+  return pow2 && (d.di == 64 || d.di == 128) && d.Hi <= 32;
+}
+
+cudaError_t launch_index_score_tc(const qsa_dims &d, const qsa_cache &c, int B,
+                                  const int32_t *seq_lens, const void *q_idx, const float *w,
+                                  float *scores, int ld, unsigned *err, cudaStream_t st) {
+  if (B == 0) return cudaSuccess;
+  TcArgs a;
+  a.kidx_pool = static_cast<const __nv_bfloat16 *>(c.kidx_pool);
+  a.q_idx = static_cast<const __nv_bfloat16 *>(q_idx);
+  a.w = w;
+  a.block_table = c.block_table;
+  a.seq_lens = seq_lens;
+  a.scores = scores;
+  a.B = B;
+  a.ld = ld;
+  a.P = d.P;
+  a.rpp = d.P / 4;
+  a.box_rows = std::min(a.rpp, TC_M);
+  a.max_pages = c.max_pages_per_seq;
+  a.num_pages = c.num_pages;
+  a.Hi = d.Hi;
+  a.stages = 2;
+  a.err = err;
+  if (d.di == 128) return d.Hi <= 16 ? launch_tc_t<128, 16>(d, c, a, st) : launch_tc_t<128, 32>(d, c, a, st);
+  return d.Hi <= 16 ? launch_tc_t<64, 16>(d, c, a, st) : launch_tc_t<64, 32>(d, c, a, st);
+}
+
+}  // namespace qsa

@@ -14,15 +14,17 @@
 // blocks. A CTA = (chunk slot, KV head, sequence); the slot count per
 // (sequence, KV head) is ceil(k / DC_BLOCKS) + R, an upper bound on the
 // chunks over all slices, so the grid is fixed on the host while the chunk
-// boundaries are found on the device. Each warp gathers 8 blocks (32 tokens
+// boundaries are found on the device. Each warp gathers 4 blocks (16 tokens
 // x 256 B of K and of V for its KV head) with 16-byte cp.async into swizzled
 // shared memory, then runs S^T = K Q^T and O^T += V^T P^T on tensor cores
 // (m16n8k16: the 16 MMA rows are tokens / head dims, the 8 columns are the
 // GQA group's query heads, so no MMA row is wasted) with an online softmax
 // in fp32 (exp2 domain). P^T moves from the accumulator layout to the B
 // operand layout with movmatrix. The warps of a CTA merge through shared
-// memory; a second small kernel merges the chunks of each slice into the
-// R partials.
+// memory into one chunk partial (scratch, L2-resident); the CTA that
+// finishes a slice last (per-slice arrival counter, zeroed by the call)
+// merges that slice's chunks into its R partial. Slot 0 of each (sequence,
+// KV head) writes the empty slices. One kernel launch plus a small memset.
 //
 // Roofline: HBM-bound; algorithmic bytes = tokens * Hkv * D * 2 * 2 per
 // sequence (each selected token's K and V rows read once).
@@ -33,12 +35,13 @@ namespace qsa {
 namespace {
 
 constexpr int DC_WARPS = 4;
-constexpr int DC_BPW = 8;                       // blocks per warp
+constexpr int DC_BPW = 4;                       // blocks per warp (one 16-token MMA tile)
 constexpr int DC_BLOCKS = DC_WARPS * DC_BPW;    // blocks per CTA chunk
 constexpr int DC_D = 128;                       // head dim
 constexpr int DC_ROWB = DC_D * 2;               // bytes per K/V row
 constexpr int DC_TOK = DC_BPW * 4;              // token rows per warp
 constexpr int DC_WARP_SMEM = 2 * DC_TOK * DC_ROWB;  // K + V tiles per warp
+constexpr int DC_SEL_SMEM = 1024;               // selection entries staged in smem
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 
@@ -46,6 +49,7 @@ struct DecodeArgs {
   const __nv_bfloat16 *k_pool, *v_pool, *q;
   const int32_t *block_table, *seq_lens, *sel;
   float *ws_o, *ws_lse;      // [B, Hkv, nslots, G, D], [B, Hkv, nslots, G]
+  unsigned *ws_cnt;          // [B, Hkv, R] chunks of each slice finished so far
   float *o_part, *lse_part;  // [R, B, Hq, D], [R, B, Hq]
   int B, Hq, Hkv, G, P, max_pages, num_pages, k, R, nslots;
   float scale_log2;
@@ -62,73 +66,89 @@ __device__ __forceinline__ int lower_bound(const int32_t *s, int n, int v) {
   return lo;
 }
 
-// Chunk layout of one sequence, computed by one full warp: for slice r, its
-// selection run starts at `start` and holds `count` blocks; its chunks use
-// slots [slot0, slot0 + ceil(count / DC_BLOCKS)). Returns the values for the
-// slice `want_r`, or locates the slice holding slot `want_slot`.
-struct SliceInfo {
-  int r, start, count, slot0, nchunks;
+// Chunk layout of one sequence, computed by one full warp. Lane l holds
+// slices l and l + 32: the run of slice r in the selection list starts at
+// st and holds ct blocks; its ch = ceil(ct / DC_BLOCKS) chunks use slots
+// [ex, ex + ch) (slots are numbered slice after slice).
+struct SliceTable {
+  int st[2], ct[2], ch[2], ex[2];
 };
 
-__device__ SliceInfo slice_info(const DecodeArgs &a, int b, int want_r, int want_slot) {
+// `s` is the sequence's selection row (ascending, first kb = min(k, nb) valid).
+__device__ SliceTable slice_table(const DecodeArgs &a, int b, const int32_t *s) {
   const int lane = threadIdx.x & 31;
   const int L = a.seq_lens[b];
   const int nb = L <= 0 ? 0 : (L + 3) >> 2;
   const int kb = min(a.k, nb);
-  const int32_t *s = a.sel + (size_t)b * a.k;
-  int st[2], ct[2], ch[2];
+  SliceTable t;
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     const int r = lane + 32 * h;
-    st[h] = ct[h] = ch[h] = 0;
+    t.st[h] = t.ct[h] = t.ch[h] = 0;
     if (r < a.R) {
       const int lo = (int)(((long long)r * nb) / a.R);
       const int hi = (int)(((long long)(r + 1) * nb) / a.R);
-      st[h] = lower_bound(s, kb, lo);
-      ct[h] = lower_bound(s, kb, hi) - st[h];
-      ch[h] = (ct[h] + DC_BLOCKS - 1) / DC_BLOCKS;
+      t.st[h] = lower_bound(s, kb, lo);
+      t.ct[h] = lower_bound(s, kb, hi) - t.st[h];
+      t.ch[h] = (t.ct[h] + DC_BLOCKS - 1) / DC_BLOCKS;
     }
   }
-  int inc0 = ch[0], inc1 = ch[1];
+  int inc0 = t.ch[0], inc1 = t.ch[1];
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     int y0 = __shfl_up_sync(0xffffffffu, inc0, o), y1 = __shfl_up_sync(0xffffffffu, inc1, o);
     if (lane >= o) { inc0 += y0; inc1 += y1; }
   }
   inc1 += __shfl_sync(0xffffffffu, inc0, 31);
-  const int ex0 = inc0 - ch[0], ex1 = inc1 - ch[1];
+  t.ex[0] = inc0 - t.ch[0];
+  t.ex[1] = inc1 - t.ch[1];
+  return t;
+}
+
+struct SliceInfo {
+  int r, start, count, slot0, nchunks;
+};
+
+// The slice holding chunk slot `slot` (r = -1 if the slot is unused).
+__device__ SliceInfo slice_of_slot(const SliceTable &t, int R, int slot) {
+  const int lane = threadIdx.x & 31;
   SliceInfo out{-1, 0, 0, 0, 0};
-  unsigned hit0, hit1;
-  if (want_r >= 0) {
-    hit0 = __ballot_sync(0xffffffffu, lane == want_r);
-    hit1 = __ballot_sync(0xffffffffu, lane + 32 == want_r);
-  } else {
-    hit0 = __ballot_sync(0xffffffffu, lane < a.R && ch[0] > 0 && want_slot >= ex0 &&
-                                          want_slot < ex0 + ch[0]);
-    hit1 = __ballot_sync(0xffffffffu, lane + 32 < a.R && ch[1] > 0 && want_slot >= ex1 &&
-                                          want_slot < ex1 + ch[1]);
-  }
-  const int h = hit0 ? 0 : (hit1 ? 1 : -1);
-  if (h >= 0) {
-    const int src = __ffs(h == 0 ? hit0 : hit1) - 1;
-    out.r = src + 32 * h;
-    out.start = __shfl_sync(0xffffffffu, h == 0 ? st[0] : st[1], src);
-    out.count = __shfl_sync(0xffffffffu, h == 0 ? ct[0] : ct[1], src);
-    out.slot0 = __shfl_sync(0xffffffffu, h == 0 ? ex0 : ex1, src);
-    out.nchunks = __shfl_sync(0xffffffffu, h == 0 ? ch[0] : ch[1], src);
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const unsigned hit = __ballot_sync(0xffffffffu, lane + 32 * h < R && t.ch[h] > 0 &&
+                                                        slot >= t.ex[h] &&
+                                                        slot < t.ex[h] + t.ch[h]);
+    if (hit && out.r < 0) {
+      const int src = __ffs(hit) - 1;
+      out.r = src + 32 * h;
+      out.start = __shfl_sync(0xffffffffu, t.st[h], src);
+      out.count = __shfl_sync(0xffffffffu, t.ct[h], src);
+      out.slot0 = __shfl_sync(0xffffffffu, t.ex[h], src);
+      out.nchunks = __shfl_sync(0xffffffffu, t.ch[h], src);
+    }
   }
   return out;
 }
 
 __global__ void __launch_bounds__(DC_WARPS * 32) sparse_decode_kernel(DecodeArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
-  __shared__ int s_info[3];  // slice r, first selection index, blocks in chunk
+  __shared__ int s_info[5];  // slice r, first selection index, blocks, slot0, chunks
   __shared__ float s_m[DC_WARPS][8], s_l[DC_WARPS][8];
+  __shared__ int s_last;
+  __shared__ int32_t s_sel[DC_SEL_SMEM];
   const int slot = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+  // the selection row, staged once so that the slice searches run in shared memory
+  const int32_t *sel_row = a.sel + (size_t)b * a.k;
+  if (a.k <= DC_SEL_SMEM) {
+    for (int i = threadIdx.x; i < a.k; i += blockDim.x) s_sel[i] = sel_row[i];
+    sel_row = s_sel;
+  }
+  __syncthreads();
   if (warp == 0) {
-    const SliceInfo si = slice_info(a, b, -1, slot);
+    const SliceTable tab = slice_table(a, b, sel_row);
+    const SliceInfo si = slice_of_slot(tab, a.R, slot);
     if (lane == 0) {
       if (si.r < 0) {
         s_info[2] = 0;
@@ -137,6 +157,26 @@ __global__ void __launch_bounds__(DC_WARPS * 32) sparse_decode_kernel(DecodeArgs
         s_info[0] = si.r;
         s_info[1] = si.start + c * DC_BLOCKS;
         s_info[2] = min(DC_BLOCKS, si.count - c * DC_BLOCKS);
+        s_info[3] = si.slot0;
+        s_info[4] = si.nchunks;
+      }
+    }
+    if (slot == 0) {
+      // slices that own no selected block: O_r = 0, LSE_r = -inf
+      if (lane == 0 && g == 0 && a.seq_lens[b] < 0) raise_err(a.err, ERR_LEN);
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        unsigned empty = __ballot_sync(0xffffffffu, lane + 32 * hh < a.R && tab.ch[hh] == 0);
+        while (empty) {
+          const int r = __ffs(empty) - 1 + 32 * hh;
+          empty &= empty - 1;
+          for (int h = 0; h < a.G; ++h) {
+            const size_t row = ((size_t)r * a.B + b) * a.Hq + g * a.G + h;
+            *reinterpret_cast<float4 *>(a.o_part + row * DC_D + lane * 4) =
+                make_float4(0.f, 0.f, 0.f, 0.f);
+            if (lane == 0) a.lse_part[row] = -INFINITY;
+          }
+        }
       }
     }
   }
@@ -147,15 +187,15 @@ __global__ void __launch_bounds__(DC_WARPS * 32) sparse_decode_kernel(DecodeArgs
   const int L = a.seq_lens[b];
   const int nb = (L + 3) >> 2;
 
-  // ---- gather: this warp's blocks [warp*8, warp*8+8) of the chunk
+  // ---- gather: this warp's blocks [warp*DC_BPW, (warp+1)*DC_BPW) of the chunk
   unsigned char *wsm = smem + warp * DC_WARP_SMEM;
   const uint32_t ks_base = smem_u32(wsm), vs_base = ks_base + DC_TOK * DC_ROWB;
-  int my_row0 = 0;       // lane < 8: first pool row of block `lane`
-  unsigned my_bits = 0;  // lane < 8: valid-token bits of that block
+  int my_row0 = 0;       // lane < DC_BPW: first pool row of block `lane`
+  unsigned my_bits = 0;  // lane < DC_BPW: valid-token bits of that block
   if (lane < DC_BPW) {
     const int bi = warp * DC_BPW + lane;
     if (bi < count) {
-      const int j = a.sel[(size_t)b * a.k + first + bi];
+      const int j = sel_row[first + bi];
       if (j < 0 || j >= nb) {
         raise_err(a.err, ERR_SEL);
       } else {
@@ -177,8 +217,8 @@ __global__ void __launch_bounds__(DC_WARPS * 32) sparse_decode_kernel(DecodeArgs
   }
   const unsigned valid =
       __reduce_or_sync(0xffffffffu, lane < DC_BPW ? my_bits << (4 * lane) : 0u);
-  // 32 rows x 16 chunks for K and for V; lane owns chunk (lane & 15) of rows
-  // (lane >> 4) + 2i.
+  // DC_TOK rows x 16 chunks for K and for V; lane owns chunk (lane & 15) of
+  // rows (lane >> 4) + 2i.
   const int chunk = lane & 15;
 #pragma unroll
   for (int i = 0; i < DC_TOK / 2; ++i) {
@@ -313,44 +353,49 @@ __global__ void __launch_bounds__(DC_WARPS * 32) sparse_decode_kernel(DecodeArgs
     const size_t row = (((size_t)b * a.Hkv + g) * a.nslots + slot) * a.G + h;
     float *dst = a.ws_o + row * DC_D + d0;
     const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) dst[e] = acc[e] * inv;
+    *reinterpret_cast<float4 *>(dst) =
+        make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+    *reinterpret_cast<float4 *>(dst + 4) =
+        make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
     if (d0 == 0) a.ws_lse[row] = lsum > 0.f ? (M + log2f(lsum)) * LN2 : -INFINITY;
   }
-}
 
-// One warp per (slice r, KV head g, query head h of the group, sequence b):
-// merge the chunks of slice r into o_part[r, b, g*G + h, :].
-__global__ void __launch_bounds__(256) decode_combine_kernel(DecodeArgs a) {
-  const int r = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const SliceInfo si = slice_info(a, b, r, -1);
-  if (threadIdx.x == 0 && r == 0 && g == 0 && a.seq_lens[b] < 0) raise_err(a.err, ERR_LEN);
-  if (warp >= a.G) return;
-  const int hq = g * a.G + warp;
-  float *dst = a.o_part + (((size_t)r * a.B + b) * a.Hq + hq) * DC_D + lane * 4;
-  float *lse_dst = a.lse_part + ((size_t)r * a.B + b) * a.Hq + hq;
-  const size_t row0 = (((size_t)b * a.Hkv + g) * a.nslots + si.slot0) * a.G + warp;
-  float M = -INFINITY;
-  for (int c = 0; c < si.nchunks; ++c) M = fmaxf(M, a.ws_lse[row0 + (size_t)c * a.G]);
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  float wsum = 0.f;
-  if (M != -INFINITY) {
-    for (int c = 0; c < si.nchunks; ++c) {
-      const size_t row = row0 + (size_t)c * a.G;
-      const float f = __expf(a.ws_lse[row] - M);
-      const float4 v = *reinterpret_cast<const float4 *>(a.ws_o + row * DC_D + lane * 4);
-      acc.x += f * v.x;
-      acc.y += f * v.y;
-      acc.z += f * v.z;
-      acc.w += f * v.w;
-      wsum += f;
-    }
+  // ---- the CTA that finishes slice r last merges its chunks into o_part[r]
+  const int r = s_info[0], slot0 = s_info[3], nchunks = s_info[4];
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const unsigned done = atomicAdd(a.ws_cnt + ((size_t)b * a.Hkv + g) * a.R + r, 1u);
+    s_last = (done + 1u == (unsigned)nchunks);
   }
-  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-  *reinterpret_cast<float4 *>(dst) =
-      make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-  if (lane == 0) *lse_dst = wsum > 0.f ? M + logf(wsum) : -INFINITY;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  if (h < a.G) {
+    const size_t row0 = (((size_t)b * a.Hkv + g) * a.nslots + slot0) * a.G + h;
+    float M = -INFINITY;
+    for (int c = 0; c < nchunks; ++c) M = fmaxf(M, __ldcg(a.ws_lse + row0 + (size_t)c * a.G));
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, wsum = 0.f;
+    if (M != -INFINITY) {
+      for (int c = 0; c < nchunks; ++c) {
+        const size_t rc = row0 + (size_t)c * a.G;
+        const float f = __expf(__ldcg(a.ws_lse + rc) - M);
+        const float4 v0 = __ldcg(reinterpret_cast<const float4 *>(a.ws_o + rc * DC_D + d0));
+        const float4 v1 = __ldcg(reinterpret_cast<const float4 *>(a.ws_o + rc * DC_D + d0 + 4));
+        acc[0] += f * v0.x; acc[1] += f * v0.y; acc[2] += f * v0.z; acc[3] += f * v0.w;
+        acc[4] += f * v1.x; acc[5] += f * v1.y; acc[6] += f * v1.z; acc[7] += f * v1.w;
+        wsum += f;
+      }
+    }
+    const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+    const size_t orow = ((size_t)r * a.B + b) * a.Hq + g * a.G + h;
+    float *o = a.o_part + orow * DC_D + d0;
+    *reinterpret_cast<float4 *>(o) =
+        make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+    *reinterpret_cast<float4 *>(o + 4) =
+        make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
+    if (d0 == 0) a.lse_part[orow] = wsum > 0.f ? M + logf(wsum) : -INFINITY;
+  }
 }
 
 }  // namespace
@@ -359,7 +404,7 @@ int decode_num_slots(int k, int R) { return (k + DC_BLOCKS - 1) / DC_BLOCKS + R;
 
 size_t decode_ws_bytes(const qsa_dims &d, int B, int k, int R) {
   const size_t rows = (size_t)B * d.Hkv * decode_num_slots(k, R) * (d.Hq / d.Hkv);
-  return rows * (DC_D + 1) * sizeof(float);
+  return rows * (DC_D + 1) * sizeof(float) + (size_t)B * d.Hkv * R * sizeof(unsigned);
 }
 
 cudaError_t launch_sparse_decode(const qsa_dims &d, const qsa_cache &c, int B,
@@ -379,6 +424,7 @@ cudaError_t launch_sparse_decode(const qsa_dims &d, const qsa_cache &c, int B,
   const size_t rows = (size_t)B * d.Hkv * a.nslots * a.G;
   a.ws_o = static_cast<float *>(ws);
   a.ws_lse = a.ws_o + rows * DC_D;
+  a.ws_cnt = reinterpret_cast<unsigned *>(a.ws_lse + rows);
   a.o_part = o_part;
   a.lse_part = lse_part;
   a.B = B;
@@ -395,10 +441,9 @@ cudaError_t launch_sparse_decode(const qsa_dims &d, const qsa_cache &c, int B,
   cudaError_t e = cudaFuncSetAttribute(sparse_decode_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  sparse_decode_kernel<<<dim3(a.nslots, d.Hkv, B), DC_WARPS * 32, smem, st>>>(a);
-  e = cudaGetLastError();
+  e = cudaMemsetAsync(a.ws_cnt, 0, (size_t)B * d.Hkv * R * sizeof(unsigned), st);
   if (e != cudaSuccess) return e;
-  decode_combine_kernel<<<dim3(R, d.Hkv, B), 256, 0, st>>>(a);
+  sparse_decode_kernel<<<dim3(a.nslots, d.Hkv, B), DC_WARPS * 32, smem, st>>>(a);
   return cudaGetLastError();
 }
 

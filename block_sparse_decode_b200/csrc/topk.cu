@@ -54,10 +54,12 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a) {
   const int b = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   extern __shared__ uint32_t keys[];
-  __shared__ unsigned hist[2][256];
+  __shared__ unsigned whist[TK_WARPS][256];  // per-warp digit counts
+  __shared__ unsigned hist[2][256];          // this CTA's counts (double-buffered)
   __shared__ unsigned wtot[TK_WARPS];
-  __shared__ int pick[2];
-  __shared__ unsigned ctot[2];  // this CTA's (#keys > T, #keys == T)
+  __shared__ int pick[3];                    // digit, keys above it, keys in it
+  __shared__ unsigned ctot[2];               // this CTA's (#keys > T, #keys == T)
+  __shared__ unsigned wgt[TK_WARPS], weq[TK_WARPS];
 
   const int L = a.seq_lens[b];
   const int nb = L < 0 ? 0 : (L + 3) >> 2;
@@ -78,9 +80,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a) {
   const int n = min(nb, lo + chunk) - lo;
   const float *src = a.scores + (size_t)b * a.ld + lo;
   for (int i = tid; i < n; i += TK_THREADS) keys[i] = score_key(src[i]);
-  for (int i = tid; i < 512; i += TK_THREADS) (&hist[0][0])[i] = 0u;
-  if (tid == 0) { pick[0] = 0; pick[1] = 0; }
-  __syncthreads();
+  if (tid == 0) { pick[0] = 0; pick[1] = 0; pick[2] = 0; }
 
   // contiguous per-warp segments of the CTA's range
   const int seg = (n + TK_WARPS - 1) / TK_WARPS;
@@ -90,26 +90,31 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a) {
   int need = a.k;
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass, buf = pass & 1;
-    if (pass >= 2) {
-      // hist[buf] was last read by the other CTAs before the previous cluster
-      // barrier, so it can be cleared now.
-      for (int i = tid; i < 256; i += TK_THREADS) hist[buf][i] = 0u;
-      __syncthreads();
+    // (hist[buf] was last read by the other CTAs before the previous cluster
+    // barrier, so it can be rewritten now)
+    for (int i = lane; i < 256; i += 32) whist[warp][i] = 0u;
+    __syncthreads();  // keys loaded (first pass), pick[] of the last pass read
+    for (int i = s0 + lane; i < s1; i += 32) {
+      const uint32_t key = keys[i];
+      if ((key & mask) == prefix) atomicAdd(&whist[warp][(key >> shift) & 255u], 1u);
     }
-    for (int base = s0; base < s1; base += 32) {
-      const int i = base + lane;
-      const uint32_t key = i < s1 ? keys[i] : 0u;
-      const bool live = i < s1 && (key & mask) == prefix;
-      const unsigned d = live ? ((key >> shift) & 255u) : 256u;
-      const unsigned peers = __match_any_sync(0xffffffffu, d);
-      if (live && lane == __ffs(peers) - 1) atomicAdd(&hist[buf][d], (unsigned)__popc(peers));
+    __syncthreads();
+    if (tid < 256) {
+      unsigned c = 0u;
+#pragma unroll
+      for (int w = 0; w < TK_WARPS; ++w) c += whist[w][tid];
+      hist[buf][tid] = c;
     }
     cluster.sync();
     // sum the 8 histograms; thread t takes digit 255 - t (descending order)
     unsigned c = 0u, cum = 0u;
     if (tid < 256) {
+      unsigned v[TOPK_CLUSTER];
+#pragma unroll
       for (int r = 0; r < TOPK_CLUSTER; ++r)
-        c += cluster.map_shared_rank(&hist[buf][0], r)[255 - tid];
+        v[r] = cluster.map_shared_rank(&hist[buf][0], r)[255 - tid];
+#pragma unroll
+      for (int r = 0; r < TOPK_CLUSTER; ++r) c += v[r];
       cum = c;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -124,26 +129,26 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a) {
       if (cum >= (unsigned)need && cum - c < (unsigned)need) {
         pick[0] = 255 - tid;
         pick[1] = (int)(cum - c);  // keys with a larger digit under the prefix
+        pick[2] = (int)c;          // keys with this digit under the prefix
       }
     }
     __syncthreads();
     prefix |= (uint32_t)pick[0] << shift;
     mask |= 255u << shift;
     need -= pick[1];
-    __syncthreads();  // pick[] is rewritten by the next pass
+    if (pick[2] == need) break;  // every key left under the prefix is kept
   }
-  const uint32_t T = prefix;
-  const int take_eq = need;  // ties at T that are kept (the lowest indices)
+  // Selection: keys whose masked value is above the prefix, plus the first
+  // `need` (lowest index) keys equal to it under the mask.
+  const int take_eq = need;
 
-  // counts per warp segment, then per CTA, then across the cluster
   unsigned gt = 0u, eq = 0u;
   for (int base = s0; base < s1; base += 32) {
     const int i = base + lane;
-    const uint32_t key = i < s1 ? keys[i] : 0u;
-    gt += __popc(__ballot_sync(0xffffffffu, i < s1 && key > T));
-    eq += __popc(__ballot_sync(0xffffffffu, i < s1 && key == T));
+    const uint32_t key = (i < s1 ? keys[i] : 0u) & mask;
+    gt += __popc(__ballot_sync(0xffffffffu, i < s1 && key > prefix));
+    eq += __popc(__ballot_sync(0xffffffffu, i < s1 && key == prefix));
   }
-  __shared__ unsigned wgt[TK_WARPS], weq[TK_WARPS];
   if (lane == 0) { wgt[warp] = gt; weq[warp] = eq; }
   __syncthreads();
   unsigned run_gt = 0u, run_eq = 0u;
@@ -165,8 +170,8 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a) {
   const unsigned lower = (1u << lane) - 1u;
   for (int base = s0; base < s1; base += 32) {
     const int i = base + lane;
-    const uint32_t key = i < s1 ? keys[i] : 0u;
-    const bool is_gt = i < s1 && key > T, is_eq = i < s1 && key == T;
+    const uint32_t key = (i < s1 ? keys[i] : 0u) & mask;
+    const bool is_gt = i < s1 && key > prefix, is_eq = i < s1 && key == prefix;
     const unsigned bg = __ballot_sync(0xffffffffu, is_gt);
     const unsigned be = __ballot_sync(0xffffffffu, is_eq);
     const unsigned gb = run_gt + __popc(bg & lower), eb = run_eq + __popc(be & lower);

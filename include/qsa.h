@@ -116,8 +116,8 @@ const char *qsa_last_error(void);
  *                     writes nothing at all.
  *   k_new, v_new      bf16 [N, Hkv, D];  kidx_new  bf16 [N, di].
  * Token i goes to page block_table[seq][pos / P], slot pos % P of k/v/kidx
- * pools. After all N tokens are written (a second launch on the same
- * stream), every token with pos % 4 == 3 stores the compressed key of its
+ * pools. After all N tokens are written, every token with pos % 4 == 3
+ * stores the compressed key of its
  * micro-block (positions pos-3..pos, read back from kidx_pool) at side slot
  * (pos % P) / 4 of the same page. So a bulk prefill in any token order gives
  * the same side cache as one token per call. Two entries with the same
@@ -153,7 +153,7 @@ size_t qsa_topk_workspace_size(int32_t B, int32_t ld_scores, int32_t k);
  *   sel     int32 [B, k]: the k_b = min(k, nb_b) best blocks by (score
  *           desc, block index asc), in ascending block order, then -1.
  * -0.0 ranks equal to +0.0. Supported: 1 <= k <= 4096,
- * ld_scores <= 425,984. ws may be NULL when its size is 0. */
+ * ld_scores <= 393,216. ws may be NULL when its size is 0. */
 qsa_status qsa_topk_select(int32_t B, const int32_t *seq_lens,
                            const float *scores, int32_t ld_scores, int32_t k,
                            int32_t *sel, void *ws, size_t ws_bytes,

@@ -42,8 +42,10 @@ def test_version_and_workspace_sizes(L):
     assert qsa.qsa_version() == 100
     assert qsa.qsa_topk_workspace_size(8, 65536, 512) == 0
     d = qsa.QsaDims(32, 4, 128, 16, 128, 64, 0.088)
-    # (ceil(512/32) + 4) slots x 4 kv heads x 8 heads x (128 + 1) floats per sequence
-    assert qsa.qsa_sparse_decode_workspace_size(d, 8, 512, 4) == 8 * 20 * 4 * 8 * 129 * 4
+    # (ceil(512/16) + 4) chunk slots x 4 kv heads x 8 heads x (128 + 1) floats per
+    # sequence, plus one arrival counter per (sequence, kv head, slice)
+    assert qsa.qsa_sparse_decode_workspace_size(d, 8, 512, 4) == \
+        8 * 36 * 4 * 8 * 129 * 4 + 8 * 4 * 4 * 4
 
 
 def _status(fn, *args):

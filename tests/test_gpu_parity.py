@@ -180,9 +180,9 @@ def test_merge_matches_oracle(R, out_bf16):
 
 # ------------------------------------------------------------ append alone
 
-def test_append_pools_bit_exact():
+@pytest.mark.parametrize("lens", [[259, 64, 3, 100], [13, 7, 30, 40], [4, 1]])
+def test_append_pools_bit_exact(lens):
     d = Dims(Hq=8, Hkv=4, D=128, Hi=4, di=128, P=16, scale=0.1)
-    lens = [259, 64, 3, 100]
     wl = make_custom(d, lens, k=8, R=1, seed=104, device=DEV, paged=True, pool_slack_pages=3)
     cache = qsa.alloc_cache(qsa.QsaDims.of(d), wl.num_pages, wl.block_table, device=DEV)
     for t in (cache.k_pool, cache.v_pool, cache.kidx_pool, cache.side_pool):
