@@ -1,46 +1,152 @@
-// qsa_index_score: s_b = sum_h w_h * max(0, q_idx_h . kc_b) for every
-// micro-block b of every sequence.
+// qsa_index_score on 5th-generation tensor cores: side-cache tiles gathered
+// into shared memory by cp.async producer warps, tcgen05.mma into TMEM, and an
+// epilogue that reads the accumulators back with tcgen05.ld.
 //
 // Page "Qwen 4 QSA gets decode context parallelism" (orcarouter.ai), section
-// "What the pull request actually changes": the indexer compresses keys into
-// micro-blocks at ratio 4 and "scores them". The weighted-ReLU head sum is
-// this library's reading of that step (the page prints no formula).
+// "What the pull request actually changes": the indexer scores the
+// micro-blocks. Score of block b: s_b = sum_h w_h * max(0, q_idx_h . kc_b)
+// (this library's reading; the page prints no formula).
 //
-// Work: a dense [blocks x di] . [di x Hi] contraction per sequence, 8 MAC per
-// side-cache byte (di = 128, Hi = 16), above what fp32 CUDA cores sustain at
-// HBM speed, so the dot products run on tensor cores (m16n8k16, bf16 in,
-// fp32 out). Each warp streams tiles of 16 side-cache rows (one per block)
-// through a 3-stage cp.async ring in shared memory (XOR-swizzled rows, so
-// ldmatrix is conflict-free) and keeps the indexer query of its current
-// sequence in registers as mma B fragments. The epilogue applies ReLU and
-// the head weights to the fp32 accumulators and reduces over heads with two
-// shuffles. The trailing partial block's key is built in the warp from the
-// per-token indexer-key pool and written into its tile row before the MMA.
-// The grid is persistent (2 CTAs of 8 warps per SM) over the flattened list
-// of (sequence, 16-block tile), so ragged batches stay balanced.
+// Why this shape: the contraction is [blocks x di] . [di x Hi], 8 MAC per
+// side-cache byte at di = 128, Hi = 16; at HBM speed that is ~50 TMAC/s,
+// beyond fp32 CUDA cores. One thread issues the MMAs (M = 128 blocks, N = 16
+// or 32 heads, K = di in steps of 16) into TMEM, so the tensor work costs a
+// handful of instructions per tile. The side cache is paged (a page holds P/4
+// rows), so a 128-row tile is a gather of several small pieces; measured on
+// B200, TMA tensor copies of such 2 KiB pieces top out near 3 TB/s, while
+// coalesced 16-byte cp.async from four producer warps keeps enough bytes in
+// flight to run at HBM speed. The producers write every 16-byte chunk
+// straight into the 128-byte-swizzled K-major layout that the MMA
+// descriptors expect, which also makes any page size work.
+//
+// CTA = 9 warps, persistent over the flattened (sequence, 128-block tile) list:
+//   warps 0-3  producers: per-row source rows looked up one batch of tiles
+//              ahead (block table -> side-pool row), then cp.async of the
+//              tile's rows and of the sequence's indexer query into a ring of
+//              stages; each thread's copies arrive on the stage's full barrier
+//   warp 4     TMEM owner; lane 0 issues the MMAs into one of two TMEM
+//              accumulators and commits to the stage's empty barrier and the
+//              accumulator's full barrier
+//   warps 5-8  epilogue: tcgen05.ld of 32 rows x N columns each, ReLU, head
+//              weights, one coalesced fp32 store per block; the trailing
+//              partial block (key built from its L mod 4 indexer keys) is
+//              scored on CUDA cores by the warp that owns its row.
+// Every mbarrier wait is bounded: on timeout the kernel sets the TIMEOUT bit,
+// stops all roles, drains what it issued (bounded) and frees TMEM.
 //
 // Roofline: HBM-bound; algorithmic bytes = nb * di * 2 per sequence.
+#include <algorithm>
+
 #include "common.cuh"
 #include "launch.h"
+#include "umma_desc.h"
 
 namespace qsa {
 namespace {
 
-constexpr int SC_WARPS = 8;
-constexpr int SC_STAGES = 3;
-constexpr int SC_ROWS = 16;  // blocks per warp tile
+constexpr int TC_M = 128;  // blocks per tile (MMA M)
+constexpr int TC_MAX_STAGES = 8;
+constexpr int TC_PROD_WARPS = 4;
+constexpr int TC_EPI_WARPS = 4;
+constexpr int TC_PROD = 32 * TC_PROD_WARPS;               // producer threads
+constexpr int TC_MMA_WARP = TC_PROD_WARPS;                // warp 4
+constexpr int TC_EPI0 = TC_PROD_WARPS + 1;                // first epilogue warp
+constexpr int TC_THREADS = 32 * (TC_PROD_WARPS + 1 + TC_EPI_WARPS);
+constexpr uint32_t TC_SPIN_LIMIT = 1u << 22;  // try_wait rounds before giving up
+constexpr uint32_t TC_DRAIN_LIMIT = 1u << 20;
+constexpr int PF_T = 4;  // tiles per row-lookup batch
 
-struct ScoreArgs {
+struct TcArgs {
   const __nv_bfloat16 *side_pool, *kidx_pool, *q_idx;
   const float *w;
   const int32_t *block_table, *seq_lens;
   float *scores;
-  int B, ld, P, max_pages, num_pages, Hi;
+  int B, ld, P, rpp, max_pages, num_pages, Hi, stages;
   unsigned *err;
 };
 
-// Index of the sequence whose tile range [prefix[b], prefix[b+1]) holds t.
-__device__ __forceinline__ int find_seq(const int *prefix, int B, int t) {
+struct TcCtrl {
+  uint64_t full[TC_MAX_STAGES];
+  uint64_t empty[TC_MAX_STAGES];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint32_t tmem_base;
+  int abort_flag;
+  int issued;    // tiles the producers issued
+  int consumed;  // tiles the MMA warp consumed
+  int done;      // tiles the epilogue finished
+};
+
+// ------------------------------------------------------------ PTX helpers
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.b32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait; on timeout (or once another role gave up) returns false. The
+// drain after an abort passes honor_abort = false: it must still wait for its
+// own copies and MMAs.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                          unsigned *err, uint32_t limit = TC_SPIN_LIMIT,
+                                          bool honor_abort = true) {
+  for (uint32_t i = 0; i < limit; ++i) {
+    if (mbar_try(bar, parity)) return true;
+    if (honor_abort && (i & 255u) == 255u && *abort_flag) return false;
+  }
+  *abort_flag = 1;
+  raise_err(err, ERR_TIMEOUT);
+  return false;
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+// Arrive on `bar` once every cp.async this thread issued so far has landed
+// (the arrival counts toward the barrier's expected count).
+__device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(tmem_d),
+      "l"(da), "l"(db), "r"(idesc), "r"(accumulate));
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+__device__ __forceinline__ void tc_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ int tc_find_seq(const int *prefix, int B, int t) {
   int lo = 0, hi = B - 1;
   while (lo < hi) {
     int mid = (lo + hi + 1) >> 1;
@@ -49,25 +155,94 @@ __device__ __forceinline__ int find_seq(const int *prefix, int B, int t) {
   return lo;
 }
 
-template <int DI, int NT>
-__global__ void __launch_bounds__(SC_WARPS * 32, 2) index_score_kernel(ScoreArgs a) {
-  constexpr int ROWB = DI * 2;            // bytes per side-cache row
-  constexpr int CH = ROWB / 16;           // 16-byte chunks per row
-  constexpr int TILEB = SC_ROWS * ROWB;   // bytes per warp tile
-  constexpr int KS = DI / 16;             // mma k-steps
-  extern __shared__ __align__(128) unsigned char smem[];
-  int *prefix = reinterpret_cast<int *>(smem);  // [B + 1] tiles before sequence b
-  int *lens = prefix + (a.B + 1);               // [B] sequence lengths
-  unsigned char *tiles = smem + (((2 * a.B + 1) * 4 + 127) & ~127);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+// Score of the trailing partial block of sequence b (whole warp; every lane
+// returns it). The key is the bf16-rounded mean of its L mod 4 indexer keys,
+// built exactly as the side cache builds complete blocks.
+template <int DI>
+__device__ float partial_block_score(const TcArgs &a, int b, int L, bool *ok_out) {
+  const int lane = threadIdx.x & 31;
+  const int nfull = L >> 2, n = L - 4 * nfull, pos = 4 * nfull;
+  const int col = pos / a.P;
+  int page = -1;
+  if (col < a.max_pages) page = a.block_table[(size_t)b * a.max_pages + col];
+  const bool ok = page >= 0 && page < a.num_pages;
+  *ok_out = ok;
+  if (!ok) {
+    if (lane == 0) raise_err(a.err, col < a.max_pages ? ERR_PAGE : ERR_BT);
+    return 0.f;
+  }
+  const uint32_t *x = reinterpret_cast<const uint32_t *>(a.kidx_pool) +
+                      ((size_t)page * a.P + pos % a.P) * (DI / 2);
+  float klo[DI / 64], khi[DI / 64];
+#pragma unroll
+  for (int i = 0; i < DI / 64; ++i) {
+    const int e = lane + 32 * i;
+    uint32_t v = x[e];
+    float lo = bf16lo(v), hi = bf16hi(v);
+    for (int u = 1; u < n; ++u) {
+      v = x[u * (DI / 2) + e];
+      lo = __fadd_rn(lo, bf16lo(v));
+      hi = __fadd_rn(hi, bf16hi(v));
+    }
+    const uint32_t kc = pack_bf16x2(__fdiv_rn(lo, (float)n), __fdiv_rn(hi, (float)n));
+    klo[i] = bf16lo(kc);
+    khi[i] = bf16hi(kc);
+  }
+  float score = 0.f;
+  for (int h = 0; h < a.Hi; ++h) {
+    const uint32_t *qrow =
+        reinterpret_cast<const uint32_t *>(a.q_idx + ((size_t)b * a.Hi + h) * DI);
+    float part = 0.f;
+#pragma unroll
+    for (int i = 0; i < DI / 64; ++i) {
+      const uint32_t q = qrow[lane + 32 * i];
+      part = fmaf(klo[i], bf16lo(q), part);
+      part = fmaf(khi[i], bf16hi(q), part);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    score = fmaf(a.w[(size_t)b * a.Hi + h], fmaxf(part, 0.f), score);
+  }
+  return score;
+}
 
-  // ---- per-CTA prefix of tiles per sequence
+template <int DI, int N>
+__global__ void __launch_bounds__(TC_THREADS, 1) index_score_tc_kernel(TcArgs a) {
+  constexpr int KH = DI / 64;         // 128-byte K halves
+  constexpr int CPR = DI / 8;         // 16-byte chunks per row
+  constexpr int A_HALF = TC_M * 128;  // bytes of one A half (128 rows)
+  constexpr int B_HALF = N * 128;     // bytes of one B half (N rows)
+  constexpr int STAGE = KH * (A_HALF + B_HALF);
+  constexpr int KSTEPS = DI / 16;
+  constexpr int B_PER_THREAD = (N * CPR + TC_PROD - 1) / TC_PROD;
+  constexpr uint32_t IDESC = f16_idesc(TC_M, N);
+
+  extern __shared__ unsigned char smem_raw[];
+  __shared__ TcCtrl ctl;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int S = a.stages;
+
+  // dynamic smem: [pad to 1024][stages][row table 4 warps x 2 x PF_T x 32][prefix B+1][lens B]
+  const uint32_t raw_s = smem_u32(smem_raw);
+  const uint32_t pad = (1024u - (raw_s & 1023u)) & 1023u;
+  const uint32_t ring_s = raw_s + pad;
+  int *rowtab = reinterpret_cast<int *>(smem_raw + pad + (size_t)S * STAGE);
+  int *prefix = rowtab + 2 * PF_T * TC_M;
+  int *lens = prefix + (a.B + 1);
+
+  // ---- per-CTA tile prefix over sequences
   __shared__ int carry;
-  __shared__ int wsum[SC_WARPS];
-  if (threadIdx.x == 0) { carry = 0; prefix[0] = 0; }
+  __shared__ int wsum[TC_THREADS / 32];
+  if (threadIdx.x == 0) {
+    carry = 0;
+    prefix[0] = 0;
+    ctl.abort_flag = 0;
+    ctl.issued = ctl.consumed = ctl.done = 0;
+  }
   __syncthreads();
-  for (int base = 0; base < a.B; base += blockDim.x) {
-    int b = base + threadIdx.x, n = 0;
+  for (int base = 0; base < a.B; base += TC_THREADS) {
+    const int b = base + threadIdx.x;
+    int n = 0;
     if (b < a.B) {
       int L = a.seq_lens[b];
       int nb = L < 0 ? 0 : (L + 3) >> 2;
@@ -77,12 +252,12 @@ __global__ void __launch_bounds__(SC_WARPS * 32, 2) index_score_kernel(ScoreArgs
         L = 0;
       }
       lens[b] = L;
-      n = (nb + SC_ROWS - 1) / SC_ROWS;
+      n = (nb + TC_M - 1) / TC_M;
     }
-    int x = n;  // inclusive warp scan
+    int x = n;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      int y = __shfl_up_sync(0xffffffffu, x, o);
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
       if (lane >= o) x += y;
     }
     if (lane == 31) wsum[warp] = x;
@@ -91,180 +266,242 @@ __global__ void __launch_bounds__(SC_WARPS * 32, 2) index_score_kernel(ScoreArgs
     for (int i = 0; i < warp; ++i) off += wsum[i];
     if (b < a.B) prefix[b + 1] = off + x;
     __syncthreads();
-    if (threadIdx.x == blockDim.x - 1) carry = off + x;
+    if (threadIdx.x == TC_THREADS - 1) carry = off + x;
     __syncthreads();
   }
   const int total = prefix[a.B];
+  const int my_tiles =
+      total > (int)blockIdx.x ? (total - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
 
-  unsigned char *ring = tiles + warp * (SC_STAGES * TILEB);
-  const uint32_t ring_s = smem_u32(ring);
-  // contiguous tile range per warp: consecutive tiles stay in one sequence
-  const int nwarps = gridDim.x * SC_WARPS, gwarp = blockIdx.x * SC_WARPS + warp;
-  const int t_begin = (int)(((long long)gwarp * total) / nwarps);
-  const int t_end = (int)(((long long)(gwarp + 1) * total) / nwarps);
-  const int rows_per_page = a.P >> 2;
-  const int32_t *bt_all = a.block_table;
-
-  // Page of row (lane & 15) of tile t: one independent load per lane, issued a
-  // tile ahead of its use. -1: no complete block there; -2: bounds error.
-  auto lookup = [&](int t) -> int {
-    if (t >= t_end) return -1;
-    const int b = find_seq(prefix, a.B, t);
-    const int j = (t - prefix[b]) * SC_ROWS + (lane & 15);
-    if (j >= (lens[b] >> 2)) return -1;
-    const int col = j / rows_per_page;
-    if (col >= a.max_pages) return -2;
-    const int page = __ldg(bt_all + (size_t)b * a.max_pages + col);
-    return (page >= 0 && page < a.num_pages) ? page : -3;
-  };
-  // cp.async of tile t into stage st, given each row's page (from lookup()).
-  auto issue = [&](int t, int st, int pg) {
-    if (t >= t_end) return;
-    const int j0 = (t - prefix[find_seq(prefix, a.B, t)]) * SC_ROWS;
-    if (lane < 16 && pg < -1) raise_err(a.err, pg == -2 ? ERR_BT : ERR_PAGE);
-#pragma unroll
-    for (int i = 0; i < SC_ROWS * CH / 32; ++i) {
-      const int q = lane + 32 * i, r = q / CH, c = q % CH;
-      const int page = __shfl_sync(0xffffffffu, pg, r);
-      if (page == -1) continue;
-      const int j = j0 + r;
-      const __nv_bfloat16 *src = a.side_pool;
-      int bytes = 0;
-      if (page >= 0) {
-        src = a.side_pool + ((size_t)page * rows_per_page + (j % rows_per_page)) * DI + c * 8;
-        bytes = 16;
-      }
-      cp_async16(ring_s + st * TILEB + swz(r, c, ROWB), src, bytes);
+  const uint32_t full0 = smem_u32(&ctl.full[0]), empty0 = smem_u32(&ctl.empty[0]);
+  const uint32_t tfull0 = smem_u32(&ctl.tfull[0]), tempty0 = smem_u32(&ctl.tempty[0]);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full0 + 8 * s, TC_PROD);
+      mbar_init(empty0 + 8 * s, 1);
     }
-  };
-
-  // prologue: pages of the first STAGES tiles, copies of the first STAGES-1
-  int pg_next[SC_STAGES];
-#pragma unroll
-  for (int i = 0; i < SC_STAGES; ++i) pg_next[i] = lookup(t_begin + i);
-#pragma unroll
-  for (int i = 0; i < SC_STAGES - 1; ++i) {
-    issue(t_begin + i, i, pg_next[i]);
-    cp_async_commit();
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(tfull0 + 8 * i, 1);
+      mbar_init(tempty0 + 8 * i, TC_EPI_WARPS * 32);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  int pg_ahead = pg_next[SC_STAGES - 1];  // pages of tile it + STAGES - 1
+  if (warp == TC_MMA_WARP) {  // TMEM: two accumulators of N fp32 columns (64 allocated)
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&ctl.tmem_base)),
+                 "r"(64)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl.tmem_base;
+  volatile int *abort_flag = &ctl.abort_flag;
 
-  uint32_t qf[NT][KS][2];
-  float wv[NT][2];
-  int qb = -1;
-
-  for (int it = 0;; ++it) {
-    const int t = t_begin + it;
-    if (t >= t_end) break;
-    issue(t + SC_STAGES - 1, (it + SC_STAGES - 1) % SC_STAGES, pg_ahead);
-    cp_async_commit();
-    pg_ahead = lookup(t + SC_STAGES);  // consumed by the next iteration
-    cp_async_wait<SC_STAGES - 1>();
-    __syncwarp();
-
-    const int st = it % SC_STAGES;
-    const int b = find_seq(prefix, a.B, t);
-    const int j0 = (t - prefix[b]) * SC_ROWS;
-    const int L = lens[b];
-    const int nfull = L >> 2, nb = (L + 3) >> 2;
-    unsigned char *tile = ring + st * TILEB;
-
-    if (b != qb) {  // indexer query of a new sequence -> B fragments, weights
-      qb = b;
-      const int g = lane >> 2, tq = lane & 3;
+  if (warp < TC_PROD_WARPS) {
+    // ------------------------------------------------------------ producers
+    // Producer warp w owns rows [32w, 32w + 32) of every tile. Lane l looks up
+    // row 32w + l: the absolute side-pool row of that block (-1: no complete
+    // block there; -2 / -3: bounds error), one batch of PF_T tiles ahead, so
+    // block-table latency stays off the copy path. Only warp-local
+    // synchronisation is needed, and every wait decision is warp-uniform.
+    const int row_l = warp * 32 + lane;
+    int *myrows = rowtab + warp * (2 * PF_T * 32);
+    auto fetch = [&](int batch, int (&pf)[PF_T]) {
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const int h = nt * 8 + g;
-        const uint32_t *qrow =
-            reinterpret_cast<const uint32_t *>(a.q_idx + ((size_t)b * a.Hi + h) * DI);
-#pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-          qf[nt][ks][0] = h < a.Hi ? qrow[ks * 8 + tq] : 0u;
-          qf[nt][ks][1] = h < a.Hi ? qrow[ks * 8 + 4 + tq] : 0u;
-        }
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int hw = nt * 8 + 2 * tq + e;
-          wv[nt][e] = hw < a.Hi ? a.w[(size_t)b * a.Hi + hw] : 0.f;
-        }
-      }
-    }
-
-    if (nfull < nb && nfull >= j0 && nfull < j0 + SC_ROWS) {
-      // trailing partial block: key = bf16_rne(fp32 sum of its n tokens / n)
-      const int n = L - 4 * nfull, pos = 4 * nfull;
-      const int col = pos / a.P;
-      int page = -1;
-      if (col < a.max_pages) page = bt_all[(size_t)b * a.max_pages + col];
-      const bool ok = page >= 0 && page < a.num_pages;
-      if (!ok && lane == 0) raise_err(a.err, col < a.max_pages ? ERR_PAGE : ERR_BT);
-      const uint32_t *x = reinterpret_cast<const uint32_t *>(a.kidx_pool) +
-                          ((size_t)(ok ? page : 0) * a.P + pos % a.P) * (DI / 2);
-      const int r = nfull - j0;
-      for (int e = lane; e < DI / 2; e += 32) {
-        float lo = 0.f, hi = 0.f;
-        if (ok) {
-          uint32_t v = x[e];
-          lo = bf16lo(v);
-          hi = bf16hi(v);
-          for (int u = 1; u < n; ++u) {
-            v = x[u * (DI / 2) + e];
-            lo = __fadd_rn(lo, bf16lo(v));
-            hi = __fadd_rn(hi, bf16hi(v));
+      for (int u = 0; u < PF_T; ++u) {
+        const int ti = batch * PF_T + u;
+        pf[u] = -1;
+        if (ti < my_tiles) {
+          const int t = blockIdx.x + ti * gridDim.x;
+          const int b = tc_find_seq(prefix, a.B, t);
+          const int j = (t - prefix[b]) * TC_M + row_l;
+          if (j < (lens[b] >> 2)) {
+            const int col = j / a.rpp;
+            if (col >= a.max_pages) {
+              pf[u] = -2;
+            } else {
+              const int page = __ldg(a.block_table + (size_t)b * a.max_pages + col);
+              pf[u] = (page >= 0 && page < a.num_pages) ? page * a.rpp + (j - col * a.rpp) : -3;
+            }
           }
-          lo = __fdiv_rn(lo, (float)n);
-          hi = __fdiv_rn(hi, (float)n);
         }
-        *reinterpret_cast<uint32_t *>(tile + swz(r, e >> 2, ROWB) + (e & 3) * 4) =
-            pack_bf16x2(lo, hi);
       }
+    };
+    int pf[PF_T];
+    fetch(0, pf);
+    int s = 0;
+    uint32_t ph = 0;
+    int issued = 0;
+    for (int ti = 0; ti < my_tiles; ++ti) {
+      if (ti % PF_T == 0) {  // publish this batch's rows (fetched a batch ago), fetch the next
+        int *dst = myrows + ((ti / PF_T) & 1) * PF_T * 32;
+#pragma unroll
+        for (int u = 0; u < PF_T; ++u) {
+          if (pf[u] < -1) raise_err(a.err, pf[u] == -2 ? ERR_BT : ERR_PAGE);
+          dst[u * 32 + lane] = pf[u];
+        }
+        __syncwarp();
+        fetch(ti / PF_T + 1, pf);
+      }
+      const int t = blockIdx.x + ti * gridDim.x;
+      const int b = tc_find_seq(prefix, a.B, t);
+      const int *rows = myrows + ((ti / PF_T) & 1) * PF_T * 32 + (ti % PF_T) * 32;
+      bool ok = true;
+      if (lane == 0) ok = mbar_wait(empty0 + 8 * s, ph ^ 1u, abort_flag, a.err);
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      __syncwarp();  // the stage is free for every lane, not only lane 0
+      const uint32_t stage_s = ring_s + (uint32_t)s * STAGE;
+      // A: this warp's 32 rows x CPR chunks; 32/CPR rows per instruction (coalesced)
+#pragma unroll
+      for (int i = 0; i < 32 * CPR / 32; ++i) {
+        const int q = lane + 32 * i, rl = q / CPR, c = q % CPR, r = warp * 32 + rl;
+        const int srow = rows[rl];
+        if (srow >= 0) {
+          const uint32_t dst =
+              stage_s + (c >> 3) * A_HALF + r * 128 + ((((c & 7) ^ (r & 7))) << 4);
+          cp_async16(dst, a.side_pool + (size_t)srow * DI + c * 8, 16);
+        }
+      }
+      // B: the sequence's indexer query, N rows (rows past Hi: zeros), split
+      // over the producer threads
+#pragma unroll
+      for (int i = 0; i < B_PER_THREAD; ++i) {
+        const int q = warp * 32 + lane + TC_PROD * i;
+        if (q < N * CPR) {
+          const int r = q / CPR, c = q % CPR;
+          const uint32_t dst = stage_s + KH * A_HALF + (c >> 3) * B_HALF + r * 128 +
+                               ((((c & 7) ^ (r & 7))) << 4);
+          const bool live = r < a.Hi;
+          cp_async16(dst, live ? (const void *)(a.q_idx + ((size_t)b * a.Hi + r) * DI + c * 8)
+                               : (const void *)a.q_idx,
+                     live ? 16 : 0);
+        }
+      }
+      cp_async_arrive(full0 + 8 * s);
+      ++issued;
+      if (++s == S) { s = 0; ph ^= 1u; }
+    }
+    if (threadIdx.x == 0) ctl.issued = issued;
+  } else if (warp == TC_MMA_WARP) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int s = 0, acc = 0;
+      uint32_t ph = 0, aph = 0;
+      int consumed = 0;
+      for (int ti = 0; ti < my_tiles; ++ti) {
+        if (!mbar_wait(tempty0 + 8 * acc, aph ^ 1u, abort_flag, a.err)) break;
+        if (!mbar_wait(full0 + 8 * s, ph, abort_flag, a.err)) break;
+        // the stage was written through the generic proxy (cp.async); make it
+        // visible to the tensor core's shared-memory reads
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        tc_fence_after();
+        const uint32_t stage_s = ring_s + (uint32_t)s * STAGE;
+        const uint32_t d = tmem + (uint32_t)(acc * 32);
+#pragma unroll
+        for (int ks = 0; ks < KSTEPS; ++ks) {
+          const int h = ks >> 2, kk = (ks & 3) * 32;
+          const uint64_t da = sw128_desc(stage_s + h * A_HALF + kk);
+          const uint64_t db = sw128_desc(stage_s + KH * A_HALF + h * B_HALF + kk);
+          tc_mma(d, da, db, IDESC, ks > 0 ? 1u : 0u);
+        }
+        tc_commit(empty0 + 8 * s);
+        tc_commit(tfull0 + 8 * acc);
+        ++consumed;
+        if (++s == S) { s = 0; ph ^= 1u; }
+        if (++acc == 2) { acc = 0; aph ^= 1u; }
+      }
+      ctl.consumed = consumed;
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    int acc = 0;
+    uint32_t aph = 0;
+    int done = 0;
+    for (int ti = 0; ti < my_tiles; ++ti) {
+      const int t = blockIdx.x + ti * gridDim.x;
+      const int b = tc_find_seq(prefix, a.B, t);
+      const int j0 = (t - prefix[b]) * TC_M;
+      const int L = lens[b];
+      const int nfull = L >> 2, nb = (L + 3) >> 2;
+      float wv[N];  // head weights, loaded before the wait so their latency hides
+#pragma unroll
+      for (int h = 0; h < N; ++h) wv[h] = h < a.Hi ? __ldg(a.w + (size_t)b * a.Hi + h) : 0.f;
+      bool ok = true;
+      if (lane == 0) ok = mbar_wait(tfull0 + 8 * acc, aph, abort_flag, a.err);
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       __syncwarp();
-    }
-
-    float acc[NT][4];
+      tc_fence_after();
+      float v[16];
+      float score = 0.f;
+      const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * 32);
+      tc_ld16(taddr, v);
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
-    const uint32_t ts = ring_s + st * TILEB;
-    const int arow = (lane & 7) + ((lane >> 3) & 1) * 8;
+      for (int h = 0; h < 16; ++h) score = fmaf(wv[h], fmaxf(v[h], 0.f), score);
+      if (N == 32) {
+        tc_ld16(taddr + 16, v);
 #pragma unroll
-    for (int ks = 0; ks < KS; ++ks) {
-      uint32_t a0, a1, a2, a3;
-      ldsm_x4(ts + swz(arow, 2 * ks + (lane >> 4), ROWB), a0, a1, a2, a3);
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-        mma_bf16_16816(acc[nt], a0, a1, a2, a3, qf[nt][ks][0], qf[nt][ks][1]);
+        for (int h = 0; h < 16; ++h) score = fmaf(wv[(16 + h) % N], fmaxf(v[h], 0.f), score);
+      }
+      tc_fence_before();
+      mbar_arrive(tempty0 + 8 * acc);  // the accumulator may be overwritten
+      const int j = j0 + q * 32 + lane;
+      if (j < nfull) a.scores[(size_t)b * a.ld + j] = score;
+      if (nfull < nb && nfull >= j0 + q * 32 && nfull < j0 + q * 32 + 32) {
+        bool ok;
+        const float sp = partial_block_score<DI>(a, b, L, &ok);
+        if (lane == 0 && ok) a.scores[(size_t)b * a.ld + nfull] = sp;
+      }
+      ++done;
+      if (++acc == 2) { acc = 0; aph ^= 1u; }
     }
-    float s0 = 0.f, s1 = 0.f;  // rows g and g + 8 of the tile
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      s0 += wv[nt][0] * fmaxf(acc[nt][0], 0.f) + wv[nt][1] * fmaxf(acc[nt][1], 0.f);
-      s1 += wv[nt][0] * fmaxf(acc[nt][2], 0.f) + wv[nt][1] * fmaxf(acc[nt][3], 0.f);
-    }
-    s0 += __shfl_xor_sync(0xffffffffu, s0, 1);
-    s0 += __shfl_xor_sync(0xffffffffu, s0, 2);
-    s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
-    s1 += __shfl_xor_sync(0xffffffffu, s1, 2);
-    if ((lane & 3) == 0) {
-      const int g = lane >> 2;
-      float *out = a.scores + (size_t)b * a.ld + j0;
-      if (j0 + g < nb) out[g] = s0;
-      if (j0 + g + 8 < nb) out[g + 8] = s1;
-    }
-    __syncwarp();  // the stage is refilled by the next iteration's issue
+    if (threadIdx.x == 32 * TC_EPI0) ctl.done = done;
   }
-  cp_async_wait<0>();
+
+  __syncthreads();
+  if (ctl.abort_flag) {
+    // drain: stages whose copies were issued but never consumed, MMAs whose
+    // accumulators were never read
+    if (threadIdx.x == 0) {
+      for (int i = ctl.consumed; i < ctl.issued; ++i)
+        mbar_wait(full0 + 8 * (i % S), (uint32_t)((i / S) & 1), abort_flag, a.err,
+                  TC_DRAIN_LIMIT, false);
+    }
+    if (threadIdx.x == 32 * TC_MMA_WARP) {
+      for (int i = ctl.done; i < ctl.consumed; ++i)
+        mbar_wait(tfull0 + 8 * (i & 1), (uint32_t)((i >> 1) & 1), abort_flag, a.err,
+                  TC_DRAIN_LIMIT, false);
+    }
+    __syncthreads();
+  }
+  if (warp == TC_MMA_WARP) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(64)
+                 : "memory");
+  }
 }
 
-template <int DI, int NT>
-cudaError_t launch_t(const ScoreArgs &a, cudaStream_t st) {
-  const size_t smem = (((size_t)(2 * a.B + 1) * 4 + 127) & ~(size_t)127) +
-                      (size_t)SC_WARPS * SC_STAGES * SC_ROWS * DI * 2;
-  auto kern = index_score_kernel<DI, NT>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+template <int DI, int N>
+cudaError_t launch_tc_t(TcArgs a, cudaStream_t st) {
+  constexpr int KH = DI / 64;
+  constexpr size_t STAGE = (size_t)KH * (TC_M * 128 + N * 128);
+  const size_t meta = (size_t)2 * PF_T * TC_M * 4 + (size_t)(2 * a.B + 1) * 4;
+  const size_t limit = 227 * 1024;
+  if (1024 + 2 * STAGE + meta > limit) return cudaErrorInvalidValue;
+  const int stages = (int)std::min<size_t>(6, (limit - 1024 - meta) / STAGE);
+  a.stages = stages;
+  const size_t smem = 1024 + (size_t)stages * STAGE + meta;
+  auto kern = index_score_tc_kernel<DI, N>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const int grid = device_sm_count() * 2;
-  kern<<<grid, SC_WARPS * 32, smem, st>>>(a);
+  const long long tiles_bound = (long long)a.B * ((a.ld + TC_M - 1) / TC_M);
+  const int grid =
+      (int)std::max<long long>(1, std::min<long long>(device_sm_count(), tiles_bound));
+  kern<<<grid, TC_THREADS, smem, st>>>(a);
   return cudaGetLastError();
 }
 
@@ -274,9 +511,7 @@ cudaError_t launch_index_score(const qsa_dims &d, const qsa_cache &c, int B,
                                const int32_t *seq_lens, const void *q_idx, const float *w,
                                float *scores, int ld, unsigned *err, cudaStream_t st) {
   if (B == 0) return cudaSuccess;
-  if (index_score_tc_supported(d))
-    return launch_index_score_tc(d, c, B, seq_lens, q_idx, w, scores, ld, err, st);
-  ScoreArgs a;
+  TcArgs a;
   a.side_pool = static_cast<const __nv_bfloat16 *>(c.side_pool);
   a.kidx_pool = static_cast<const __nv_bfloat16 *>(c.kidx_pool);
   a.q_idx = static_cast<const __nv_bfloat16 *>(q_idx);
@@ -287,25 +522,15 @@ cudaError_t launch_index_score(const qsa_dims &d, const qsa_cache &c, int B,
   a.B = B;
   a.ld = ld;
   a.P = d.P;
+  a.rpp = d.P / 4;
   a.max_pages = c.max_pages_per_seq;
   a.num_pages = c.num_pages;
   a.Hi = d.Hi;
+  a.stages = 2;
   a.err = err;
-  const int nt = (d.Hi + 7) / 8;
-  if (d.di == 128) {
-    switch (nt) {
-      case 1: return launch_t<128, 1>(a, st);
-      case 2: return launch_t<128, 2>(a, st);
-      case 3: return launch_t<128, 3>(a, st);
-      default: return launch_t<128, 4>(a, st);
-    }
-  }
-  switch (nt) {
-    case 1: return launch_t<64, 1>(a, st);
-    case 2: return launch_t<64, 2>(a, st);
-    case 3: return launch_t<64, 3>(a, st);
-    default: return launch_t<64, 4>(a, st);
-  }
+  if (d.di == 128)
+    return d.Hi <= 16 ? launch_tc_t<128, 16>(a, st) : launch_tc_t<128, 32>(a, st);
+  return d.Hi <= 16 ? launch_tc_t<64, 16>(a, st) : launch_tc_t<64, 32>(a, st);
 }
 
 }  // namespace qsa

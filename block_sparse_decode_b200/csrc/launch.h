@@ -23,12 +23,6 @@ cudaError_t launch_index_score(const qsa_dims &d, const qsa_cache &c, int B,
                                const int32_t *seq_lens, const void *q_idx, const float *w,
                                float *scores, int ld, unsigned *err, cudaStream_t st);
 
-// tcgen05 + TMA variant of the scoring kernel (page sizes it can address).
-bool index_score_tc_supported(const qsa_dims &d);
-cudaError_t launch_index_score_tc(const qsa_dims &d, const qsa_cache &c, int B,
-                                  const int32_t *seq_lens, const void *q_idx, const float *w,
-                                  float *scores, int ld, unsigned *err, cudaStream_t st);
-
 constexpr int TOPK_CLUSTER = 8;
 constexpr int TOPK_MAX_KEYS_PER_CTA = 49152;  // 192 KiB of keys per CTA
 cudaError_t launch_topk(int B, const int32_t *seq_lens, const float *scores, int ld, int k,

@@ -361,16 +361,18 @@ __global__ void __launch_bounds__(DC_WARPS * 32) sparse_decode_kernel(DecodeArgs
   }
 
   // ---- the CTA that finishes slice r last merges its chunks into o_part[r]
+  // (barrier, then one gpu-scope fence and the arrival by thread 0: the fence
+  // is cumulative over the CTA's partial writes the barrier ordered before it)
   const int r = s_info[0], slot0 = s_info[3], nchunks = s_info[4];
-  __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) {
+    __threadfence();
     const unsigned done = atomicAdd(a.ws_cnt + ((size_t)b * a.Hkv + g) * a.R + r, 1u);
+    __threadfence();
     s_last = (done + 1u == (unsigned)nchunks);
   }
   __syncthreads();
   if (!s_last) return;
-  __threadfence();
   if (h < a.G) {
     const size_t row0 = (((size_t)b * a.Hkv + g) * a.nslots + slot0) * a.G + h;
     float M = -INFINITY;
