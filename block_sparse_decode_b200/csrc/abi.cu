@@ -175,8 +175,10 @@ qsa_status qsa_index_score(const qsa_dims *dims, const qsa_cache *cache, int32_t
     if (ld_scores <= 0) return fail(QSA_ERR_INVALID_ARG, "ld_scores must be positive");
     if (B > 0 && (seq_lens == nullptr || q_idx == nullptr || w == nullptr || scores == nullptr))
       return fail(QSA_ERR_INVALID_ARG, "an argument array is NULL");
-    if (B > 0 && ((reinterpret_cast<uintptr_t>(q_idx) & 3u) != 0))
-      return fail(QSA_ERR_INVALID_ARG, "q_idx not 4-byte aligned");
+    if (B > 0 && !aligned16(q_idx)) return fail(QSA_ERR_INVALID_ARG, "q_idx not 16-byte aligned");
+    if (!index_score_supported(*dims))
+      return fail(QSA_ERR_UNSUPPORTED,
+                  "qsa_index_score needs the page size P to be a power of two in [32, 1024]");
     QSA_ERRWORD(err);
     return cuda_status(launch_index_score(*dims, *cache, B, seq_lens, q_idx, w, scores, ld_scores,
                                           err, reinterpret_cast<cudaStream_t>(stream)),

@@ -1,6 +1,6 @@
-// qsa_index_score on 5th-generation tensor cores: side-cache tiles gathered
-// into shared memory by cp.async producer warps, tcgen05.mma into TMEM, and an
-// epilogue that reads the accumulators back with tcgen05.ld.
+// qsa_index_score on 5th-generation tensor cores: side-cache tiles moved by
+// TMA into shared memory, tcgen05.mma into TMEM, and an epilogue that reads
+// the accumulators back with tcgen05.ld.
 //
 // Page "Qwen 4 QSA gets decode context parallelism" (orcarouter.ai), section
 // "What the pull request actually changes": the indexer scores the
@@ -11,31 +11,40 @@
 // side-cache byte at di = 128, Hi = 16; at HBM speed that is ~50 TMAC/s,
 // beyond fp32 CUDA cores. One thread issues the MMAs (M = 128 blocks, N = 16
 // or 32 heads, K = di in steps of 16) into TMEM, so the tensor work costs a
-// handful of instructions per tile. The side cache is paged (a page holds P/4
-// rows), so a 128-row tile is a gather of several small pieces; measured on
-// B200, TMA tensor copies of such 2 KiB pieces top out near 3 TB/s, while
-// coalesced 16-byte cp.async from four producer warps keeps enough bytes in
-// flight to run at HBM speed. The producers write every 16-byte chunk
-// straight into the 128-byte-swizzled K-major layout that the MMA
-// descriptors expect, which also makes any page size work.
+// few instructions per tile. The side cache is paged (P/4 rows per page): a
+// 128-row tile is a gather of 128/(P/4) page pieces. Each piece is one TMA
+// box per 128-byte K half, landing in the 128-byte-swizzled K-major layout
+// the MMA descriptors expect; the data never passes through the load/store
+// pipe, so the producer's own bookkeeping never queues behind it.
 //
-// CTA = 9 warps, persistent over the flattened (sequence, 128-block tile) list:
-//   warps 0-3  producers: per-row source rows looked up one batch of tiles
-//              ahead (block table -> side-pool row), then cp.async of the
-//              tile's rows and of the sequence's indexer query into a ring of
-//              stages; each thread's copies arrive on the stage's full barrier
-//   warp 4     TMEM owner; lane 0 issues the MMAs into one of two TMEM
+// Page ids: under full HBM load a block-table read waits several
+// microseconds behind the in-flight tile data, so per-tile lookups would
+// stall the producer. Instead the CTA copies the page ids of its tiles into
+// a shared table first (4-byte cp.async by every warp, before any tile
+// traffic; two halves, the second refilled hundreds of tiles ahead when a
+// CTA has that many tiles), and the producer reads the table.
+//
+// CTA = 6 warps, persistent over the flattened (sequence, 128-block tile) list:
+//   warp 0     producer: expect-tx, TMA boxes of the tile's page pieces and
+//              of the sequence's indexer query, into a ring of stages
+//   warp 1     TMEM owner; lane 0 issues the MMAs into one of two TMEM
 //              accumulators and commits to the stage's empty barrier and the
 //              accumulator's full barrier
-//   warps 5-8  epilogue: tcgen05.ld of 32 rows x N columns each, ReLU, head
+//   warps 2-5  epilogue: tcgen05.ld of 32 rows x N columns each, ReLU, head
 //              weights, one coalesced fp32 store per block; the trailing
 //              partial block (key built from its L mod 4 indexer keys) is
 //              scored on CUDA cores by the warp that owns its row.
 // Every mbarrier wait is bounded: on timeout the kernel sets the TIMEOUT bit,
 // stops all roles, drains what it issued (bounded) and frees TMEM.
 //
+// Supported: P a power of two in [32, 1024] (a page piece is a multiple of 8
+// rows, so every box starts on a 1 KiB swizzle atom, and pieces tile the 128
+// rows exactly), di in {64, 128}, Hi <= 32.
 // Roofline: HBM-bound; algorithmic bytes = nb * di * 2 per sequence.
+#include <cuda.h>
+
 #include <algorithm>
+#include <mutex>
 
 #include "common.cuh"
 #include "launch.h"
@@ -46,22 +55,24 @@ namespace {
 
 constexpr int TC_M = 128;  // blocks per tile (MMA M)
 constexpr int TC_MAX_STAGES = 8;
-constexpr int TC_PROD_WARPS = 4;
 constexpr int TC_EPI_WARPS = 4;
-constexpr int TC_PROD = 32 * TC_PROD_WARPS;               // producer threads
-constexpr int TC_MMA_WARP = TC_PROD_WARPS;                // warp 4
-constexpr int TC_EPI0 = TC_PROD_WARPS + 1;                // first epilogue warp
-constexpr int TC_THREADS = 32 * (TC_PROD_WARPS + 1 + TC_EPI_WARPS);
+constexpr int TC_MMA_WARP = 1;                            // warp 0 is the producer
+constexpr int TC_EPI0 = 2;                                // first epilogue warp
+constexpr int TC_THREADS = 32 * (2 + TC_EPI_WARPS);
 constexpr uint32_t TC_SPIN_LIMIT = 1u << 22;  // try_wait rounds before giving up
 constexpr uint32_t TC_DRAIN_LIMIT = 1u << 20;
-constexpr int PF_T = 4;  // tiles per row-lookup batch
+constexpr int TBL = 4096;  // shared page-table entries (two halves)
+__device__ const int32_t k_no_page = -1;
 
 struct TcArgs {
-  const __nv_bfloat16 *side_pool, *kidx_pool, *q_idx;
+  const __nv_bfloat16 *kidx_pool, *q_idx;
   const float *w;
   const int32_t *block_table, *seq_lens;
   float *scores;
   int B, ld, P, rpp, max_pages, num_pages, Hi, stages;
+  int box;  // tile rows per page piece: min(P/4, 128)
+  int ept;  // page pieces per tile: 128 / box
+  int tpc;  // tiles per half of the shared page table
   unsigned *err;
 };
 
@@ -70,6 +81,8 @@ struct TcCtrl {
   uint64_t empty[TC_MAX_STAGES];
   uint64_t tfull[2];
   uint64_t tempty[2];
+  uint64_t tbl0;    // first page-table half filled (every CTA thread)
+  uint64_t tbl[2];  // later refills of a half (producer warp)
   uint32_t tmem_base;
   int abort_flag;
   int issued;    // tiles the producers issued
@@ -105,6 +118,26 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   *abort_flag = 1;
   raise_err(err, ERR_TIMEOUT);
   return false;
+}
+__device__ __forceinline__ void mbar_arrive_expect(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, uint32_t bar,
+                                            int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(map), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar,
+                                            int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(map), "r"(bar), "r"(c0), "r"(c1)
+      : "memory");
 }
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
@@ -207,14 +240,14 @@ __device__ float partial_block_score(const TcArgs &a, int b, int L, bool *ok_out
 }
 
 template <int DI, int N>
-__global__ void __launch_bounds__(TC_THREADS, 1) index_score_tc_kernel(TcArgs a) {
+__global__ void __launch_bounds__(TC_THREADS, 1)
+    index_score_tc_kernel(const __grid_constant__ CUtensorMap side_map,
+                          const __grid_constant__ CUtensorMap q_map, TcArgs a) {
   constexpr int KH = DI / 64;         // 128-byte K halves
-  constexpr int CPR = DI / 8;         // 16-byte chunks per row
   constexpr int A_HALF = TC_M * 128;  // bytes of one A half (128 rows)
   constexpr int B_HALF = N * 128;     // bytes of one B half (N rows)
   constexpr int STAGE = KH * (A_HALF + B_HALF);
   constexpr int KSTEPS = DI / 16;
-  constexpr int B_PER_THREAD = (N * CPR + TC_PROD - 1) / TC_PROD;
   constexpr uint32_t IDESC = f16_idesc(TC_M, N);
 
   extern __shared__ unsigned char smem_raw[];
@@ -222,12 +255,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1) index_score_tc_kernel(TcArgs a)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = a.stages;
 
-  // dynamic smem: [pad to 1024][stages][row table 4 warps x 2 x PF_T x 32][prefix B+1][lens B]
+  // dynamic smem: [pad to 1024][stages][page table TBL][prefix B+1][lens B]
   const uint32_t raw_s = smem_u32(smem_raw);
   const uint32_t pad = (1024u - (raw_s & 1023u)) & 1023u;
   const uint32_t ring_s = raw_s + pad;
-  int *rowtab = reinterpret_cast<int *>(smem_raw + pad + (size_t)S * STAGE);
-  int *prefix = rowtab + 2 * PF_T * TC_M;
+  int *prefix = reinterpret_cast<int *>(smem_raw + pad + (size_t)S * STAGE + TBL * 4);
   int *lens = prefix + (a.B + 1);
 
   // ---- per-CTA tile prefix over sequences
@@ -273,19 +305,52 @@ __global__ void __launch_bounds__(TC_THREADS, 1) index_score_tc_kernel(TcArgs a)
   const int my_tiles =
       total > (int)blockIdx.x ? (total - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
 
+  // Shared page table: half h holds, for tpc consecutive tiles of this CTA,
+  // the page ids of the tile's ept page pieces (-1: the piece holds no
+  // complete block). Warps fill tiles round-robin with 4-byte cp.async; every
+  // filling thread arrives on the half's barrier when its copies land.
+  int *table = reinterpret_cast<int *>(smem_raw + pad + (size_t)S * STAGE);
+  auto tile_start = [&](int ti, int &b, int &j0) {
+    const int t = blockIdx.x + ti * gridDim.x;
+    b = tc_find_seq(prefix, a.B, t);
+    j0 = (t - prefix[b]) * TC_M;
+  };
+  auto fill_table = [&](int chunk, int wfirst, int nwarps) {
+    int *half = table + (chunk & 1) * (TBL / 2);
+    const int ntiles = min(a.tpc, my_tiles - chunk * a.tpc);
+    for (int til = warp - wfirst; til < ntiles; til += nwarps) {
+      int b, j0;
+      tile_start(chunk * a.tpc + til, b, j0);
+      const int col0 = j0 / a.rpp, nfull = lens[b] >> 2;
+      for (int k = lane; k < a.ept; k += 32) {
+        const int col = col0 + k;
+        const bool live = (j0 + k * a.box) < nfull && col < a.max_pages;
+        if ((j0 + k * a.box) < nfull && col >= a.max_pages) raise_err(a.err, ERR_BT);
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(
+                         smem_u32(half + til * a.ept + k)),
+                     "l"(live ? a.block_table + (size_t)b * a.max_pages + col : &k_no_page)
+                     : "memory");
+      }
+    }
+  };
   const uint32_t full0 = smem_u32(&ctl.full[0]), empty0 = smem_u32(&ctl.empty[0]);
   const uint32_t tfull0 = smem_u32(&ctl.tfull[0]), tempty0 = smem_u32(&ctl.tempty[0]);
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(full0 + 8 * s, TC_PROD);
+      mbar_init(full0 + 8 * s, 1);
       mbar_init(empty0 + 8 * s, 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(tfull0 + 8 * i, 1);
       mbar_init(tempty0 + 8 * i, TC_EPI_WARPS * 32);
+      mbar_init(smem_u32(&ctl.tbl[i]), 32);
     }
+    mbar_init(smem_u32(&ctl.tbl0), TC_THREADS);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  __syncthreads();  // barriers initialised before the first table copy arrives
+  fill_table(0, 0, TC_THREADS / 32);
+  cp_async_arrive(smem_u32(&ctl.tbl0));
   if (warp == TC_MMA_WARP) {  // TMEM: two accumulators of N fp32 columns (64 allocated)
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(&ctl.tmem_base)),
@@ -299,91 +364,65 @@ __global__ void __launch_bounds__(TC_THREADS, 1) index_score_tc_kernel(TcArgs a)
   const uint32_t tmem = ctl.tmem_base;
   volatile int *abort_flag = &ctl.abort_flag;
 
-  if (warp < TC_PROD_WARPS) {
-    // ------------------------------------------------------------ producers
-    // Producer warp w owns rows [32w, 32w + 32) of every tile. Lane l looks up
-    // row 32w + l: the absolute side-pool row of that block (-1: no complete
-    // block there; -2 / -3: bounds error), one batch of PF_T tiles ahead, so
-    // block-table latency stays off the copy path. Only warp-local
-    // synchronisation is needed, and every wait decision is warp-uniform.
-    const int row_l = warp * 32 + lane;
-    int *myrows = rowtab + warp * (2 * PF_T * 32);
-    auto fetch = [&](int batch, int (&pf)[PF_T]) {
-#pragma unroll
-      for (int u = 0; u < PF_T; ++u) {
-        const int ti = batch * PF_T + u;
-        pf[u] = -1;
-        if (ti < my_tiles) {
-          const int t = blockIdx.x + ti * gridDim.x;
-          const int b = tc_find_seq(prefix, a.B, t);
-          const int j = (t - prefix[b]) * TC_M + row_l;
-          if (j < (lens[b] >> 2)) {
-            const int col = j / a.rpp;
-            if (col >= a.max_pages) {
-              pf[u] = -2;
-            } else {
-              const int page = __ldg(a.block_table + (size_t)b * a.max_pages + col);
-              pf[u] = (page >= 0 && page < a.num_pages) ? page * a.rpp + (j - col * a.rpp) : -3;
-            }
-          }
-        }
-      }
-    };
-    int pf[PF_T];
-    fetch(0, pf);
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
     int s = 0;
     uint32_t ph = 0;
     int issued = 0;
     for (int ti = 0; ti < my_tiles; ++ti) {
-      if (ti % PF_T == 0) {  // publish this batch's rows (fetched a batch ago), fetch the next
-        int *dst = myrows + ((ti / PF_T) & 1) * PF_T * 32;
-#pragma unroll
-        for (int u = 0; u < PF_T; ++u) {
-          if (pf[u] < -1) raise_err(a.err, pf[u] == -2 ? ERR_BT : ERR_PAGE);
-          dst[u * 32 + lane] = pf[u];
-        }
+      const int chunk = ti / a.tpc, tl = ti - chunk * a.tpc;
+      if (tl == 0) {  // this half of the page table must have landed
+        bool ok = true;
+        if (lane == 0)
+          ok = chunk == 0 ? mbar_wait(smem_u32(&ctl.tbl0), 0u, abort_flag, a.err)
+                          : mbar_wait(smem_u32(&ctl.tbl[chunk & 1]),
+                                      (uint32_t)(((chunk - 1) >> 1) & 1), abort_flag, a.err);
+        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
         __syncwarp();
-        fetch(ti / PF_T + 1, pf);
       }
-      const int t = blockIdx.x + ti * gridDim.x;
-      const int b = tc_find_seq(prefix, a.B, t);
-      const int *rows = myrows + ((ti / PF_T) & 1) * PF_T * 32 + (ti % PF_T) * 32;
+      // Refill the other half for the next chunk: after the first fill only
+      // this warp reads the table, and it left that half a chunk ago.
+      if (tl == 1 && (chunk + 1) * a.tpc < my_tiles) {
+        fill_table(chunk + 1, 0, 1);
+        cp_async_arrive(smem_u32(&ctl.tbl[(chunk + 1) & 1]));
+      }
+      int b, j0;
+      tile_start(ti, b, j0);
+      const int rows = max(0, min(TC_M, (lens[b] >> 2) - j0));  // complete blocks
+      const int npiece = (rows + a.box - 1) / a.box;
+      int page = -1;
+      if (lane < npiece) {
+        page = table[(chunk & 1) * (TBL / 2) + tl * a.ept + lane];
+        if (page < 0 || page >= a.num_pages) {
+          if (page != -1) raise_err(a.err, ERR_PAGE);
+          page = -1;
+        }
+      }
       bool ok = true;
       if (lane == 0) ok = mbar_wait(empty0 + 8 * s, ph ^ 1u, abort_flag, a.err);
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-      __syncwarp();  // the stage is free for every lane, not only lane 0
+      __syncwarp();
+      const unsigned live = __ballot_sync(0xffffffffu, page >= 0);
       const uint32_t stage_s = ring_s + (uint32_t)s * STAGE;
-      // A: this warp's 32 rows x CPR chunks; 32/CPR rows per instruction (coalesced)
+      const uint32_t bar = full0 + 8 * s;
+      if (lane == 0)
+        mbar_arrive_expect(bar, (uint32_t)(__popc(live) * a.box * 128 * KH + B_HALF * KH));
+      __syncwarp();
+      if (page >= 0) {
+        const int rip = (j0 + lane * a.box) % a.rpp;  // row in page (rpp > 128 only)
 #pragma unroll
-      for (int i = 0; i < 32 * CPR / 32; ++i) {
-        const int q = lane + 32 * i, rl = q / CPR, c = q % CPR, r = warp * 32 + rl;
-        const int srow = rows[rl];
-        if (srow >= 0) {
-          const uint32_t dst =
-              stage_s + (c >> 3) * A_HALF + r * 128 + ((((c & 7) ^ (r & 7))) << 4);
-          cp_async16(dst, a.side_pool + (size_t)srow * DI + c * 8, 16);
-        }
+        for (int h = 0; h < KH; ++h)
+          tma_load_3d(stage_s + h * A_HALF + lane * a.box * 128, &side_map, bar, h * 64, rip, page);
       }
-      // B: the sequence's indexer query, N rows (rows past Hi: zeros), split
-      // over the producer threads
+      if (lane == 0) {
 #pragma unroll
-      for (int i = 0; i < B_PER_THREAD; ++i) {
-        const int q = warp * 32 + lane + TC_PROD * i;
-        if (q < N * CPR) {
-          const int r = q / CPR, c = q % CPR;
-          const uint32_t dst = stage_s + KH * A_HALF + (c >> 3) * B_HALF + r * 128 +
-                               ((((c & 7) ^ (r & 7))) << 4);
-          const bool live = r < a.Hi;
-          cp_async16(dst, live ? (const void *)(a.q_idx + ((size_t)b * a.Hi + r) * DI + c * 8)
-                               : (const void *)a.q_idx,
-                     live ? 16 : 0);
-        }
+        for (int h = 0; h < KH; ++h)
+          tma_load_2d(stage_s + KH * A_HALF + h * B_HALF, &q_map, bar, h * 64, b * a.Hi);
       }
-      cp_async_arrive(full0 + 8 * s);
       ++issued;
       if (++s == S) { s = 0; ph ^= 1u; }
     }
-    if (threadIdx.x == 0) ctl.issued = issued;
+    if (lane == 0) ctl.issued = issued;
   } else if (warp == TC_MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -393,18 +432,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1) index_score_tc_kernel(TcArgs a)
       for (int ti = 0; ti < my_tiles; ++ti) {
         if (!mbar_wait(tempty0 + 8 * acc, aph ^ 1u, abort_flag, a.err)) break;
         if (!mbar_wait(full0 + 8 * s, ph, abort_flag, a.err)) break;
-        // the stage was written through the generic proxy (cp.async); make it
-        // visible to the tensor core's shared-memory reads
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         tc_fence_after();
         const uint32_t stage_s = ring_s + (uint32_t)s * STAGE;
         const uint32_t d = tmem + (uint32_t)(acc * 32);
+        // descriptors of the stage base; each k-step adds its byte offset / 16 to
+        // the start-address field (no carry: shared addresses stay below 256 KiB)
+        const uint64_t da0 = sw128_desc(stage_s), db0 = sw128_desc(stage_s + KH * A_HALF);
 #pragma unroll
         for (int ks = 0; ks < KSTEPS; ++ks) {
           const int h = ks >> 2, kk = (ks & 3) * 32;
-          const uint64_t da = sw128_desc(stage_s + h * A_HALF + kk);
-          const uint64_t db = sw128_desc(stage_s + KH * A_HALF + h * B_HALF + kk);
-          tc_mma(d, da, db, IDESC, ks > 0 ? 1u : 0u);
+          tc_mma(d, da0 + (uint64_t)((h * A_HALF + kk) >> 4),
+                 db0 + (uint64_t)((h * B_HALF + kk) >> 4), IDESC, ks > 0 ? 1u : 0u);
         }
         tc_commit(empty0 + 8 * s);
         tc_commit(tfull0 + 8 * acc);
@@ -484,35 +522,84 @@ __global__ void __launch_bounds__(TC_THREADS, 1) index_score_tc_kernel(TcArgs a)
   }
 }
 
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// cuTensorMapEncodeTiled from the driver (no link-time libcuda dependency).
+EncodeTiledFn encode_fn(cudaError_t *status) {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  static cudaError_t st = cudaSuccess;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    st = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+    if (st == cudaSuccess && q != cudaDriverEntryPointSuccess) st = cudaErrorNotSupported;
+    fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  *status = st;
+  return fn;
+}
+
 template <int DI, int N>
-cudaError_t launch_tc_t(TcArgs a, cudaStream_t st) {
+cudaError_t launch_tc_t(const qsa_cache &c, TcArgs a, cudaStream_t st) {
+  cudaError_t e;
+  EncodeTiledFn enc = encode_fn(&e);
+  if (e != cudaSuccess) return e;
+  if (enc == nullptr) return cudaErrorNotSupported;
+  // side pool viewed as [num_pages][rpp rows][DI]; q_idx as [B*Hi][DI]
+  CUtensorMap side_map, q_map;
+  {
+    const cuuint64_t dims[3] = {(cuuint64_t)DI, (cuuint64_t)a.rpp, (cuuint64_t)c.num_pages};
+    const cuuint64_t strides[2] = {(cuuint64_t)DI * 2, (cuuint64_t)a.rpp * DI * 2};
+    const cuuint32_t box[3] = {64u, (cuuint32_t)a.box, 1u};
+    const cuuint32_t estr[3] = {1u, 1u, 1u};
+    if (enc(&side_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, c.side_pool, dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)DI, (cuuint64_t)a.B * a.Hi};
+    const cuuint64_t strides[1] = {(cuuint64_t)DI * 2};
+    const cuuint32_t box[2] = {64u, (cuuint32_t)N};
+    const cuuint32_t estr[2] = {1u, 1u};
+    if (enc(&q_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<__nv_bfloat16 *>(a.q_idx),
+            dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
   constexpr int KH = DI / 64;
   constexpr size_t STAGE = (size_t)KH * (TC_M * 128 + N * 128);
-  const size_t meta = (size_t)2 * PF_T * TC_M * 4 + (size_t)(2 * a.B + 1) * 4;
+  const size_t meta = (size_t)TBL * 4 + (size_t)(2 * a.B + 1) * 4;
   const size_t limit = 227 * 1024;
   if (1024 + 2 * STAGE + meta > limit) return cudaErrorInvalidValue;
-  const int stages = (int)std::min<size_t>(6, (limit - 1024 - meta) / STAGE);
-  a.stages = stages;
-  const size_t smem = 1024 + (size_t)stages * STAGE + meta;
+  a.stages = (int)std::min<size_t>(6, (limit - 1024 - meta) / STAGE);
+  const size_t smem = 1024 + (size_t)a.stages * STAGE + meta;
   auto kern = index_score_tc_kernel<DI, N>;
-  cudaError_t e =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const long long tiles_bound = (long long)a.B * ((a.ld + TC_M - 1) / TC_M);
   const int grid =
       (int)std::max<long long>(1, std::min<long long>(device_sm_count(), tiles_bound));
-  kern<<<grid, TC_THREADS, smem, st>>>(a);
+  kern<<<grid, TC_THREADS, smem, st>>>(side_map, q_map, a);
   return cudaGetLastError();
 }
 
 }  // namespace
+
+bool index_score_supported(const qsa_dims &d) {
+  const bool pow2 = d.P >= 32 && d.P <= 1024 && (d.P & (d.P - 1)) == 0;
+  return pow2 && (d.di == 64 || d.di == 128) && d.Hi <= 32;
+}
 
 cudaError_t launch_index_score(const qsa_dims &d, const qsa_cache &c, int B,
                                const int32_t *seq_lens, const void *q_idx, const float *w,
                                float *scores, int ld, unsigned *err, cudaStream_t st) {
   if (B == 0) return cudaSuccess;
   TcArgs a;
-  a.side_pool = static_cast<const __nv_bfloat16 *>(c.side_pool);
   a.kidx_pool = static_cast<const __nv_bfloat16 *>(c.kidx_pool);
   a.q_idx = static_cast<const __nv_bfloat16 *>(q_idx);
   a.w = w;
@@ -523,14 +610,17 @@ cudaError_t launch_index_score(const qsa_dims &d, const qsa_cache &c, int B,
   a.ld = ld;
   a.P = d.P;
   a.rpp = d.P / 4;
+  a.box = std::min(a.rpp, TC_M);
+  a.ept = TC_M / a.box;
+  a.tpc = (TBL / 2) / a.ept;
   a.max_pages = c.max_pages_per_seq;
   a.num_pages = c.num_pages;
   a.Hi = d.Hi;
   a.stages = 2;
   a.err = err;
   if (d.di == 128)
-    return d.Hi <= 16 ? launch_tc_t<128, 16>(a, st) : launch_tc_t<128, 32>(a, st);
-  return d.Hi <= 16 ? launch_tc_t<64, 16>(a, st) : launch_tc_t<64, 32>(a, st);
+    return d.Hi <= 16 ? launch_tc_t<128, 16>(c, a, st) : launch_tc_t<128, 32>(c, a, st);
+  return d.Hi <= 16 ? launch_tc_t<64, 16>(c, a, st) : launch_tc_t<64, 32>(c, a, st);
 }
 
 }  // namespace qsa

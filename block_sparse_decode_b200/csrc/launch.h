@@ -19,6 +19,7 @@ cudaError_t launch_append(const qsa_dims &d, const qsa_cache &c, int N, const in
                           const int32_t *tok_pos, const void *k_new, const void *v_new,
                           const void *kidx_new, unsigned *err, cudaStream_t st);
 
+bool index_score_supported(const qsa_dims &d);  // page sizes the TMA gather can address
 cudaError_t launch_index_score(const qsa_dims &d, const qsa_cache &c, int B,
                                const int32_t *seq_lens, const void *q_idx, const float *w,
                                float *scores, int ld, unsigned *err, cudaStream_t st);

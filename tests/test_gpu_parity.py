@@ -76,9 +76,9 @@ def test_ragged_paged_full_heads(R):
 
 
 @pytest.mark.parametrize("dims,lens,k", [
-    (Dims(Hq=4, Hkv=4, D=128, Hi=5, di=64, P=16, scale=0.11), [77, 1030, 3], 40),
+    (Dims(Hq=4, Hkv=4, D=128, Hi=5, di=64, P=32, scale=0.11), [77, 1030, 3], 40),
     (Dims(Hq=12, Hkv=2, D=128, Hi=24, di=128, P=128, scale=0.09), [4096, 515, 6000], 100),
-    (Dims(Hq=2, Hkv=1, D=128, Hi=1, di=128, P=4, scale=0.2), [33, 257], 7),
+    (Dims(Hq=2, Hkv=1, D=128, Hi=1, di=128, P=1024, scale=0.2), [33, 2570], 7),
     (Dims(Hq=16, Hkv=2, D=128, Hi=32, di=64, P=64, scale=0.088), [1500, 2600], 1),
 ])
 def test_other_dims(dims, lens, k):
