@@ -24,13 +24,14 @@
 // traffic; two halves, the second refilled hundreds of tiles ahead when a
 // CTA has that many tiles), and the producer reads the table.
 //
-// CTA = 6 warps, persistent over the flattened (sequence, 128-block tile) list:
-//   warp 0     producer: expect-tx, TMA boxes of the tile's page pieces and
-//              of the sequence's indexer query, into a ring of stages
-//   warp 1     TMEM owner; lane 0 issues the MMAs into one of two TMEM
+// CTA = 7 warps, persistent over the flattened (sequence, 128-block tile) list:
+//   warps 0-1  producers (alternate tiles): expect-tx, TMA boxes of the
+//              tile's page pieces and, when the stage holds another
+//              sequence's, of the indexer query, into a ring of stages
+//   warp 2     TMEM owner; lane 0 issues the MMAs into one of two TMEM
 //              accumulators and commits to the stage's empty barrier and the
 //              accumulator's full barrier
-//   warps 2-5  epilogue: tcgen05.ld of 32 rows x N columns each, ReLU, head
+//   warps 3-6  epilogue: tcgen05.ld of 32 rows x N columns each, ReLU, head
 //              weights, one coalesced fp32 store per block; the trailing
 //              partial block (key built from its L mod 4 indexer keys) is
 //              scored on CUDA cores by the warp that owns its row.
@@ -56,9 +57,10 @@ namespace {
 constexpr int TC_M = 128;  // blocks per tile (MMA M)
 constexpr int TC_MAX_STAGES = 8;
 constexpr int TC_EPI_WARPS = 4;
-constexpr int TC_MMA_WARP = 1;                            // warp 0 is the producer
-constexpr int TC_EPI0 = 2;                                // first epilogue warp
-constexpr int TC_THREADS = 32 * (2 + TC_EPI_WARPS);
+constexpr int TC_PROD_WARPS = 2;                          // producers take alternate tiles
+constexpr int TC_MMA_WARP = TC_PROD_WARPS;                // warp 2
+constexpr int TC_EPI0 = TC_PROD_WARPS + 1;                // first epilogue warp
+constexpr int TC_THREADS = 32 * (TC_PROD_WARPS + 1 + TC_EPI_WARPS);
 constexpr uint32_t TC_SPIN_LIMIT = 1u << 22;  // try_wait rounds before giving up
 constexpr uint32_t TC_DRAIN_LIMIT = 1u << 20;
 constexpr int TBL = 4096;  // shared page-table entries (two halves)
@@ -85,7 +87,8 @@ struct TcCtrl {
   uint64_t tbl[2];  // later refills of a half (producer warp)
   uint32_t tmem_base;
   int abort_flag;
-  int issued;    // tiles the producers issued
+  int issued[TC_PROD_WARPS];  // per producer warp: first tile index it did not issue
+  int qseq[TC_MAX_STAGES];    // sequence whose indexer query a stage holds
   int consumed;  // tiles the MMA warp consumed
   int done;      // tiles the epilogue finished
 };
@@ -269,7 +272,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     carry = 0;
     prefix[0] = 0;
     ctl.abort_flag = 0;
-    ctl.issued = ctl.consumed = ctl.done = 0;
+    ctl.consumed = ctl.done = 0;
+    for (int w = 0; w < TC_PROD_WARPS; ++w) ctl.issued[w] = w;
+    for (int i = 0; i < TC_MAX_STAGES; ++i) ctl.qseq[i] = -1;
   }
   __syncthreads();
   for (int base = 0; base < a.B; base += TC_THREADS) {
@@ -364,14 +369,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   const uint32_t tmem = ctl.tmem_base;
   volatile int *abort_flag = &ctl.abort_flag;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    int s = 0;
-    uint32_t ph = 0;
-    int issued = 0;
-    for (int ti = 0; ti < my_tiles; ++ti) {
+  if (warp < TC_PROD_WARPS) {
+    // ------------------------------------------------------------ producers
+    // Warp w issues tiles w, w + 2, ...; stage and phase follow from the tile
+    // index, so the MMA warp consumes tiles in order. One warp's bookkeeping
+    // overlaps the other's TMA issue.
+    int last_chunk = -1, refilled = 0;
+    int ti = warp;
+    for (; ti < my_tiles; ti += TC_PROD_WARPS) {
       const int chunk = ti / a.tpc, tl = ti - chunk * a.tpc;
-      if (tl == 0) {  // this half of the page table must have landed
+      if (chunk != last_chunk) {  // this half of the page table must have landed
         bool ok = true;
         if (lane == 0)
           ok = chunk == 0 ? mbar_wait(smem_u32(&ctl.tbl0), 0u, abort_flag, a.err)
@@ -379,12 +386,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                                       (uint32_t)(((chunk - 1) >> 1) & 1), abort_flag, a.err);
         if (!__shfl_sync(0xffffffffu, ok, 0)) break;
         __syncwarp();
+        last_chunk = chunk;
       }
-      // Refill the other half for the next chunk: after the first fill only
-      // this warp reads the table, and it left that half a chunk ago.
-      if (tl == 1 && (chunk + 1) * a.tpc < my_tiles) {
+      // Refill the other half for the next chunk once both producers are past
+      // the previous one (a producer runs at most S tiles ahead of the other:
+      // it waits for the stage of tile ti - S, issued by either warp).
+      if (warp == 0 && refilled <= chunk && tl >= S + 2 && (chunk + 1) * a.tpc < my_tiles) {
         fill_table(chunk + 1, 0, 1);
         cp_async_arrive(smem_u32(&ctl.tbl[(chunk + 1) & 1]));
+        refilled = chunk + 1;
       }
       int b, j0;
       tile_start(ti, b, j0);
@@ -398,31 +408,31 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           page = -1;
         }
       }
+      const int s = ti % S;
+      const uint32_t ph = (uint32_t)((ti / S) & 1);
       bool ok = true;
       if (lane == 0) ok = mbar_wait(empty0 + 8 * s, ph ^ 1u, abort_flag, a.err);
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       __syncwarp();
       const unsigned live = __ballot_sync(0xffffffffu, page >= 0);
+      const bool new_q = ctl.qseq[s] != b;  // the stage's query buffer holds another sequence
       const uint32_t stage_s = ring_s + (uint32_t)s * STAGE;
       const uint32_t bar = full0 + 8 * s;
-      if (lane == 0)
-        mbar_arrive_expect(bar, (uint32_t)(__popc(live) * a.box * 128 * KH + B_HALF * KH));
+      if (lane == 0) {
+        mbar_arrive_expect(bar, (uint32_t)(__popc(live) * a.box * 128 * KH + (new_q ? B_HALF * KH : 0)));
+        ctl.qseq[s] = b;
+      }
       __syncwarp();
       if (page >= 0) {
-        const int rip = (j0 + lane * a.box) % a.rpp;  // row in page (rpp > 128 only)
+        const int rip = (j0 + lane * a.box) % a.rpp;  // row in page (P > 512 only)
 #pragma unroll
         for (int h = 0; h < KH; ++h)
           tma_load_3d(stage_s + h * A_HALF + lane * a.box * 128, &side_map, bar, h * 64, rip, page);
       }
-      if (lane == 0) {
-#pragma unroll
-        for (int h = 0; h < KH; ++h)
-          tma_load_2d(stage_s + KH * A_HALF + h * B_HALF, &q_map, bar, h * 64, b * a.Hi);
-      }
-      ++issued;
-      if (++s == S) { s = 0; ph ^= 1u; }
+      if (new_q && lane < KH)
+        tma_load_2d(stage_s + KH * A_HALF + lane * B_HALF, &q_map, bar, lane * 64, b * a.Hi);
     }
-    if (lane == 0) ctl.issued = issued;
+    if (lane == 0) ctl.issued[warp] = ti;
   } else if (warp == TC_MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -504,9 +514,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     // drain: stages whose copies were issued but never consumed, MMAs whose
     // accumulators were never read
     if (threadIdx.x == 0) {
-      for (int i = ctl.consumed; i < ctl.issued; ++i)
-        mbar_wait(full0 + 8 * (i % S), (uint32_t)((i / S) & 1), abort_flag, a.err,
-                  TC_DRAIN_LIMIT, false);
+      for (int i = ctl.consumed; i < my_tiles; ++i)
+        if (i < ctl.issued[i % TC_PROD_WARPS])
+          mbar_wait(full0 + 8 * (i % S), (uint32_t)((i / S) & 1), abort_flag, a.err,
+                    TC_DRAIN_LIMIT, false);
     }
     if (threadIdx.x == 32 * TC_MMA_WARP) {
       for (int i = ctl.done; i < ctl.consumed; ++i)
@@ -576,7 +587,8 @@ cudaError_t launch_tc_t(const qsa_cache &c, TcArgs a, cudaStream_t st) {
   const size_t meta = (size_t)TBL * 4 + (size_t)(2 * a.B + 1) * 4;
   const size_t limit = 227 * 1024;
   if (1024 + 2 * STAGE + meta > limit) return cudaErrorInvalidValue;
-  a.stages = (int)std::min<size_t>(6, (limit - 1024 - meta) / STAGE);
+  // an even stage count keeps each stage with one producer warp (alternate tiles)
+  a.stages = (int)std::min<size_t>(6, (limit - 1024 - meta) / STAGE) & ~1;
   const size_t smem = 1024 + (size_t)a.stages * STAGE + meta;
   auto kern = index_score_tc_kernel<DI, N>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
