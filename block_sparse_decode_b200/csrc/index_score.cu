@@ -24,14 +24,14 @@
 // traffic; two halves, the second refilled hundreds of tiles ahead when a
 // CTA has that many tiles), and the producer reads the table.
 //
-// CTA = 7 warps, persistent over the flattened (sequence, 128-block tile) list:
-//   warps 0-1  producers (alternate tiles): expect-tx, TMA boxes of the
+// CTA = 8 warps, persistent over the flattened (sequence, 128-block tile) list:
+//   warps 0-2  producers (tiles round-robin): expect-tx, TMA boxes of the
 //              tile's page pieces and, when the stage holds another
 //              sequence's, of the indexer query, into a ring of stages
-//   warp 2     TMEM owner; lane 0 issues the MMAs into one of two TMEM
+//   warp 3     TMEM owner; lane 0 issues the MMAs into one of two TMEM
 //              accumulators and commits to the stage's empty barrier and the
 //              accumulator's full barrier
-//   warps 3-6  epilogue: tcgen05.ld of 32 rows x N columns each, ReLU, head
+//   warps 4-7  epilogue: tcgen05.ld of 32 rows x N columns each, ReLU, head
 //              weights, one coalesced fp32 store per block; the trailing
 //              partial block (key built from its L mod 4 indexer keys) is
 //              scored on CUDA cores by the warp that owns its row.
@@ -57,8 +57,8 @@ namespace {
 constexpr int TC_M = 128;  // blocks per tile (MMA M)
 constexpr int TC_MAX_STAGES = 8;
 constexpr int TC_EPI_WARPS = 4;
-constexpr int TC_PROD_WARPS = 2;                          // producers take alternate tiles
-constexpr int TC_MMA_WARP = TC_PROD_WARPS;                // warp 2
+constexpr int TC_PROD_WARPS = 3;                          // producers take tiles round-robin
+constexpr int TC_MMA_WARP = TC_PROD_WARPS;                // warp 3
 constexpr int TC_EPI0 = TC_PROD_WARPS + 1;                // first epilogue warp
 constexpr int TC_THREADS = 32 * (TC_PROD_WARPS + 1 + TC_EPI_WARPS);
 constexpr uint32_t TC_SPIN_LIMIT = 1u << 22;  // try_wait rounds before giving up
@@ -371,7 +371,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
   if (warp < TC_PROD_WARPS) {
     // ------------------------------------------------------------ producers
-    // Warp w issues tiles w, w + 2, ...; stage and phase follow from the tile
+    // Warp w issues tiles w, w + 3, ...; stage and phase follow from the tile
     // index, so the MMA warp consumes tiles in order. One warp's bookkeeping
     // overlaps the other's TMA issue.
     int last_chunk = -1, refilled = 0;
@@ -388,10 +388,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         __syncwarp();
         last_chunk = chunk;
       }
-      // Refill the other half for the next chunk once both producers are past
-      // the previous one (a producer runs at most S tiles ahead of the other:
-      // it waits for the stage of tile ti - S, issued by either warp).
-      if (warp == 0 && refilled <= chunk && tl >= S + 2 && (chunk + 1) * a.tpc < my_tiles) {
+      // Refill the other half for the next chunk once every producer is past
+      // the previous one: a producer at tile ti has seen the stage of tile
+      // ti - S consumed, and the MMA consumes in order, so every other
+      // producer has issued beyond ti - S - TC_PROD_WARPS.
+      if (warp == 0 && refilled <= chunk && tl >= S + TC_PROD_WARPS &&
+          (chunk + 1) * a.tpc < my_tiles) {
         fill_table(chunk + 1, 0, 1);
         cp_async_arrive(smem_u32(&ctl.tbl[(chunk + 1) & 1]));
         refilled = chunk + 1;
@@ -587,8 +589,11 @@ cudaError_t launch_tc_t(const qsa_cache &c, TcArgs a, cudaStream_t st) {
   const size_t meta = (size_t)TBL * 4 + (size_t)(2 * a.B + 1) * 4;
   const size_t limit = 227 * 1024;
   if (1024 + 2 * STAGE + meta > limit) return cudaErrorInvalidValue;
-  // an even stage count keeps each stage with one producer warp (alternate tiles)
-  a.stages = (int)std::min<size_t>(6, (limit - 1024 - meta) / STAGE) & ~1;
+  // a multiple of the producer count keeps each stage with one producer warp
+  a.stages = (int)std::min<size_t>(6, (limit - 1024 - meta) / STAGE);
+  a.stages -= a.stages % TC_PROD_WARPS;
+  if (a.stages < TC_PROD_WARPS || a.tpc < a.stages + TC_PROD_WARPS + 1)
+    return cudaErrorInvalidValue;
   const size_t smem = 1024 + (size_t)a.stages * STAGE + meta;
   auto kern = index_score_tc_kernel<DI, N>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
