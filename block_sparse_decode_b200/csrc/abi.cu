@@ -56,6 +56,8 @@ unsigned *device_error_word(cudaError_t *status) {
   return g_err_ptr[dev];
 }
 
+void set_last_error(const char *msg) { t_last_error = msg ? msg : ""; }
+
 int device_sm_count() {
   const int dev = current_device();
   if (dev < 0 || dev >= kMaxDevices) return 148;

@@ -14,6 +14,7 @@ namespace qsa {
 // Device address of this device's error word (set up once per device).
 unsigned *device_error_word(cudaError_t *status);
 int device_sm_count();
+void set_last_error(const char *msg);  // message returned by qsa_last_error()
 
 cudaError_t launch_append(const qsa_dims &d, const qsa_cache &c, int N, const int32_t *tok_seq,
                           const int32_t *tok_pos, const void *k_new, const void *v_new,

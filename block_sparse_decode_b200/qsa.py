@@ -29,7 +29,8 @@ QSA_ERR_TIMEOUT = 5
 # Symbols declared in include/qsa.h (checked by the test suite).
 EXPORTS = ("qsa_version", "qsa_last_error", "qsa_append", "qsa_index_score",
            "qsa_topk_workspace_size", "qsa_topk_select", "qsa_sparse_decode_workspace_size",
-           "qsa_sparse_decode", "qsa_merge", "qsa_check_device_errors")
+           "qsa_sparse_decode", "qsa_sparse_decode_static", "qsa_merge",
+           "qsa_check_device_errors")
 
 
 class QsaError(RuntimeError):
@@ -74,6 +75,7 @@ def lib() -> ctypes.CDLL:
         "qsa_topk_select": (I32, [I32, P, P, I32, I32, P, P, SZ, P]),
         "qsa_sparse_decode_workspace_size": (SZ, [DP, I32, I32, I32]),
         "qsa_sparse_decode": (I32, [DP, CP, I32, P, P, P, I32, I32, P, P, P, SZ, P]),
+        "qsa_sparse_decode_static": (I32, [DP, CP, I32, P, P, P, I32, I32, P, P, P]),
         "qsa_merge": (I32, [I32, I32, I32, I32, P, P, P, I32, P, P]),
         "qsa_check_device_errors": (I32, [P, ctypes.POINTER(I32)]),
     }
@@ -218,6 +220,20 @@ def qsa_sparse_decode(dims: QsaDims, cache: QsaCache, seq_lens, q, sel, k: int, 
                                    _ptr(lse_part, torch.float32, "lse_part"),
                                    _ptr(ws, None, "ws"), ws.numel() * ws.element_size(),
                                    _stream(stream)))
+
+
+def qsa_sparse_decode_static(dims: QsaDims, cache: QsaCache, seq_lens, q, sel, k: int, R: int,
+                             o_part, lse_part, stream=None):
+    """qsa_sparse_decode with the library's static device scratch (no
+    workspace, no allocation; see include/qsa.h for its limits)."""
+    B = int(seq_lens.shape[0])
+    _check(lib().qsa_sparse_decode_static(ctypes.byref(dims.c()), ctypes.byref(cache.c()), B,
+                                          _ptr(seq_lens, torch.int32, "seq_lens"),
+                                          _ptr(q, torch.bfloat16, "q"),
+                                          _ptr(sel, torch.int32, "sel"), int(k), int(R),
+                                          _ptr(o_part, torch.float32, "o_part"),
+                                          _ptr(lse_part, torch.float32, "lse_part"),
+                                          _stream(stream)))
 
 
 def qsa_merge(o_part, lse_part, out, lse_out=None, stream=None):

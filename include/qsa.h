@@ -187,6 +187,33 @@ qsa_status qsa_sparse_decode(const qsa_dims *dims, const qsa_cache *cache,
                              int32_t R, float *o_part, float *lse_part,
                              void *ws, size_t ws_bytes, qsa_stream_t stream);
 
+/* Size of the static device scratch of qsa_sparse_decode_static (32 MiB). */
+#define QSA_STATIC_SCRATCH_BYTES (32u << 20)
+
+/* qsa_sparse_decode without a workspace argument, for callers that cannot
+ * allocate device memory: a plain C host that only holds the input and
+ * output buffers it was handed, a process whose device memory is entirely
+ * owned by another allocator's pool (a raw cudaMalloc would fail or fragment
+ * it), or a latency-critical loop where cudaMalloc / cudaFree may
+ * synchronise the device. It has no counterpart on the page; it is an
+ * interface convenience of this library.
+ * Same arguments, results and errors as qsa_sparse_decode, except that the
+ * scratch lives in a fixed device array inside the library
+ * (QSA_STATIC_SCRATCH_BYTES per device, held by every device that loads the
+ * library until the process exits). A call whose scratch need
+ * (qsa_sparse_decode_workspace_size) exceeds that returns
+ * QSA_ERR_UNSUPPORTED. The call allocates nothing.
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture. All calls share the one array, which keeps the last call's
+ * contents (each call clears, on its stream, what must start at zero):
+ * calls whose executions overlap on the GPU race and corrupt each other. */
+qsa_status qsa_sparse_decode_static(const qsa_dims *dims, const qsa_cache *cache,
+                                    int32_t B, const int32_t *seq_lens,
+                                    const void *q, const int32_t *sel, int32_t k,
+                                    int32_t R, float *o_part, float *lse_part,
+                                    qsa_stream_t stream);
+
 /* LSE-weighted combine of R partial results (page sections "What the pull
  * request actually changes", second bullet, and "Questions worth answering
  * directly": partial attention results are merged afterwards).
