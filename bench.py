@@ -12,7 +12,7 @@ write larger than L2) before every timed step, outside the step's events.
 Prints one JSON line (rank 0). ``--impl reference`` times the CPU oracle on
 the same workload instead (a bounded sample per step).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 3]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload b8x256k]
     torchrun --nproc-per-node N bench.py --gpus N ...   (replicas, weak scaling)
 """
 
@@ -46,7 +46,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--config", type=int, default=3, choices=[2, 3, 4, 5])
+    ap.add_argument("--workload", default="b8x256k",
+                    choices=["b32x32k", "b8x256k", "ragged64", "steady128x64k"])
     ap.add_argument("--batch", type=int, default=None,
                     help="override the batch size (smaller profiling case)")
     ap.add_argument("--k", type=int, default=None)
@@ -146,22 +147,22 @@ def algorithmic_bytes(seq_lens, dims, k):
 
 def run_ours(args, rank, world, local_rank):
     from block_sparse_decode_b200 import qsa
-    from synth import make_custom, config_spec, seed_for
+    from synth import make_custom, preset_spec, seed_for
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    spec = config_spec(args.config)
+    spec = preset_spec(args.workload)
     k = args.k or spec["k"]
     R = args.R or spec["R"]
     lens = list(spec["seq_lens"])
     if args.batch:
         lens = (lens * ((args.batch + len(lens) - 1) // len(lens)))[:args.batch]
-    if args.config == 5:
+    if args.workload == "steady128x64k":
         lens = [spec["prefill"] + 1] * len(lens)
-    seed = seed_for(args.config) + 7919 * rank
+    seed = seed_for(args.workload) + 7919 * rank
     wl = make_custom(spec["dims"], lens, k=k, R=R, seed=seed, device=dev,
                      paged=spec["paged"], needles=spec["needles"], mixture=spec["mixture"],
-                     name=f"config{args.config}", config_id=args.config)
+                     name=args.workload)
     dims = qsa.QsaDims.of(wl.dims)
     B = wl.B
 
@@ -316,7 +317,7 @@ def run_ours(args, rank, world, local_rank):
     score_ms = kern_ms["index_score"]
     dec_ms = kern_ms["sparse_decode"]
     achieved = side_b / (score_ms / 1e3) / 1e9
-    traffic = profile_traffic("index_score.cu", "index_score_config3.md")
+    traffic = profile_traffic("index_score.cu", "index_score_b8x256k.md")
     attended = sum(min(4 * k, L) for L in wl.seq_lens)
     res = {
         "metric": METRIC,
@@ -331,7 +332,7 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": f"config{args.config}: B={B} x L={max(wl.seq_lens)} tokens, "
+        "config": {"workload": f"{args.workload}: B={B} x L={max(wl.seq_lens)} tokens, "
                                f"32q/4kv heads x 128, indexer 16x128, top-{k} blocks of 4, "
                                f"R={R}, paged P=64 (shuffled)",
                    "batch": B, "context": max(wl.seq_lens), "k": k, "R": R,
@@ -399,15 +400,16 @@ def cpu_baseline(sample, dims, k, R, budget_s=12.0):
 # ------------------------------------------------------------ reference arm
 
 def run_reference(args):
-    from synth import make_custom, config_spec, seed_for
+    from synth import make_custom, preset_spec, seed_for
     from block_sparse_decode_b200.qsa import QsaDims
 
-    spec = config_spec(args.config)
+    spec = preset_spec(args.workload)
     k = args.k or spec["k"]
     R = args.R or spec["R"]
-    L = max(spec["seq_lens"]) if args.config != 5 else spec["prefill"] + 1
+    L = (max(spec["seq_lens"]) if args.workload != "steady128x64k"
+         else spec["prefill"] + 1)
     B = len(spec["seq_lens"]) if not args.batch else args.batch
-    wl = make_custom(spec["dims"], [L], k=k, R=R, seed=seed_for(args.config), device="cpu",
+    wl = make_custom(spec["dims"], [L], k=k, R=R, seed=seed_for(args.workload), device="cpu",
                      paged=spec["paged"], needles=spec["needles"], mixture=spec["mixture"])
     K, V, X = wl.seq_tokens(0)
     sample = dict(K=K, V=V, X=X, q=wl.q[0], q_idx=wl.q_idx[0], w=wl.w[0], L=L)
@@ -425,7 +427,7 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": {"workload": f"config{args.config}: one {L}-token sequence per step "
+            "config": {"workload": f"{args.workload}: one {L}-token sequence per step "
                                    f"(B={B} workload sampled), top-{k}, R={R}",
                        "batch": 1, "context": L, "k": k, "R": R},
             "cpu_baseline": {"value": v, "unit": "seqs/s", "cores": _threads(),

@@ -10,8 +10,8 @@ sides always see the same bytes.
 from .workloads import (  # noqa: F401
     Dims,
     Workload,
-    CONFIG_IDS,
-    config_spec,
+    PRESETS,
+    preset_spec,
     make_workload,
     make_custom,
     step_queries,

@@ -8,14 +8,18 @@ still worth your time" (262,144-token native context). The page fixes no head
 counts or value distributions; the five presets below are this library's
 test and benchmark workloads:
 
-  1  tiny: B=2, L = 4099 and 1500, 8 q / 2 kv heads, indexer 4 x 64,
-     contiguous cache, 3 planted needle blocks per sequence, k=512, R=2
-  2  B=32 x 32,768 tokens, 32 q / 4 kv heads, indexer 16 x 128, paged (P=64,
-     shuffled pages), k=512, R=1
-  3  B=8 x 262,144 tokens, heads as 2, indexer keys and K drawn from a
-     90/10 mixture (N(0,I), N(0,I) + 3u), 8 planted needles, k=512, R=4
-  4  B=64 ragged, L log-uniform in [1,024, 262,144], k=512, R in {1,2,4,8}
-  5  B=128, 65,536-token prefill then 64 decode steps, k in {256,512,1024}, R=4
+  tiny           B=2, L = 4099 and 1500, 8 q / 2 kv heads, indexer 4 x 64,
+                 contiguous cache, 3 planted needle blocks per sequence,
+                 k=512, R=2
+  b32x32k        B=32 x 32,768 tokens, 32 q / 4 kv heads, indexer 16 x 128,
+                 paged (P=64, shuffled pages), k=512, R=1
+  b8x256k        B=8 x 262,144 tokens, heads as b32x32k, indexer keys and K
+                 drawn from a 90/10 mixture (N(0,I), N(0,I) + 3u), 8 planted
+                 needles, k=512, R=4
+  ragged64       B=64 ragged, L log-uniform in [1,024, 262,144], k=512,
+                 R in {1,2,4,8}
+  steady128x64k  B=128, 65,536-token prefill then 64 decode steps,
+                 k in {256,512,1024}, R=4
 
 Everything is drawn in fp32 from one ``torch.Generator`` per tensor stream and
 rounded to bf16 by torch's round-to-nearest-even conversion. Nothing in this
@@ -29,7 +33,7 @@ from dataclasses import dataclass, field
 
 import torch
 
-CONFIG_IDS = (1, 2, 3, 4, 5)
+PRESETS = ("tiny", "b32x32k", "b8x256k", "ragged64", "steady128x64k")
 BASE_SEED = 20261202
 
 # RNG stream ids, in the fixed order the tensors are drawn.
@@ -37,8 +41,9 @@ _S_LENS, _S_K, _S_V, _S_KIDX, _S_Q, _S_QIDX, _S_W, _S_PAGES, _S_NEEDLE, _S_MIX =
 _S_STEP = 100  # + step index: per-step queries of the append workload
 
 
-def seed_for(config_id: int) -> int:
-    return BASE_SEED + int(config_id)
+def seed_for(preset: str) -> int:
+    """Base seed of a preset (fixed, so every run draws the same bytes)."""
+    return BASE_SEED + 1 + PRESETS.index(preset)
 
 
 @dataclass(frozen=True)
@@ -76,7 +81,6 @@ class Workload:
     """
 
     name: str
-    config_id: int
     seed: int
     dims: Dims
     seq_lens: list
@@ -179,7 +183,7 @@ def _plant_needles(wl: Workload, n_needles: int, gen_device):
     wl.needles = needles
 
 
-def _lens_config4(seed, device):
+def _lens_ragged64(seed):
     g = _gen("cpu", seed, _S_LENS)
     u = torch.rand(64, generator=g, dtype=torch.float64)
     lo, hi = math.log(1024.0), math.log(262144.0)
@@ -199,31 +203,30 @@ def _lens_config4(seed, device):
     return lens
 
 
-def config_spec(config_id: int) -> dict:
+def preset_spec(preset: str) -> dict:
     """Sizes of a preset, without drawing anything."""
-    if config_id == 1:
+    if preset == "tiny":
         return dict(dims=DIMS_TINY, seq_lens=[4099, 1500], k=512, R=2, paged=False,
                     needles=3, mixture=False)
-    if config_id == 2:
+    if preset == "b32x32k":
         return dict(dims=DIMS_FULL, seq_lens=[32768] * 32, k=512, R=1, paged=True,
                     needles=0, mixture=False)
-    if config_id == 3:
+    if preset == "b8x256k":
         return dict(dims=DIMS_FULL, seq_lens=[262144] * 8, k=512, R=4, paged=True,
                     needles=8, mixture=True)
-    if config_id == 4:
-        return dict(dims=DIMS_FULL, seq_lens=_lens_config4(seed_for(4), "cpu"), k=512, R=4,
+    if preset == "ragged64":
+        return dict(dims=DIMS_FULL, seq_lens=_lens_ragged64(seed_for(preset)), k=512, R=4,
                     paged=True, needles=0, mixture=False, R_sweep=(1, 2, 4, 8))
-    if config_id == 5:
+    if preset == "steady128x64k":
         return dict(dims=DIMS_FULL, seq_lens=[65537] * 128, cap_lens=[65536 + 64] * 128,
                     k=512, R=4, paged=True, needles=0, mixture=False,
                     k_sweep=(256, 512, 1024), prefill=65536, steps=64)
-    raise ValueError(f"unknown config {config_id}")
+    raise ValueError(f"unknown preset {preset!r}; known: {', '.join(PRESETS)}")
 
 
 def make_custom(dims: Dims, seq_lens, k: int, R: int, seed: int, device="cpu",
                 paged: bool = True, needles: int = 0, mixture: bool = False,
-                cap_lens=None, name: str = "custom", config_id: int = 0,
-                pool_slack_pages: int = 0) -> Workload:
+                cap_lens=None, name: str = "custom", pool_slack_pages: int = 0) -> Workload:
     """Draw a workload of arbitrary size (used by the presets and by small tests)."""
     device = torch.device(device)
     seq_lens = [int(x) for x in seq_lens]
@@ -250,7 +253,7 @@ def make_custom(dims: Dims, seq_lens, k: int, R: int, seed: int, device="cpu",
     w = torch.rand((B, dims.Hi), generator=_gen(device, seed, _S_W), device=device,
                    dtype=torch.float32)
     bt, num_pages = _page_table(cap_lens, dims.P, _gen(device, seed, _S_PAGES), device, paged)
-    wl = Workload(name=name, config_id=config_id, seed=seed, dims=dims, seq_lens=seq_lens,
+    wl = Workload(name=name, seed=seed, dims=dims, seq_lens=seq_lens,
                   cap_lens=cap_lens, k=k, R=R, tok_off=tok_off, k_tok=k_tok, v_tok=v_tok,
                   kidx_tok=kidx_tok, q=q, q_idx=q_idx, w=w, block_table=bt,
                   num_pages=num_pages + pool_slack_pages)
@@ -259,14 +262,13 @@ def make_custom(dims: Dims, seq_lens, k: int, R: int, seed: int, device="cpu",
     return wl
 
 
-def make_workload(config_id: int, device="cpu", seed: int | None = None) -> Workload:
-    """Draw preset ``config_id`` (1..5) on ``device``."""
-    spec = config_spec(config_id)
-    seed = seed_for(config_id) if seed is None else seed
+def make_workload(preset: str, device="cpu", seed: int | None = None) -> Workload:
+    """Draw one of ``PRESETS`` on ``device``."""
+    spec = preset_spec(preset)
+    seed = seed_for(preset) if seed is None else seed
     wl = make_custom(spec["dims"], spec["seq_lens"], spec["k"], spec["R"], seed, device,
                      paged=spec["paged"], needles=spec["needles"], mixture=spec["mixture"],
-                     cap_lens=spec.get("cap_lens"), name=f"config{config_id}",
-                     config_id=config_id)
+                     cap_lens=spec.get("cap_lens"), name=preset)
     wl.extra = {k: v for k, v in spec.items()
                 if k in ("R_sweep", "k_sweep", "prefill", "steps")}
     return wl

@@ -57,7 +57,7 @@ def _check_seq(run, b, L=None, q=None, q_idx=None, w=None, full=True):
 
 @pytest.mark.parametrize("R", [2, 1, 3, 8])
 def test_tiny_preset_end_to_end(R):
-    wl = make_workload(1, device=DEV)
+    wl = make_workload("tiny", device=DEV)
     run = GpuRun(wl, R=R)
     run.step()
     for b in range(wl.B):
@@ -288,8 +288,8 @@ def _sampled(wl, n):
     return idx
 
 
-def test_preset2_full_size():
-    wl = make_workload(2, device=DEV)
+def test_b32x32k_full_size():
+    wl = make_workload("b32x32k", device=DEV)
     run = GpuRun(wl)
     run.step()
     for b in _sampled(wl, 3):
@@ -298,8 +298,8 @@ def test_preset2_full_size():
     torch.cuda.empty_cache()
 
 
-def test_preset3_full_size_split_equals_unsplit():
-    wl = make_workload(3, device=DEV)
+def test_b8x256k_split_equals_unsplit():
+    wl = make_workload("b8x256k", device=DEV)
     run = GpuRun(wl)
     run.step()
     for b in _sampled(wl, 2):
@@ -318,8 +318,8 @@ def test_preset3_full_size_split_equals_unsplit():
 
 
 @pytest.mark.parametrize("R", [1, 2, 4, 8])
-def test_preset4_ragged_full_size(R):
-    wl = make_workload(4, device=DEV)
+def test_ragged64_full_size(R):
+    wl = make_workload("ragged64", device=DEV)
     run = GpuRun(wl, R=R)
     run.step()
     lens = np.array(wl.seq_lens)
@@ -333,8 +333,8 @@ def test_preset4_ragged_full_size(R):
     torch.cuda.empty_cache()
 
 
-def test_preset5_append_steps():
-    wl = make_workload(5, device=DEV)
+def test_steady128x64k_append_steps():
+    wl = make_workload("steady128x64k", device=DEV)
     spec_prefill, steps = wl.extra["prefill"], wl.extra["steps"]
     for k in (256, 512, 1024):
         run = GpuRun(wl, k=k, prefill=[spec_prefill] * wl.B)

@@ -145,8 +145,8 @@ def test_all_zero_index_keys_select_first_blocks():
     assert oracle.topk_blocks(s, 512).tolist() == list(range(512))
 
 
-def test_planted_needles_always_selected_tiny_config():
-    wl = make_workload(1, device="cpu")
+def test_planted_needles_always_selected_tiny_preset():
+    wl = make_workload("tiny", device="cpu")
     for b in range(wl.B):
         K, V, X = wl.seq_tokens(b)
         res = oracle.decode_sequence(bits(X), bits(K), bits(V), bits(wl.q[b]), bits(wl.q_idx[b]),
@@ -227,7 +227,7 @@ def test_full_selection_equals_dense_attention_loops():
 
 def test_full_selection_equals_sdpa_fp64():
     # the tiny preset's 1500-token sequence has 375 < 512 blocks: all selected
-    wl = make_workload(1, device="cpu")
+    wl = make_workload("tiny", device="cpu")
     b, L = 1, wl.seq_lens[1]
     K, V, X = wl.seq_tokens(b)
     res = oracle.decode_sequence(bits(X), bits(K), bits(V), bits(wl.q[b]), bits(wl.q_idx[b]),
