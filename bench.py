@@ -137,6 +137,26 @@ class ClockSampler:
                 "samples": len(rows)}
 
 
+def replica_seed(preset: str, rank: int) -> int:
+    """Seed of the replica on ``rank``: every GPU draws its own batch."""
+    from synth import seed_for
+    return seed_for(preset) + 7919 * rank
+
+
+def max_over_ranks(x: float, device) -> float:
+    """The largest ``x`` over all ranks (the job is as slow as its slowest
+    replica); the identity on a single process."""
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    if torch.distributed.is_initialized() and torch.distributed.get_world_size() > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(world: int, units_per_rank: int, ms_per_step: float) -> float:
+    """Whole-job throughput: units processed by all ranks per second."""
+    return world * units_per_rank / (ms_per_step / 1e3)
+
+
 def algorithmic_bytes(seq_lens, dims, k):
     side = sum(((L + 3) // 4) * dims.di * 2 for L in seq_lens)
     kv = sum(min(4 * k, L) * dims.Hkv * dims.D * 2 * 2 for L in seq_lens)
@@ -159,7 +179,7 @@ def run_ours(args, rank, world, local_rank):
         lens = (lens * ((args.batch + len(lens) - 1) // len(lens)))[:args.batch]
     if args.workload == "steady128x64k":
         lens = [spec["prefill"] + 1] * len(lens)
-    seed = seed_for(args.workload) + 7919 * rank
+    seed = replica_seed(args.workload, rank)
     wl = make_custom(spec["dims"], lens, k=k, R=R, seed=seed, device=dev,
                      paged=spec["paged"], needles=spec["needles"], mixture=spec["mixture"],
                      name=args.workload)
@@ -267,10 +287,7 @@ def run_ours(args, rank, world, local_rank):
         torch.distributed.barrier()
     qsa.qsa_check_device_errors()
 
-    tot = torch.tensor([sum(step_ms)], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(tot, op=torch.distributed.ReduceOp.MAX)
-    ms_per_step = float(tot.item()) / args.steps
+    ms_per_step = max_over_ranks(sum(step_ms), dev) / args.steps
 
     # per-kernel durations: each call in its own graph, timed like the step
     # (L2 flushed before every launch, events on the launching stream)
@@ -304,11 +321,8 @@ def run_ours(args, rank, world, local_rank):
             s1.synchronize()
             if i >= max(3, args.warmup):
                 e_ms.append(s0.elapsed_time(s1))
-        et = torch.tensor([sum(e_ms)], dtype=torch.float64, device=dev)
-        if world > 1:
-            torch.distributed.all_reduce(et, op=torch.distributed.ReduceOp.MAX)
-        e_step = float(et.item()) / args.steps
-        e2e = {"value": world * B / (e_step / 1e3), "unit": "seqs/s",
+        e_step = max_over_ranks(sum(e_ms), dev) / args.steps
+        e2e = {"value": job_rate(world, B, e_step), "unit": "seqs/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": e_step, "api": "eager qsa_* calls through the ctypes binding"}
 
@@ -321,7 +335,7 @@ def run_ours(args, rank, world, local_rank):
     attended = sum(min(4 * k, L) for L in wl.seq_lens)
     res = {
         "metric": METRIC,
-        "value": world * B / (ms_per_step / 1e3),
+        "value": job_rate(world, B, ms_per_step),
         "unit": "seqs/s",
         "n_gpus": world,
         "steps": args.steps,
@@ -339,7 +353,7 @@ def run_ours(args, rank, world, local_rank):
                    "l2": "flushed before every timed step (512 MiB write, then 512 MiB read)",
                    "step": "CUDA graph of append+score+topk+decode+merge",
                    "parallelism": f"replicas x{world}"},
-        "attended_tokens_per_s": world * attended / (ms_per_step / 1e3),
+        "attended_tokens_per_s": job_rate(world, attended, ms_per_step),
         "roofline": {"bound": "hbm", "kernel": "qsa_index_score", "achieved": achieved,
                      "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_source": peak_kind,
