@@ -97,11 +97,13 @@ __device__ __forceinline__ void compress_block(const AppendArgs &a, int tok, int
 }
 
 __global__ void __launch_bounds__(256) append_tokens_kernel(AppendArgs a) {
+  pdl_wait();
   const int tok = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (tok < a.N) write_token(a, tok, threadIdx.x & 31);
 }
 
 __global__ void __launch_bounds__(256) append_compress_kernel(AppendArgs a) {
+  pdl_wait();
   const int tok = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (tok < a.N) compress_block(a, tok, threadIdx.x & 31);
 }
@@ -112,8 +114,10 @@ constexpr int SMALL_WARPS = 32;
 constexpr int SMALL_MAX_N = 4 * SMALL_WARPS;
 __global__ void __launch_bounds__(SMALL_WARPS * 32) append_small_kernel(AppendArgs a) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_wait();
   for (int tok = warp; tok < a.N; tok += SMALL_WARPS) write_token(a, tok, lane);
   __syncthreads();
+  pdl_trigger();
   for (int tok = warp; tok < a.N; tok += SMALL_WARPS) compress_block(a, tok, lane);
 }
 
@@ -143,17 +147,12 @@ cudaError_t launch_append(const qsa_dims &d, const qsa_cache &c, int N, const in
   a.x_vec = d.di / 8;
   a.di = d.di;
   a.err = err;
-  if (N <= SMALL_MAX_N) {
-    append_small_kernel<<<1, SMALL_WARPS * 32, 0, st>>>(a);
-    return cudaGetLastError();
-  }
+  if (N <= SMALL_MAX_N) return launch_pdl(append_small_kernel, 1, SMALL_WARPS * 32, 0, st, a);
   const int threads = 256, per_block = threads / 32;
   const int blocks = (N + per_block - 1) / per_block;
-  append_tokens_kernel<<<blocks, threads, 0, st>>>(a);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(append_tokens_kernel, blocks, threads, 0, st, a);
   if (e != cudaSuccess) return e;
-  append_compress_kernel<<<blocks, threads, 0, st>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(append_compress_kernel, blocks, threads, 0, st, a);
 }
 
 }  // namespace qsa

@@ -23,6 +23,18 @@ __device__ __forceinline__ void raise_err(unsigned *err, unsigned bit) {
   atomicOr(err, bit);
 }
 
+// ---------------------------------------------------------------- PDL
+// Every kernel is launched as a programmatic dependent of the kernel before
+// it on the stream (launch_pdl). It may run its prologue while that kernel
+// finishes, but every CTA executes pdl_wait() before it touches anything an
+// earlier kernel wrote (and before it exits), so the completion of a grid
+// still implies the completion of all work before it. pdl_trigger() lets the
+// next kernel start launching; CTAs call it once their main work is done.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
+
 // ---------------------------------------------------------------- bf16
 
 __device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }

@@ -68,8 +68,7 @@ extern "C" qsa_status qsa_sparse_decode_static(const qsa_dims *dims, const qsa_c
       qsa::set_last_error(msg);
       return QSA_ERR_CUDA;
     }
-    // the regular entry point does every argument check and clears, on the
-    // stream, the part of the scratch that must start at zero
+    // the regular entry point does every argument check
     return qsa_sparse_decode(dims, cache, B, seq_lens, q, sel, k, R, o_part, lse_part, scratch,
                              qsa::kStaticScratchBytes, stream);
   } catch (...) {

@@ -366,6 +366,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // everything above reads inputs only; the side cache and the per-token
+  // indexer keys come from the append kernel before this one
+  pdl_wait();
   const uint32_t tmem = ctl.tmem_base;
   volatile int *abort_flag = &ctl.abort_flag;
 
@@ -512,6 +515,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   }
 
   __syncthreads();
+  pdl_trigger();
   if (ctl.abort_flag) {
     // drain: stages whose copies were issued but never consumed, MMAs whose
     // accumulators were never read
@@ -601,8 +605,7 @@ cudaError_t launch_tc_t(const qsa_cache &c, TcArgs a, cudaStream_t st) {
   const long long tiles_bound = (long long)a.B * ((a.ld + TC_M - 1) / TC_M);
   const int grid =
       (int)std::max<long long>(1, std::min<long long>(device_sm_count(), tiles_bound));
-  kern<<<grid, TC_THREADS, smem, st>>>(side_map, q_map, a);
-  return cudaGetLastError();
+  return launch_pdl(kern, grid, TC_THREADS, smem, st, side_map, q_map, a);
 }
 
 }  // namespace

@@ -11,6 +11,24 @@
 
 namespace qsa {
 
+// Launch `kern` as a programmatic dependent of the previous kernel on the
+// stream (see pdl_wait / pdl_trigger in common.cuh).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<Args &&>(args)...);
+}
+
 // Device address of this device's error word (set up once per device).
 unsigned *device_error_word(cudaError_t *status);
 int device_sm_count();
@@ -30,7 +48,6 @@ constexpr int TOPK_MAX_KEYS_PER_CTA = 49152;  // 192 KiB of keys per CTA
 cudaError_t launch_topk(int B, const int32_t *seq_lens, const float *scores, int ld, int k,
                         int32_t *sel, unsigned *err, cudaStream_t st);
 
-int decode_num_slots(int k, int R);
 size_t decode_ws_bytes(const qsa_dims &d, int B, int k, int R);
 cudaError_t launch_sparse_decode(const qsa_dims &d, const qsa_cache &c, int B,
                                  const int32_t *seq_lens, const void *q, const int32_t *sel,

@@ -19,6 +19,7 @@ __global__ void __launch_bounds__(256) merge_kernel(int R, int rows, int D, cons
                                                     const float *lse_part, void *out,
                                                     int out_is_bf16, float *lse_out) {
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  pdl_wait();
   if (row >= rows) return;
   float M = -INFINITY;
   for (int r = 0; r < R; ++r) M = fmaxf(M, lse_part[(size_t)r * rows + row]);
@@ -72,9 +73,8 @@ cudaError_t launch_merge(int R, int B, int Hq, int D, const float *o_part, const
                          void *out, int out_is_bf16, float *lse_out, cudaStream_t st) {
   const int rows = B * Hq;
   if (rows == 0) return cudaSuccess;
-  merge_kernel<<<(rows + 7) / 8, 256, 0, st>>>(R, rows, D, o_part, lse_part, out, out_is_bf16,
-                                               lse_out);
-  return cudaGetLastError();
+  return launch_pdl(merge_kernel, (rows + 7) / 8, 256, 0, st, R, rows, D, o_part, lse_part, out,
+                    out_is_bf16, lse_out);
 }
 
 }  // namespace qsa

@@ -9,404 +9,555 @@
 // the slices are the block ranges [floor(r*nb/R), floor((r+1)*nb/R)) of one
 // GPU and the one selection serves all of them.
 //
-// Work decomposition: the selected blocks of slice r form a contiguous run of
-// the (ascending) selection list; each run is cut into chunks of DC_BLOCKS
-// blocks. A CTA = (chunk slot, KV head, sequence); the slot count per
-// (sequence, KV head) is ceil(k / DC_BLOCKS) + R, an upper bound on the
-// chunks over all slices, so the grid is fixed on the host while the chunk
-// boundaries are found on the device. Each warp gathers 4 blocks (16 tokens
-// x 256 B of K and of V for its KV head) with 16-byte cp.async into swizzled
-// shared memory, then runs S^T = K Q^T and O^T += V^T P^T on tensor cores
-// (m16n8k16: the 16 MMA rows are tokens / head dims, the 8 columns are the
-// GQA group's query heads, so no MMA row is wasted) with an online softmax
-// in fp32 (exp2 domain). P^T moves from the accumulator layout to the B
-// operand layout with movmatrix. The warps of a CTA merge through shared
-// memory into one chunk partial (scratch, L2-resident); the CTA that
-// finishes a slice last (per-slice arrival counter, zeroed by the call)
-// merges that slice's chunks into its R partial. Slot 0 of each (sequence,
-// KV head) writes the empty slices. One kernel launch plus a small memset.
+// Work decomposition. The selected blocks of slice r are a contiguous run of
+// the ascending selection list; the run is cut into tiles of 4 blocks (16
+// tokens), so a tile never spans two slices. The sequence's NT tiles, slice
+// after slice, are split into ncb contiguous ranges, one per CTA (grid = ncb x
+// head groups x B, ncb picked on the host so that about two CTAs per SM are in
+// flight). Each CTA has one warp per KV head (up to 4); all warps walk the
+// same tiles, so the heads of a token (1 KiB of K, 1 KiB of V at 4 KV heads)
+// are read at about the same time.
 //
-// Roofline: HBM-bound; algorithmic bytes = tokens * Hkv * D * 2 * 2 per
-// sequence (each selected token's K and V rows read once).
+// Per CTA: (1) copy the selection row to shared memory and read L_b; (2) one
+// warp builds the slice table (start and count of each slice's run, tile
+// prefix); (3) all threads look up the physical row of every block of the
+// CTA's range in one pass of block-table loads; (4) each warp streams its
+// head's tiles (8 KiB of K+V per tile) through an ST-stage cp.async ring into
+// XOR-swizzled shared memory and runs S^T = K Q^T and O^T += V^T P^T on
+// tensor cores (m16n8k16: the 16 MMA rows are tokens / head dims, the 8
+// columns the GQA group's query heads) with an online softmax in fp32 (exp2
+// domain); P^T moves from the accumulator layout to the B-operand layout with
+// movmatrix. (5) At the end of each slice's run the warp holds the partial of
+// its range. A slice that lies inside one CTA's range is written to o_part /
+// lse_part directly; only the first and the last slice of a range can be
+// shared with neighbouring CTAs, and their partials go to scratch, keyed by
+// CTA + slice (distinct for all pairs, since ranges and slices are both
+// ordered). (6) A second, small kernel, launched as a programmatic dependent
+// of the first, combines the partials of each shared slice once all streaming
+// is done (every load of a row batched, so it costs a couple of L2 round
+// trips); no atomics, fences or counters are needed.
+//
+// Roofline: HBM-bound; algorithmic bytes = selected tokens * Hkv * D * 2 * 2
+// (each selected token's K and V rows read once).
 #include "common.cuh"
 #include "launch.h"
 
 namespace qsa {
 namespace {
 
-constexpr int DC_WARPS = 4;
-constexpr int DC_BPW = 4;                       // blocks per warp (one 16-token MMA tile)
-constexpr int DC_BLOCKS = DC_WARPS * DC_BPW;    // blocks per CTA chunk
-constexpr int DC_D = 128;                       // head dim
-constexpr int DC_ROWB = DC_D * 2;               // bytes per K/V row
-constexpr int DC_TOK = DC_BPW * 4;              // token rows per warp
-constexpr int DC_WARP_SMEM = 2 * DC_TOK * DC_ROWB;  // K + V tiles per warp
-constexpr int DC_SEL_SMEM = 1024;               // selection entries staged in smem
+constexpr int DV_D = 128;                    // head dim
+constexpr int DV_ROWB = DV_D * 2;            // bytes per K or V row of one head
+constexpr int DV_TOK = 16;                   // tokens per tile (MMA rows)
+constexpr int DV_STAGE = 2 * DV_TOK * DV_ROWB;  // K tile + V tile of one head: 8 KiB
+constexpr int DV_WARPS = 4;                  // KV heads per CTA
+constexpr int DV_TBL_BLOCKS = 1024;          // blocks per CTA range (host guarantees)
+constexpr int DV_TBL_TILES = DV_TBL_BLOCKS / 4;
+constexpr int DV_RMAX = 64;
+constexpr int DV_CTAS_PER_SM = 2;
+constexpr int DV_SLOTS = DV_CTAS_PER_SM * 148;  // CTAs in flight on a B200
+constexpr size_t DV_SMEM_LIMIT = 113 * 1024;    // shared memory per CTA so that two fit an SM
+constexpr int DV_CB_ROWS = 8;                   // query-head rows per combine CTA
+constexpr int DV_CB_BATCH = 8;                  // records loaded together by the combine
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 
 struct DecodeArgs {
   const __nv_bfloat16 *k_pool, *v_pool, *q;
   const int32_t *block_table, *seq_lens, *sel;
-  float *ws_o, *ws_lse;      // [B, Hkv, nslots, G, D], [B, Hkv, nslots, G]
-  unsigned *ws_cnt;          // [B, Hkv, R] chunks of each slice finished so far
   float *o_part, *lse_part;  // [R, B, Hq, D], [R, B, Hq]
-  int B, Hq, Hkv, G, P, max_pages, num_pages, k, R, nslots;
+  float *rec_o, *rec_lse;    // [B, rb, Hq, D], [B, rb, Hq]: partials of shared slices
+  int2 *span;                // [B, R]: contributors (c_lo, c_hi) of a shared slice
+  int B, Hq, Hkv, G, P, max_pages, num_pages, k, k_pad, R, ncb, rb;
+  int ring_bytes;            // DV_WARPS * ST * DV_STAGE
   float scale_log2;
   unsigned *err;
 };
+
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(dst), "l"(src) : "memory");
+}
 
 // First position in the ascending list s[0..n) whose value is >= v.
 __device__ __forceinline__ int lower_bound(const int32_t *s, int n, int v) {
   int lo = 0, hi = n;
   while (lo < hi) {
-    int mid = (lo + hi) >> 1;
+    const int mid = (lo + hi) >> 1;
     if (s[mid] < v) lo = mid + 1; else hi = mid;
   }
   return lo;
 }
 
-// Chunk layout of one sequence, computed by one full warp. Lane l holds
-// slices l and l + 32: the run of slice r in the selection list starts at
-// st and holds ct blocks; its ch = ceil(ct / DC_BLOCKS) chunks use slots
-// [ex, ex + ch) (slots are numbered slice after slice).
-struct SliceTable {
-  int st[2], ct[2], ch[2], ex[2];
-};
-
-// `s` is the sequence's selection row (ascending, first kb = min(k, nb) valid).
-__device__ SliceTable slice_table(const DecodeArgs &a, int b, const int32_t *s) {
-  const int lane = threadIdx.x & 31;
-  const int L = a.seq_lens[b];
-  const int nb = L <= 0 ? 0 : (L + 3) >> 2;
-  const int kb = min(a.k, nb);
-  SliceTable t;
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int r = lane + 32 * h;
-    t.st[h] = t.ct[h] = t.ch[h] = 0;
-    if (r < a.R) {
-      const int lo = (int)(((long long)r * nb) / a.R);
-      const int hi = (int)(((long long)(r + 1) * nb) / a.R);
-      t.st[h] = lower_bound(s, kb, lo);
-      t.ct[h] = lower_bound(s, kb, hi) - t.st[h];
-      t.ch[h] = (t.ct[h] + DC_BLOCKS - 1) / DC_BLOCKS;
-    }
+// Slice holding tile v: the largest r < R with pre[r] <= v (pre ascending,
+// pre[R] = NT > v).
+__device__ __forceinline__ int slice_of_tile(const int *pre, int R, int v) {
+  int lo = 0, hi = R - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (pre[mid] <= v) lo = mid; else hi = mid - 1;
   }
-  int inc0 = t.ch[0], inc1 = t.ch[1];
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    int y0 = __shfl_up_sync(0xffffffffu, inc0, o), y1 = __shfl_up_sync(0xffffffffu, inc1, o);
-    if (lane >= o) { inc0 += y0; inc1 += y1; }
-  }
-  inc1 += __shfl_sync(0xffffffffu, inc0, 31);
-  t.ex[0] = inc0 - t.ch[0];
-  t.ex[1] = inc1 - t.ch[1];
-  return t;
+  return lo;
 }
 
-struct SliceInfo {
-  int r, start, count, slot0, nchunks;
-};
-
-// The slice holding chunk slot `slot` (r = -1 if the slot is unused).
-__device__ SliceInfo slice_of_slot(const SliceTable &t, int R, int slot) {
-  const int lane = threadIdx.x & 31;
-  SliceInfo out{-1, 0, 0, 0, 0};
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const unsigned hit = __ballot_sync(0xffffffffu, lane + 32 * h < R && t.ch[h] > 0 &&
-                                                        slot >= t.ex[h] &&
-                                                        slot < t.ex[h] + t.ch[h]);
-    if (hit && out.r < 0) {
-      const int src = __ffs(hit) - 1;
-      out.r = src + 32 * h;
-      out.start = __shfl_sync(0xffffffffu, t.st[h], src);
-      out.count = __shfl_sync(0xffffffffu, t.ct[h], src);
-      out.slot0 = __shfl_sync(0xffffffffu, t.ex[h], src);
-      out.nchunks = __shfl_sync(0xffffffffu, t.ch[h], src);
-    }
-  }
-  return out;
+// CTA whose tile range [floor(c*NT/ncb), floor((c+1)*NT/ncb)) holds tile v.
+__device__ __forceinline__ int cta_of_tile(int v, int NT, int ncb) {
+  return (int)(((long long)(v + 1) * ncb + NT - 1) / NT) - 1;
 }
 
-__global__ void __launch_bounds__(DC_WARPS * 32) sparse_decode_kernel(DecodeArgs a) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  __shared__ int s_info[5];  // slice r, first selection index, blocks, slot0, chunks
-  __shared__ float s_m[DC_WARPS][8], s_l[DC_WARPS][8];
-  __shared__ int s_last;
-  __shared__ int32_t s_sel[DC_SEL_SMEM];
-  const int slot = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  // the selection row, staged once so that the slice searches run in shared memory
-  const int32_t *sel_row = a.sel + (size_t)b * a.k;
-  if (a.k <= DC_SEL_SMEM) {
-    for (int i = threadIdx.x; i < a.k; i += blockDim.x) s_sel[i] = sel_row[i];
-    sel_row = s_sel;
-  }
-  __syncthreads();
-  if (warp == 0) {
-    const SliceTable tab = slice_table(a, b, sel_row);
-    const SliceInfo si = slice_of_slot(tab, a.R, slot);
-    if (lane == 0) {
-      if (si.r < 0) {
-        s_info[2] = 0;
-      } else {
-        const int c = slot - si.slot0;
-        s_info[0] = si.r;
-        s_info[1] = si.start + c * DC_BLOCKS;
-        s_info[2] = min(DC_BLOCKS, si.count - c * DC_BLOCKS);
-        s_info[3] = si.slot0;
-        s_info[4] = si.nchunks;
-      }
-    }
-    if (slot == 0) {
-      // slices that own no selected block: O_r = 0, LSE_r = -inf
-      if (lane == 0 && g == 0 && a.seq_lens[b] < 0) raise_err(a.err, ERR_LEN);
+// Online-softmax state of one warp: heads 2tq, 2tq+1 of the group (tq = lane
+// & 3), accumulators O^T in the m16n8 layout (8 tiles of 16 head dims).
+struct Acc {
+  float m0, m1, l0, l1;
+  float o[8][4];
+  __device__ __forceinline__ void reset() {
+    m0 = m1 = -INFINITY;
+    l0 = l1 = 0.f;
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        unsigned empty = __ballot_sync(0xffffffffu, lane + 32 * hh < a.R && tab.ch[hh] == 0);
-        while (empty) {
-          const int r = __ffs(empty) - 1 + 32 * hh;
-          empty &= empty - 1;
-          for (int h = 0; h < a.G; ++h) {
-            const size_t row = ((size_t)r * a.B + b) * a.Hq + g * a.G + h;
-            *reinterpret_cast<float4 *>(a.o_part + row * DC_D + lane * 4) =
-                make_float4(0.f, 0.f, 0.f, 0.f);
-            if (lane == 0) a.lse_part[row] = -INFINITY;
-          }
-        }
-      }
-    }
+    for (int mt = 0; mt < 8; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
   }
-  __syncthreads();
-  const int count = s_info[2];
-  if (count <= 0) return;  // slot beyond this sequence's chunks
-  const int first = s_info[1];
-  const int L = a.seq_lens[b];
-  const int nb = (L + 3) >> 2;
+};
 
-  // ---- gather: this warp's blocks [warp*DC_BPW, (warp+1)*DC_BPW) of the chunk
-  unsigned char *wsm = smem + warp * DC_WARP_SMEM;
-  const uint32_t ks_base = smem_u32(wsm), vs_base = ks_base + DC_TOK * DC_ROWB;
-  int my_row0 = 0;       // lane < DC_BPW: first pool row of block `lane`
-  unsigned my_bits = 0;  // lane < DC_BPW: valid-token bits of that block
-  if (lane < DC_BPW) {
-    const int bi = warp * DC_BPW + lane;
-    if (bi < count) {
-      const int j = sel_row[first + bi];
-      if (j < 0 || j >= nb) {
-        raise_err(a.err, ERR_SEL);
-      } else {
-        const int col = (4 * j) / a.P;
-        if (col >= a.max_pages) {
-          raise_err(a.err, ERR_BT);
-        } else {
-          const int page = a.block_table[(size_t)b * a.max_pages + col];
-          if (page < 0 || page >= a.num_pages) {
-            raise_err(a.err, ERR_PAGE);
-          } else {
-            my_row0 = page * a.P + (4 * j) % a.P;
-            const int nv = min(4, L - 4 * j);
-            my_bits = (1u << nv) - 1u;
-          }
-        }
-      }
-    }
-  }
-  const unsigned valid =
-      __reduce_or_sync(0xffffffffu, lane < DC_BPW ? my_bits << (4 * lane) : 0u);
-  // DC_TOK rows x 16 chunks for K and for V; lane owns chunk (lane & 15) of
-  // rows (lane >> 4) + 2i.
-  const int chunk = lane & 15;
+// One 16-token tile of one head: K rows at kbase, V rows at vbase (swizzled), token
+// i valid iff bit i of `valid`.
+__device__ __forceinline__ void attend_tile(Acc &s_, uint32_t kbase, uint32_t vbase, unsigned valid,
+                                            const uint32_t (&qf)[8][2], float scale_log2,
+                                            int lane) {
+  const int gq = lane >> 2;
+  const int arow = (lane & 7) + ((lane >> 3) & 1) * 8;  // K: non-transposed x4
+  const int akc = lane >> 4;
+  const int vrow = (lane & 7) + ((lane >> 4) & 1) * 8;  // V: transposed x4
+  const int vkc = (lane >> 3) & 1;
+  // S^T[16 tokens x 8 heads] in two independent accumulation chains
+  float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-  for (int i = 0; i < DC_TOK / 2; ++i) {
-    const int row = (lane >> 4) + 2 * i;
-    const int row0 = __shfl_sync(0xffffffffu, my_row0, row >> 2);
-    const bool ok = (valid >> row) & 1u;
-    const size_t off = ((size_t)(row0 + (row & 3)) * a.Hkv + g) * DC_D + chunk * 8;
-    const uint32_t so = swz(row, chunk, DC_ROWB);
-    cp_async16(ks_base + so, ok ? (const void *)(a.k_pool + off) : (const void *)a.k_pool,
-               ok ? 16 : 0);
-    cp_async16(vs_base + so, ok ? (const void *)(a.v_pool + off) : (const void *)a.v_pool,
-               ok ? 16 : 0);
+  for (int ks = 0; ks < 4; ++ks) {
+    uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
+    ldsm_x4(kbase + swz(arow, 2 * ks + akc, DV_ROWB), a0, a1, a2, a3);
+    ldsm_x4(kbase + swz(arow, 2 * (ks + 4) + akc, DV_ROWB), b0, b1, b2, b3);
+    mma_bf16_16816(sa, a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
+    mma_bf16_16816(sb, b0, b1, b2, b3, qf[ks + 4][0], qf[ks + 4][1]);
   }
-  cp_async_commit();
+  // s[0], s[1]: token gq, heads 2tq, 2tq+1; s[2], s[3]: token gq + 8
+  const bool v0 = (valid >> gq) & 1u, v1 = (valid >> (gq + 8)) & 1u;
+  const float x0 = v0 ? (sa[0] + sb[0]) * scale_log2 : -INFINITY;
+  const float x1 = v0 ? (sa[1] + sb[1]) * scale_log2 : -INFINITY;
+  const float x2 = v1 ? (sa[2] + sb[2]) * scale_log2 : -INFINITY;
+  const float x3 = v1 ? (sa[3] + sb[3]) * scale_log2 : -INFINITY;
+  float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+  for (int o_ = 4; o_ < 32; o_ <<= 1) {
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o_));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o_));
+  }
+  const float mn0 = fmaxf(s_.m0, mx0), mn1 = fmaxf(s_.m1, mx1);
+  const float base0 = mn0 == -INFINITY ? 0.f : mn0, base1 = mn1 == -INFINITY ? 0.f : mn1;
+  const float c0 = exp2f(s_.m0 - base0), c1 = exp2f(s_.m1 - base1);
+  const float p0 = exp2f(x0 - base0), p1 = exp2f(x1 - base1);
+  const float p2 = exp2f(x2 - base0), p3 = exp2f(x3 - base1);
+  float r0 = p0 + p2, r1 = p1 + p3;
+#pragma unroll
+  for (int o_ = 4; o_ < 32; o_ <<= 1) {
+    r0 += __shfl_xor_sync(0xffffffffu, r0, o_);
+    r1 += __shfl_xor_sync(0xffffffffu, r1, o_);
+  }
+  s_.l0 = s_.l0 * c0 + r0;
+  s_.l1 = s_.l1 * c1 + r1;
+  s_.m0 = mn0;
+  s_.m1 = mn1;
+  // P^T (tokens x heads) in accumulator layout -> B operand (k = tokens, n = heads)
+  const uint32_t pb0 = movmatrix_t(pack_bf16x2(p0, p1));
+  const uint32_t pb1 = movmatrix_t(pack_bf16x2(p2, p3));
+#pragma unroll
+  for (int mt = 0; mt < 8; ++mt) {
+    s_.o[mt][0] *= c0;
+    s_.o[mt][1] *= c1;
+    s_.o[mt][2] *= c0;
+    s_.o[mt][3] *= c1;
+    uint32_t a0, a1, a2, a3;
+    ldsm_x4_t(vbase + swz(vrow, 2 * mt + vkc, DV_ROWB), a0, a1, a2, a3);
+    mma_bf16_16816(s_.o[mt], a0, a1, a2, a3, pb0, pb1);
+  }
+}
 
-  // ---- query fragments (B operand of S^T = K Q^T): head g*G + lane/4
+// Write the normalised partial of heads (2tq, 2tq+1) < G: o [.., D] rows at
+// o_rows (row stride D, head h at o_rows + h*D), LSE (natural log) at lse_rows.
+__device__ __forceinline__ void store_partial(const Acc &s_, float *o_rows, float *lse_rows, int G,
+                                              int lane) {
+  const int gq = lane >> 2, tq = lane & 3;
+  const int h0 = 2 * tq, h1 = 2 * tq + 1;
+  const float inv0 = s_.l0 > 0.f ? 1.f / s_.l0 : 0.f;
+  const float inv1 = s_.l1 > 0.f ? 1.f / s_.l1 : 0.f;
+#pragma unroll
+  for (int mt = 0; mt < 8; ++mt) {
+    const int d = mt * 16 + gq;
+    if (h0 < G) {
+      o_rows[h0 * DV_D + d] = s_.o[mt][0] * inv0;
+      o_rows[h0 * DV_D + d + 8] = s_.o[mt][2] * inv0;
+    }
+    if (h1 < G) {
+      o_rows[h1 * DV_D + d] = s_.o[mt][1] * inv1;
+      o_rows[h1 * DV_D + d + 8] = s_.o[mt][3] * inv1;
+    }
+  }
+  if (gq == 0) {
+    if (h0 < G) lse_rows[h0] = s_.l0 > 0.f ? (s_.m0 + log2f(s_.l0)) * LN2 : -INFINITY;
+    if (h1 < G) lse_rows[h1] = s_.l1 > 0.f ? (s_.m1 + log2f(s_.l1)) * LN2 : -INFINITY;
+  }
+}
+
+// Tile range [v0, v0 + n) of rank c when NT tiles are split over ncb CTAs.
+__device__ __forceinline__ void tile_range(int c, int NT, int ncb, int &v0, int &n) {
+  if (c >= ncb) {
+    v0 = n = 0;
+    return;
+  }
+  v0 = (int)(((long long)c * NT) / ncb);
+  n = (int)(((long long)(c + 1) * NT) / ncb) - v0;
+}
+
+template <int ST>
+__global__ void __launch_bounds__(DV_WARPS * 32, DV_CTAS_PER_SM) sparse_decode_kernel(DecodeArgs a) {
+  extern __shared__ __align__(1024) unsigned char smem[];
+  __shared__ int s_st[DV_RMAX], s_ct[DV_RMAX], s_pre[DV_RMAX + 1];
+  __shared__ int s_L;
+  const int c = blockIdx.x, CL = a.ncb;
+  const int hg = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
+  const int g = hg * DV_WARPS + warp;  // KV head of this warp
+  const bool has_head = g < a.Hkv;
+  // shared memory: ring | selection row | page table
+  int32_t *s_sel = reinterpret_cast<int32_t *>(smem + a.ring_bytes);
+  int32_t *s_row = s_sel + a.k_pad;                                    // first pool row of a block
+  uint8_t *s_nv = reinterpret_cast<uint8_t *>(s_row + DV_TBL_BLOCKS);  // its valid tokens
+
+  // (1) L_b, the block-table row into L2, the query; then, once the top-k
+  // kernel before this one has finished, the selection row
+  {
+    if (tid == 0) s_L = a.seq_lens[b];
+    // the CTAs of a sequence pull its block-table row into L2 together, so
+    // the page lookups after the slice search hit L2
+    const char *bt_row = reinterpret_cast<const char *>(a.block_table + (size_t)b * a.max_pages);
+    const int lines = (a.max_pages * 4 + 127) >> 7;
+    for (int i = c + CL * tid; i < lines; i += CL * (int)blockDim.x)
+      asm volatile("prefetch.global.L2 [%0];\n" ::"l"(bt_row + ((size_t)i << 7)));
+  }
+  // query fragments (B operand of S^T = K Q^T): head g*G + lane/4
   const int gq = lane >> 2, tq = lane & 3;
   uint32_t qf[8][2];
   {
-    const bool hv = gq < a.G;
+    const bool hv = has_head && gq < a.G;
     const uint32_t *qrow = reinterpret_cast<const uint32_t *>(
-        a.q + ((size_t)b * a.Hq + g * a.G + (hv ? gq : 0)) * DC_D);
+        a.q + ((size_t)b * a.Hq + (hv ? g * a.G + gq : 0)) * DV_D);
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
       qf[ks][0] = hv ? qrow[ks * 8 + tq] : 0u;
       qf[ks][1] = hv ? qrow[ks * 8 + 4 + tq] : 0u;
     }
   }
-  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // heads 2tq, 2tq+1
-  float o[8][4];
-#pragma unroll
-  for (int mt = 0; mt < 8; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
-
+  pdl_wait();
+  {
+    const int32_t *srow = a.sel + (size_t)b * a.k;
+    for (int i = tid; i < a.k; i += blockDim.x) cp_async4(smem_u32(s_sel + i), srow + i);
+    cp_async_commit();
+  }
   cp_async_wait<0>();
-  __syncwarp();
-
-  const int arow = (lane & 7) + ((lane >> 3) & 1) * 8;   // K: non-transposed x4
-  const int akc = lane >> 4;
-  const int vrow = (lane & 7) + ((lane >> 4) & 1) * 8;   // V: transposed x4
-  const int vkc = (lane >> 3) & 1;
-#pragma unroll
-  for (int tt = 0; tt < DC_TOK / 16; ++tt) {
-    if (((valid >> (16 * tt)) & 0xffffu) == 0u) continue;  // warp-uniform
-    float s[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      uint32_t a0, a1, a2, a3;
-      ldsm_x4(ks_base + swz(tt * 16 + arow, 2 * ks + akc, DC_ROWB), a0, a1, a2, a3);
-      mma_bf16_16816(s, a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
-    }
-    // s[0], s[1]: token gq, heads 2tq, 2tq+1; s[2], s[3]: token gq + 8
-    const bool v0 = (valid >> (16 * tt + gq)) & 1u, v1 = (valid >> (16 * tt + gq + 8)) & 1u;
-    float x0 = v0 ? s[0] * a.scale_log2 : -INFINITY;
-    float x1 = v0 ? s[1] * a.scale_log2 : -INFINITY;
-    float x2 = v1 ? s[2] * a.scale_log2 : -INFINITY;
-    float x3 = v1 ? s[3] * a.scale_log2 : -INFINITY;
-    float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
-#pragma unroll
-    for (int o_ = 4; o_ < 32; o_ <<= 1) {
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o_));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o_));
-    }
-    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-    const float base0 = mn0 == -INFINITY ? 0.f : mn0, base1 = mn1 == -INFINITY ? 0.f : mn1;
-    const float c0 = exp2f(m0 - base0), c1 = exp2f(m1 - base1);
-    const float p0 = exp2f(x0 - base0), p1 = exp2f(x1 - base1);
-    const float p2 = exp2f(x2 - base0), p3 = exp2f(x3 - base1);
-    float r0 = p0 + p2, r1 = p1 + p3;
-#pragma unroll
-    for (int o_ = 4; o_ < 32; o_ <<= 1) {
-      r0 += __shfl_xor_sync(0xffffffffu, r0, o_);
-      r1 += __shfl_xor_sync(0xffffffffu, r1, o_);
-    }
-    l0 = l0 * c0 + r0;
-    l1 = l1 * c1 + r1;
-    m0 = mn0;
-    m1 = mn1;
-#pragma unroll
-    for (int mt = 0; mt < 8; ++mt) {
-      o[mt][0] *= c0;
-      o[mt][1] *= c1;
-      o[mt][2] *= c0;
-      o[mt][3] *= c1;
-    }
-    // P^T (tokens x heads) in accumulator layout -> B operand (k = tokens, n = heads)
-    const uint32_t pb0 = movmatrix_t(pack_bf16x2(p0, p1));
-    const uint32_t pb1 = movmatrix_t(pack_bf16x2(p2, p3));
-#pragma unroll
-    for (int mt = 0; mt < 8; ++mt) {
-      uint32_t a0, a1, a2, a3;
-      ldsm_x4_t(vs_base + swz(tt * 16 + vrow, 2 * mt + vkc, DC_ROWB), a0, a1, a2, a3);
-      mma_bf16_16816(o[mt], a0, a1, a2, a3, pb0, pb1);
-    }
-  }
-
-  // ---- merge the warps of the CTA through shared memory
-  __syncthreads();  // every warp is done with its K/V tiles
-  float *s_o = reinterpret_cast<float *>(smem);  // [DC_WARPS][8 heads][D]
-  if (gq == 0) {
-    s_m[warp][2 * tq] = m0;
-    s_m[warp][2 * tq + 1] = m1;
-    s_l[warp][2 * tq] = l0;
-    s_l[warp][2 * tq + 1] = l1;
-  }
-#pragma unroll
-  for (int mt = 0; mt < 8; ++mt) {
-    float *w0 = s_o + (warp * 8 + 2 * tq) * DC_D + mt * 16 + gq;
-    float *w1 = w0 + DC_D;
-    w0[0] = o[mt][0];
-    w1[0] = o[mt][1];
-    w0[8] = o[mt][2];
-    w1[8] = o[mt][3];
-  }
   __syncthreads();
-  // thread -> (head h, 8 consecutive dims)
-  const int h = threadIdx.x >> 4, d0 = (threadIdx.x & 15) * 8;
-  if (h < a.G) {
-    float M = -INFINITY;
+
+  // (2) slice table: slice r's run starts at st[r] and holds ct[r] blocks;
+  // its tiles are [pre[r], pre[r+1]) of the sequence's NT = pre[R] tiles
+  const int L = s_L;
+  const int nb = L <= 0 ? 0 : (L + 3) >> 2;
+  const int kb = min(a.k, nb);
+  if (warp == 0) {
+    int st[2], ct[2], nt[2];
 #pragma unroll
-    for (int w = 0; w < DC_WARPS; ++w) M = fmaxf(M, s_m[w][h]);
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, lsum = 0.f;
-    if (M != -INFINITY) {
-#pragma unroll
-      for (int w = 0; w < DC_WARPS; ++w) {
-        const float f = exp2f(s_m[w][h] - M);
-        lsum += f * s_l[w][h];
-        const float *src = s_o + (w * 8 + h) * DC_D + d0;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] += f * src[e];
+    for (int h = 0; h < 2; ++h) {
+      const int r = lane + 32 * h;
+      st[h] = ct[h] = nt[h] = 0;
+      if (r < a.R) {
+        const int lo = (int)(((long long)r * nb) / a.R);
+        const int hi = (int)(((long long)(r + 1) * nb) / a.R);
+        st[h] = lower_bound(s_sel, kb, lo);
+        ct[h] = lower_bound(s_sel, kb, hi) - st[h];
+        nt[h] = (ct[h] + 3) >> 2;
       }
     }
-    const size_t row = (((size_t)b * a.Hkv + g) * a.nslots + slot) * a.G + h;
-    float *dst = a.ws_o + row * DC_D + d0;
-    const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
-    *reinterpret_cast<float4 *>(dst) =
-        make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
-    *reinterpret_cast<float4 *>(dst + 4) =
-        make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
-    if (d0 == 0) a.ws_lse[row] = lsum > 0.f ? (M + log2f(lsum)) * LN2 : -INFINITY;
-  }
-
-  // ---- the CTA that finishes slice r last merges its chunks into o_part[r]
-  // (barrier, then one gpu-scope fence and the arrival by thread 0: the fence
-  // is cumulative over the CTA's partial writes the barrier ordered before it)
-  const int r = s_info[0], slot0 = s_info[3], nchunks = s_info[4];
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    const unsigned done = atomicAdd(a.ws_cnt + ((size_t)b * a.Hkv + g) * a.R + r, 1u);
-    __threadfence();
-    s_last = (done + 1u == (unsigned)nchunks);
-  }
-  __syncthreads();
-  if (!s_last) return;
-  if (h < a.G) {
-    const size_t row0 = (((size_t)b * a.Hkv + g) * a.nslots + slot0) * a.G + h;
-    float M = -INFINITY;
-    for (int c = 0; c < nchunks; ++c) M = fmaxf(M, __ldcg(a.ws_lse + row0 + (size_t)c * a.G));
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, wsum = 0.f;
-    if (M != -INFINITY) {
-      for (int c = 0; c < nchunks; ++c) {
-        const size_t rc = row0 + (size_t)c * a.G;
-        const float f = __expf(__ldcg(a.ws_lse + rc) - M);
-        const float4 v0 = __ldcg(reinterpret_cast<const float4 *>(a.ws_o + rc * DC_D + d0));
-        const float4 v1 = __ldcg(reinterpret_cast<const float4 *>(a.ws_o + rc * DC_D + d0 + 4));
-        acc[0] += f * v0.x; acc[1] += f * v0.y; acc[2] += f * v0.z; acc[3] += f * v0.w;
-        acc[4] += f * v1.x; acc[5] += f * v1.y; acc[6] += f * v1.z; acc[7] += f * v1.w;
-        wsum += f;
+    int inc0 = nt[0], inc1 = nt[1];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y0 = __shfl_up_sync(0xffffffffu, inc0, o), y1 = __shfl_up_sync(0xffffffffu, inc1, o);
+      if (lane >= o) {
+        inc0 += y0;
+        inc1 += y1;
       }
     }
-    const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-    const size_t orow = ((size_t)r * a.B + b) * a.Hq + g * a.G + h;
-    float *o = a.o_part + orow * DC_D + d0;
-    *reinterpret_cast<float4 *>(o) =
-        make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
-    *reinterpret_cast<float4 *>(o + 4) =
-        make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
-    if (d0 == 0) a.lse_part[orow] = wsum > 0.f ? M + logf(wsum) : -INFINITY;
+    inc1 += __shfl_sync(0xffffffffu, inc0, 31);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int r = lane + 32 * h;
+      if (r < a.R) {
+        s_st[r] = st[h];
+        s_ct[r] = ct[h];
+        s_pre[r] = (h ? inc1 : inc0) - nt[h];
+      }
+    }
+    const int total = __shfl_sync(0xffffffffu, inc1, 31);
+    if (lane == 0) {
+      s_pre[a.R] = total;
+      if (L < 0 && c == 0 && hg == 0) raise_err(a.err, ERR_LEN);
+    }
   }
+  __syncthreads();
+
+  // (3) this CTA's tiles [v0, v0 + ntile) and the pool row of each of their
+  // blocks; at most NT CTAs share the sequence, so every range is non-empty
+  const int NT = s_pre[a.R];
+  const int ncb = min(CL, NT);
+  int v0, ntile;
+  tile_range(c, NT, ncb, v0, ntile);
+  if (ntile > DV_TBL_TILES) {  // excluded by the host's choice of ncb
+    if (tid == 0) raise_err(a.err, ERR_SEL);
+    ntile = DV_TBL_TILES;
+  }
+  const int nslot = 4 * ntile;
+  for (int q0 = 0; q0 < nslot; q0 += 4 * (int)blockDim.x) {
+    long long idx[4];
+    int jj[4], pg[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int q = q0 + tid + u * (int)blockDim.x;
+      idx[u] = -1;
+      jj[u] = 0;
+      if (q < nslot) {
+        const int v = v0 + (q >> 2);
+        const int r = slice_of_tile(s_pre, a.R, v);
+        const int off = 4 * (v - s_pre[r]) + (q & 3);
+        if (off < s_ct[r]) {
+          const int j = s_sel[s_st[r] + off];
+          if (j < 0 || j >= nb) {
+            raise_err(a.err, ERR_SEL);
+          } else {
+            const int col = (4 * j) / a.P;
+            if (col >= a.max_pages) {
+              raise_err(a.err, ERR_BT);
+            } else {
+              idx[u] = (long long)b * a.max_pages + col;
+              jj[u] = j;
+            }
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) pg[u] = idx[u] >= 0 ? __ldg(a.block_table + idx[u]) : -1;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int q = q0 + tid + u * (int)blockDim.x;
+      if (q < nslot) {
+        int row = -1, nv = 0;
+        if (idx[u] >= 0) {
+          if (pg[u] < 0 || pg[u] >= a.num_pages) {
+            raise_err(a.err, ERR_PAGE);
+          } else {
+            row = pg[u] * a.P + (4 * jj[u]) % a.P;
+            nv = min(4, L - 4 * jj[u]);
+          }
+        }
+        s_row[q] = row;
+        s_nv[q] = (uint8_t)nv;
+      }
+    }
+  }
+  __syncthreads();
+
+  // contributors [c_lo, c_hi] of slice r (non-empty), from the tile split
+  auto contributors = [&](int r, int &c_lo, int &c_hi) {
+    const int pre = s_pre[r], nt = s_pre[r + 1] - pre;
+    c_lo = cta_of_tile(pre, NT, ncb);
+    c_hi = cta_of_tile(pre + nt - 1, NT, ncb);
+  };
+  // which slices the combine kernel must merge, and from which CTAs
+  if (c == 0 && hg == 0) {
+    for (int r = tid; r < a.R; r += blockDim.x) {
+      int2 sp = make_int2(0, -1);
+      if (s_ct[r] != 0) contributors(r, sp.x, sp.y);
+      a.span[(size_t)b * a.R + r] = sp;
+    }
+  }
+  // slices that own no selected block: O_r = 0, LSE_r = -inf (CTA 0 writes them)
+  if (has_head && c == 0) {
+    for (int r = 0; r < a.R; ++r) {
+      if (s_ct[r] != 0) continue;
+      for (int h = 0; h < a.G; ++h) {
+        const size_t row = ((size_t)r * a.B + b) * a.Hq + g * a.G + h;
+        reinterpret_cast<float4 *>(a.o_part + row * DV_D)[lane] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (lane == 0) a.lse_part[row] = -INFINITY;
+      }
+    }
+  }
+
+  const uint32_t ring = smem_u32(smem) + warp * ST * DV_STAGE;
+
+  // (4) stream this head's tiles through the ring
+  if (has_head && ntile > 0) {
+    const int chunk = lane & 15;
+    auto issue = [&](int t) {
+      if (t < ntile) {
+        const uint32_t kbuf = ring + (t % ST) * DV_STAGE, vbuf = kbuf + DV_TOK * DV_ROWB;
+#pragma unroll
+        for (int i = 0; i < DV_TOK / 2; ++i) {
+          const int row = (lane >> 4) + 2 * i;
+          const int slot = 4 * t + (row >> 2);
+          const int row0 = s_row[slot];
+          const bool ok = (row & 3) < (int)s_nv[slot];
+          const size_t off = ((size_t)(row0 + (row & 3)) * a.Hkv + g) * DV_D + chunk * 8;
+          const uint32_t so = swz(row, chunk, DV_ROWB);
+          cp_async16(kbuf + so, ok ? (const void *)(a.k_pool + off) : (const void *)a.k_pool,
+                     ok ? 16 : 0);
+          cp_async16(vbuf + so, ok ? (const void *)(a.v_pool + off) : (const void *)a.v_pool,
+                     ok ? 16 : 0);
+        }
+      }
+      cp_async_commit();
+    };
+#pragma unroll
+    for (int t = 0; t < ST - 1; ++t) issue(t);
+
+    Acc acc;
+    acc.reset();
+    int cur = -1;                            // slice of the running segment
+    int rs = slice_of_tile(s_pre, a.R, v0);  // slice of the current tile
+    // (5) partial of slice r over this CTA's tiles
+    auto flush = [&](int r) {
+      int c_lo, c_hi;
+      contributors(r, c_lo, c_hi);
+      if (c_lo == c_hi) {  // the only contributor: the partial is slice r's result
+        const size_t row = ((size_t)r * a.B + b) * a.Hq + g * a.G;
+        store_partial(acc, a.o_part + row * DV_D, a.lse_part + row, a.G, lane);
+      } else {  // shared with neighbouring CTAs: a record for the combine kernel
+        const size_t row = ((size_t)b * a.rb + c + r) * a.Hq + g * a.G;
+        store_partial(acc, a.rec_o + row * DV_D, a.rec_lse + row, a.G, lane);
+      }
+    };
+    for (int t = 0; t < ntile; ++t) {
+      const int v = v0 + t;
+      while (s_pre[rs + 1] <= v) ++rs;
+      if (rs != cur) {
+        if (cur >= 0) {
+          flush(cur);
+          acc.reset();
+        }
+        cur = rs;
+      }
+      __syncwarp();  // every lane is done with the stage the next issue overwrites
+      issue(t + ST - 1);
+      cp_async_wait<ST - 1>();
+      __syncwarp();
+      unsigned valid = 0;
+#pragma unroll
+      for (int blk = 0; blk < 4; ++blk) valid |= ((1u << s_nv[4 * t + blk]) - 1u) << (4 * blk);
+      const uint32_t kbuf = ring + (t % ST) * DV_STAGE;
+      if (valid) attend_tile(acc, kbuf, kbuf + DV_TOK * DV_ROWB, valid, qf, a.scale_log2, lane);
+    }
+    cp_async_wait<0>();
+    pdl_trigger();
+    flush(cur);
+  }
+}
+
+// (6) One CTA per (group of DV_CB_ROWS query heads, slice, sequence); thread
+// (row, d4) combines dims 4*d4..4*d4+3 of one query head over the records of
+// the slice's contributors: first the max of their LSEs, then the weighted
+// sum, DV_CB_BATCH records' loads in flight at a time.
+__global__ void __launch_bounds__(DV_CB_ROWS * 32) decode_combine_kernel(DecodeArgs a) {
+  pdl_wait();  // the records come from the decode kernel before this one
+  const int b = blockIdx.z, r = blockIdx.y;
+  const int q = blockIdx.x * DV_CB_ROWS + (threadIdx.x >> 5), d4 = threadIdx.x & 31;
+  const int2 sp = a.span[(size_t)b * a.R + r];
+  if (sp.y <= sp.x || q >= a.Hq) return;  // written by the decode kernel itself
+  const int n = sp.y - sp.x + 1;
+  const size_t row0 = ((size_t)b * a.rb + sp.x + r) * a.Hq + q;  // record i at row0 + i*Hq
+  float M = -INFINITY;
+  for (int i0 = 0; i0 < n; i0 += DV_CB_BATCH) {
+    float l[DV_CB_BATCH];
+#pragma unroll
+    for (int u = 0; u < DV_CB_BATCH; ++u)
+      l[u] = __ldcg(a.rec_lse + row0 + (size_t)min(i0 + u, n - 1) * a.Hq);
+#pragma unroll
+    for (int u = 0; u < DV_CB_BATCH; ++u) M = fmaxf(M, l[u]);
+  }
+  float acc[4] = {0.f, 0.f, 0.f, 0.f}, wsum = 0.f;
+  if (M != -INFINITY) {
+    for (int i0 = 0; i0 < n; i0 += DV_CB_BATCH) {
+      float l[DV_CB_BATCH];
+      float4 v[DV_CB_BATCH];
+#pragma unroll
+      for (int u = 0; u < DV_CB_BATCH; ++u) {
+        const size_t rr = row0 + (size_t)min(i0 + u, n - 1) * a.Hq;
+        l[u] = __ldcg(a.rec_lse + rr);
+        v[u] = __ldcg(reinterpret_cast<const float4 *>(a.rec_o + rr * DV_D) + d4);
+      }
+#pragma unroll
+      for (int u = 0; u < DV_CB_BATCH; ++u) {
+        const float w = i0 + u < n ? __expf(l[u] - M) : 0.f;
+        wsum += w;
+        acc[0] += w * v[u].x;
+        acc[1] += w * v[u].y;
+        acc[2] += w * v[u].z;
+        acc[3] += w * v[u].w;
+      }
+    }
+  }
+  const size_t orow = ((size_t)r * a.B + b) * a.Hq + q;
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+  reinterpret_cast<float4 *>(a.o_part + orow * DV_D)[d4] =
+      make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+  if (d4 == 0) a.lse_part[orow] = wsum > 0.f ? M + logf(wsum) : -INFINITY;
+}
+
+struct DecodePlan {
+  int nhg, ncb, rb, stages, k_pad;
+  size_t smem;
+};
+
+DecodePlan plan_decode(const qsa_dims &d, int B, int k, int R) {
+  DecodePlan p;
+  p.nhg = (d.Hkv + DV_WARPS - 1) / DV_WARPS;
+  p.k_pad = (k + 3) & ~3;
+  const size_t extra = (size_t)p.k_pad * 4 + (size_t)DV_TBL_BLOCKS * 5;
+  const size_t static_smem = 1024;
+  const size_t fit = (DV_SMEM_LIMIT - static_smem - extra) / ((size_t)DV_WARPS * DV_STAGE);
+  p.stages = fit >= 4 ? 4 : (fit >= 3 ? 3 : 2);
+  p.smem = (size_t)DV_WARPS * p.stages * DV_STAGE + extra;
+  // CTAs per sequence: enough to keep DV_SLOTS CTAs busy, at most one per
+  // tile, and enough that a CTA's tile range fits its page table
+  const long long ntmax = (k + 3) / 4 + R - 1;
+  long long ncb = DV_SLOTS / ((long long)B * p.nhg);
+  if (ncb > ntmax) ncb = ntmax;
+  if (ncb < 1) ncb = 1;
+  const long long need = (ntmax + DV_TBL_TILES - 1) / DV_TBL_TILES;
+  if (ncb < need) ncb = need;
+  p.ncb = (int)ncb;
+  p.rb = p.ncb + R - 1;
+  return p;
+}
+
+template <int ST>
+cudaError_t launch_st(const DecodeArgs &a, const DecodePlan &p, int B, cudaStream_t st) {
+  cudaError_t e = cudaFuncSetAttribute(sparse_decode_kernel<ST>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
+  if (e != cudaSuccess) return e;
+  e = launch_pdl(sparse_decode_kernel<ST>, dim3(p.ncb, p.nhg, B), DV_WARPS * 32, p.smem, st, a);
+  if (e != cudaSuccess || p.ncb == 1) return e;  // one CTA per sequence: nothing to combine
+  return launch_pdl(decode_combine_kernel, dim3((a.Hq + DV_CB_ROWS - 1) / DV_CB_ROWS, a.R, B),
+                    DV_CB_ROWS * 32, 0, st, a);
 }
 
 }  // namespace
 
-int decode_num_slots(int k, int R) { return (k + DC_BLOCKS - 1) / DC_BLOCKS + R; }
-
 size_t decode_ws_bytes(const qsa_dims &d, int B, int k, int R) {
-  const size_t rows = (size_t)B * d.Hkv * decode_num_slots(k, R) * (d.Hq / d.Hkv);
-  return rows * (DC_D + 1) * sizeof(float) + (size_t)B * d.Hkv * R * sizeof(unsigned);
+  const DecodePlan p = plan_decode(d, B, k, R);
+  const size_t rows = (size_t)B * p.rb * d.Hq;
+  return rows * (DV_D + 1) * sizeof(float) + (size_t)B * R * sizeof(int2);
 }
 
 cudaError_t launch_sparse_decode(const qsa_dims &d, const qsa_cache &c, int B,
@@ -414,6 +565,7 @@ cudaError_t launch_sparse_decode(const qsa_dims &d, const qsa_cache &c, int B,
                                  int k, int R, float *o_part, float *lse_part, void *ws,
                                  unsigned *err, cudaStream_t st) {
   if (B == 0) return cudaSuccess;
+  const DecodePlan p = plan_decode(d, B, k, R);
   DecodeArgs a;
   a.k_pool = static_cast<const __nv_bfloat16 *>(c.k_pool);
   a.v_pool = static_cast<const __nv_bfloat16 *>(c.v_pool);
@@ -421,32 +573,32 @@ cudaError_t launch_sparse_decode(const qsa_dims &d, const qsa_cache &c, int B,
   a.block_table = c.block_table;
   a.seq_lens = seq_lens;
   a.sel = sel;
-  a.nslots = decode_num_slots(k, R);
-  a.G = d.Hq / d.Hkv;
-  const size_t rows = (size_t)B * d.Hkv * a.nslots * a.G;
-  a.ws_o = static_cast<float *>(ws);
-  a.ws_lse = a.ws_o + rows * DC_D;
-  a.ws_cnt = reinterpret_cast<unsigned *>(a.ws_lse + rows);
   a.o_part = o_part;
   a.lse_part = lse_part;
+  const size_t rows = (size_t)B * p.rb * d.Hq;
+  a.rec_o = static_cast<float *>(ws);
+  a.rec_lse = a.rec_o + rows * DV_D;
+  a.span = reinterpret_cast<int2 *>(a.rec_lse + rows);
   a.B = B;
   a.Hq = d.Hq;
   a.Hkv = d.Hkv;
+  a.G = d.Hq / d.Hkv;
   a.P = d.P;
   a.max_pages = c.max_pages_per_seq;
   a.num_pages = c.num_pages;
   a.k = k;
+  a.k_pad = p.k_pad;
   a.R = R;
+  a.ncb = p.ncb;
+  a.rb = p.rb;
+  a.ring_bytes = DV_WARPS * p.stages * DV_STAGE;
   a.scale_log2 = d.scale * LOG2E;
   a.err = err;
-  const size_t smem = (size_t)DC_WARPS * DC_WARP_SMEM;
-  cudaError_t e = cudaFuncSetAttribute(sparse_decode_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  e = cudaMemsetAsync(a.ws_cnt, 0, (size_t)B * d.Hkv * R * sizeof(unsigned), st);
-  if (e != cudaSuccess) return e;
-  sparse_decode_kernel<<<dim3(a.nslots, d.Hkv, B), DC_WARPS * 32, smem, st>>>(a);
-  return cudaGetLastError();
+  switch (p.stages) {
+    case 4: return launch_st<4>(a, p, B, st);
+    case 3: return launch_st<3>(a, p, B, st);
+    default: return launch_st<2>(a, p, B, st);
+  }
 }
 
 }  // namespace qsa

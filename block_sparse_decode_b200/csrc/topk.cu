@@ -12,8 +12,9 @@
 // over the key bits (4 passes of 8 bits, most significant first) finds the
 // k-th largest key T and how many keys equal to T are taken: every pass
 // counts the digits of the keys still matching the prefix into a per-CTA
-// histogram (warp-aggregated shared atomics), the 8 histograms are summed
-// through distributed shared memory, and every CTA picks the same digit. The
+// histogram (per-warp shared histograms, lanes with equal digits adding
+// once), the 8 histograms are summed through distributed shared memory, and
+// every CTA picks the same digit. The
 // compaction then writes each selected block at position
 //   (#keys > T before it) + min(#keys == T before it, ties taken),
 // which is ascending index order; the per-CTA counts are exchanged through
@@ -31,6 +32,7 @@ namespace {
 
 constexpr int TK_THREADS = 512;
 constexpr int TK_WARPS = TK_THREADS / 32;
+constexpr int TK_LOADS = 16;  // score loads per thread issued together
 
 struct TopkArgs {
   const float *scores;
@@ -64,6 +66,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a) {
   const int L = a.seq_lens[b];
   const int nb = L < 0 ? 0 : (L + 3) >> 2;
   int32_t *out = a.sel + (size_t)b * a.k;
+  pdl_wait();  // the scores come from the kernel before this one
   if (L < 0 || nb > a.ld) {  // uniform over the cluster
     if (crank == 0 && tid == 0) raise_err(a.err, ERR_LEN);
     for (int i = crank * TK_THREADS + tid; i < a.k; i += TOPK_CLUSTER * TK_THREADS) out[i] = -1;
@@ -79,7 +82,20 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a) {
   const int lo = min(nb, crank * chunk);
   const int n = min(nb, lo + chunk) - lo;
   const float *src = a.scores + (size_t)b * a.ld + lo;
-  for (int i = tid; i < n; i += TK_THREADS) keys[i] = score_key(src[i]);
+  // TK_LOADS loads per thread in flight before any is used
+  for (int i0 = 0; i0 < n; i0 += TK_THREADS * TK_LOADS) {
+    float v[TK_LOADS];
+#pragma unroll
+    for (int u = 0; u < TK_LOADS; ++u) {
+      const int i = i0 + u * TK_THREADS + tid;
+      v[u] = i < n ? src[i] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < TK_LOADS; ++u) {
+      const int i = i0 + u * TK_THREADS + tid;
+      if (i < n) keys[i] = score_key(v[u]);
+    }
+  }
   if (tid == 0) { pick[0] = 0; pick[1] = 0; pick[2] = 0; }
 
   // contiguous per-warp segments of the CTA's range
@@ -94,9 +110,15 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a) {
     // barrier, so it can be rewritten now)
     for (int i = lane; i < 256; i += 32) whist[warp][i] = 0u;
     __syncthreads();  // keys loaded (first pass), pick[] of the last pass read
-    for (int i = s0 + lane; i < s1; i += 32) {
-      const uint32_t key = keys[i];
-      if ((key & mask) == prefix) atomicAdd(&whist[warp][(key >> shift) & 255u], 1u);
+    // lanes with the same digit add once (their count): heavy-tailed scores
+    // put most keys of the leading passes into a few bins
+    for (int base = s0; base < s1; base += 32) {
+      const int i = base + lane;
+      const uint32_t key = i < s1 ? keys[i] : 0u;
+      const bool hit = i < s1 && (key & mask) == prefix;
+      const unsigned bin = hit ? (key >> shift) & 255u : 256u + lane;
+      const unsigned peers = __match_any_sync(0xffffffffu, bin);
+      if (hit && lane == __ffs(peers) - 1) atomicAdd(&whist[warp][bin], (unsigned)__popc(peers));
     }
     __syncthreads();
     if (tid < 256) {
@@ -138,6 +160,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a) {
     need -= pick[1];
     if (pick[2] == need) break;  // every key left under the prefix is kept
   }
+  pdl_trigger();
   // Selection: keys whose masked value is above the prefix, plus the first
   // `need` (lowest index) keys equal to it under the mask.
   const int take_eq = need;
@@ -199,13 +222,15 @@ cudaError_t launch_topk(int B, const int32_t *seq_lens, const float *scores, int
   cfg.blockDim = dim3(TK_THREADS, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = TOPK_CLUSTER;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, topk_kernel, a);
 }
 

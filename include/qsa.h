@@ -164,9 +164,10 @@ qsa_status qsa_topk_select(int32_t B, const int32_t *seq_lens,
                            qsa_stream_t stream);
 
 /* Scratch bytes qsa_sparse_decode needs for B sequences, top-k k, R slices.
- * The scratch holds per-chunk partial results; it needs no initialisation
- * and is fully rewritten by every call (calls sharing one scratch buffer
- * must be ordered on the GPU). */
+ * The scratch holds the partial results of slices that several CTAs share
+ * and the list of those slices; it needs no initialisation and every call
+ * writes what it later reads (calls sharing one scratch buffer must be
+ * ordered on the GPU). */
 size_t qsa_sparse_decode_workspace_size(const qsa_dims *dims, int32_t B,
                                         int32_t k, int32_t R);
 
@@ -205,9 +206,8 @@ qsa_status qsa_sparse_decode(const qsa_dims *dims, const qsa_cache *cache,
  * QSA_ERR_UNSUPPORTED. The call allocates nothing.
  * The first call on a device looks up the array's device address (once per
  * device, with that device current); make that first call before any stream
- * capture. All calls share the one array, which keeps the last call's
- * contents (each call clears, on its stream, what must start at zero):
- * calls whose executions overlap on the GPU race and corrupt each other. */
+ * capture. All calls share the one array: calls whose executions overlap on
+ * the GPU race and corrupt each other. */
 qsa_status qsa_sparse_decode_static(const qsa_dims *dims, const qsa_cache *cache,
                                     int32_t B, const int32_t *seq_lens,
                                     const void *q, const int32_t *sel, int32_t k,

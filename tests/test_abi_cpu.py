@@ -42,10 +42,14 @@ def test_version_and_workspace_sizes(L):
     assert qsa.qsa_version() == 100
     assert qsa.qsa_topk_workspace_size(8, 65536, 512) == 0
     d = qsa.QsaDims(32, 4, 128, 16, 128, 64, 0.088)
-    # (ceil(512/16) + 4) chunk slots x 4 kv heads x 8 heads x (128 + 1) floats per
-    # sequence, plus one arrival counter per (sequence, kv head, slice)
-    assert qsa.qsa_sparse_decode_workspace_size(d, 8, 512, 4) == \
-        8 * 36 * 4 * 8 * 129 * 4 + 8 * 4 * 4 * 4
+    # records of shared slices: 296 CTA slots / B sequences CTAs per sequence
+    # (at most one per tile, at least ceil((k/4 + R - 1) / 256) for the page
+    # table), keyed by CTA + slice, each 32 heads x (128 + 1) floats; plus one
+    # (c_lo, c_hi) pair per (sequence, slice)
+    for B, k, R, ncb in ((8, 512, 4, 37), (512, 512, 4, 1), (512, 4096, 4, 5),
+                         (2, 512, 2, 129), (1, 1, 1, 1)):
+        assert qsa.qsa_sparse_decode_workspace_size(d, B, k, R) == \
+            B * (ncb + R - 1) * 32 * 129 * 4 + B * R * 8, (B, k, R)
 
 
 def _status(fn, *args):

@@ -260,11 +260,49 @@ def test_invalid_arguments_rejected_on_host():
         qsa.qsa_sparse_decode(run.dims, run.cache, run.seq_lens, wl.q, run.buf.sel, 8, 65,
                               run.buf.o_part, run.buf.lse_part, run.buf.ws)
     assert ei.value.status == qsa.QSA_ERR_UNSUPPORTED
+    o_mis = torch.empty(run.buf.o_part.numel() + 1, dtype=torch.float32, device=DEV)[1:]
+    with pytest.raises(qsa.QsaError) as ei:  # o_part not 16-byte aligned
+        qsa.qsa_sparse_decode(run.dims, run.cache, run.seq_lens, wl.q, run.buf.sel, 8, 1,
+                              o_mis.view_as(run.buf.o_part), run.buf.lse_part, run.buf.ws)
+    assert ei.value.status == qsa.QSA_ERR_INVALID_ARG
     small_ws = torch.empty(16, dtype=torch.uint8, device=DEV)
     with pytest.raises(qsa.QsaError) as ei:
         qsa.qsa_sparse_decode(run.dims, run.cache, run.seq_lens, wl.q, run.buf.sel, 8, 1,
                               run.buf.o_part, run.buf.lse_part, small_ws)
     assert ei.value.status == qsa.QSA_ERR_INVALID_ARG
+
+
+def test_decode_shapes_back_to_back():
+    # calls of different B, k and R in a row (different CTA splits and slice
+    # layouts) sharing one scratch buffer, each checked against the oracle
+    wl = make_custom(DIMS_FULL, [9000, 3001, 17, 40000], k=512, R=4, seed=109, device=DEV)
+    run = GpuRun(wl)
+    run.step()
+    sel = run.buf.sel
+    ws = torch.empty(max(qsa.qsa_sparse_decode_workspace_size(run.dims, B, k, R)
+                         for B, k, R in ((4, 512, 4), (2, 512, 7), (4, 128, 1))),
+                     dtype=torch.uint8, device=DEV)
+    for B, k, R in ((4, 512, 4), (2, 512, 7), (4, 128, 1), (4, 512, 4), (2, 512, 7)):
+        o = torch.full((R, B, run.dims.Hq, run.dims.D), float("nan"), device=DEV)
+        lse = torch.full((R, B, run.dims.Hq), float("nan"), device=DEV)
+        sl = run.seq_lens[:B]
+        if k == 512:
+            s_ = sel[:B]
+        else:  # a smaller selection: the first k of every row, still ascending
+            nb = [(L + 3) // 4 for L in wl.seq_lens[:B]]
+            s_ = torch.stack([torch.arange(k, device=DEV, dtype=torch.int32) * max(1, n // k)
+                              for n in nb]).contiguous()
+            for b, n in enumerate(nb):
+                if n < k:
+                    s_[b, n:] = -1
+                    s_[b, :n] = torch.arange(n, device=DEV, dtype=torch.int32)
+        qsa.qsa_sparse_decode(run.dims, run.cache, sl, wl.q[:B].contiguous(), s_, k, R, o, lse,
+                              ws)
+        assert qsa.qsa_check_device_errors() == 0
+        for b in range(B):
+            ref = oracle_sequence(wl, b, k=k, R=R, sel=s_[b].cpu().numpy())
+            check_attention(o[:, b].cpu().numpy(), lse[:, b].cpu().numpy(), ref["O_part"],
+                            ref["LSE_part"], what=f"B={B} k={k} R={R} b={b}")
 
 
 def test_empty_batch_is_a_no_op():

@@ -45,6 +45,30 @@ def test_static_scratch_decode_matches_workspace_decode():
                             what=f"static scratch b={b}")
 
 
+def test_static_scratch_serves_the_largest_k_and_R():
+    # k = 4096 and R = 64, the largest the call accepts, at a small batch: the
+    # scratch need fits the static array, and the result equals the regular
+    # entry point's
+    d = qsa.QsaDims.of(DIMS_FULL)
+    need = qsa.qsa_sparse_decode_workspace_size(d, 2, 4096, 64)
+    assert 0 < need <= (32 << 20)
+    wl = make_custom(DIMS_FULL, [20000, 16390], k=4096, R=64, seed=202, device="cuda",
+                     paged=True)
+    run = GpuRun(wl)
+    run.step()
+    ref_o = run.buf.o_part.clone()
+    ref_l = run.buf.lse_part.clone()
+    o = torch.full_like(ref_o, float("nan"))
+    l = torch.full_like(ref_l, float("nan"))
+    qsa.qsa_sparse_decode_static(run.dims, run.cache, run.seq_lens, wl.q, run.buf.sel, wl.k,
+                                 wl.R, o, l)
+    assert qsa.qsa_check_device_errors() == 0
+    for b in range(wl.B):
+        check_attention(o[:, b].cpu().numpy(), l[:, b].cpu().numpy(),
+                        ref_o[:, b].cpu().numpy(), ref_l[:, b].cpu().numpy(),
+                        what=f"static scratch k=4096 R=64 b={b}")
+
+
 def test_static_scratch_rejects_oversized_calls():
     # B = 4096 sequences at k = 4096, R = 64 needs far more than the static array
     need = qsa.qsa_sparse_decode_workspace_size(qsa.QsaDims.of(DIMS_FULL), 4096, 4096, 64)
