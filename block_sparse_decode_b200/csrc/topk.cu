@@ -12,9 +12,8 @@
 // over the key bits (4 passes of 8 bits, most significant first) finds the
 // k-th largest key T and how many keys equal to T are taken: every pass
 // counts the digits of the keys still matching the prefix into a per-CTA
-// histogram (per-warp shared histograms, lanes with equal digits adding
-// once), the 8 histograms are summed through distributed shared memory, and
-// every CTA picks the same digit. The
+// histogram (per-warp shared histograms), the 8 histograms are summed
+// through distributed shared memory, and every CTA picks the same digit. The
 // compaction then writes each selected block at position
 //   (#keys > T before it) + min(#keys == T before it, ties taken),
 // which is ascending index order; the per-CTA counts are exchanged through
@@ -110,15 +109,9 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a) {
     // barrier, so it can be rewritten now)
     for (int i = lane; i < 256; i += 32) whist[warp][i] = 0u;
     __syncthreads();  // keys loaded (first pass), pick[] of the last pass read
-    // lanes with the same digit add once (their count): heavy-tailed scores
-    // put most keys of the leading passes into a few bins
-    for (int base = s0; base < s1; base += 32) {
-      const int i = base + lane;
-      const uint32_t key = i < s1 ? keys[i] : 0u;
-      const bool hit = i < s1 && (key & mask) == prefix;
-      const unsigned bin = hit ? (key >> shift) & 255u : 256u + lane;
-      const unsigned peers = __match_any_sync(0xffffffffu, bin);
-      if (hit && lane == __ffs(peers) - 1) atomicAdd(&whist[warp][bin], (unsigned)__popc(peers));
+    for (int i = s0 + lane; i < s1; i += 32) {
+      const uint32_t key = keys[i];
+      if ((key & mask) == prefix) atomicAdd(&whist[warp][(key >> shift) & 255u], 1u);
     }
     __syncthreads();
     if (tid < 256) {
