@@ -8,9 +8,9 @@
 // entries here write nothing at all).
 //
 // Two phases: the first writes K, V and the per-token indexer key of every
-// token (one warp per token, 16-byte stores); the second, for every token
-// with pos % 4 == 3, reads the block's 4 indexer keys back from the pool and
-// writes their mean. Ordering the phases makes a bulk prefill (tokens of a
+// token (one warp per token, 16-byte loads and stores); the second, for every
+// token with pos % 4 == 3, reads the block's 4 indexer keys back from the pool
+// and writes their mean. Ordering the phases makes a bulk prefill (tokens of a
 // block written by the same call, in any order) give the same side cache as
 // one token per call. Up to 128 tokens (decode: one per sequence) both phases
 // run in one CTA separated by a barrier, one launch; larger calls use two
@@ -55,32 +55,52 @@ __device__ __forceinline__ int locate(const AppendArgs &a, int s, int p, int lan
 }
 
 // Phase 1 for one token (one warp): K, V and indexer key into the pools.
-__device__ __forceinline__ void write_token(const AppendArgs &a, int tok, int lane) {
+// Returns (page, position) of the token; page -1 if it writes nothing.
+// The token's input rows are loaded together with its sequence and position,
+// before the page lookup that depends on them.
+__device__ __forceinline__ int2 write_token(const AppendArgs &a, int tok, int lane) {
   const int s = a.tok_seq[tok], p = a.tok_pos[tok];
-  if (s < 0 || p < 0) return;  // padding / synthetic entry: no write anywhere
-  const int page = locate(a, s, p, lane);
-  if (page < 0) return;
-  const size_t row = (size_t)page * a.P + (p % a.P);
   const uint4 *ks = a.k_new + (size_t)tok * a.kv_vec;
   const uint4 *vs = a.v_new + (size_t)tok * a.kv_vec;
+  const uint4 *xs = a.x_new + (size_t)tok * a.x_vec;
+  constexpr int U = 2;  // 16-byte vectors of K (and of V) held per lane: Hkv*D <= 512
+  uint4 kr[U], vr[U], xr = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int i = lane + 32 * u;
+    if (i < a.kv_vec) {
+      kr[u] = ks[i];
+      vr[u] = vs[i];
+    }
+  }
+  if (lane < a.x_vec) xr = xs[lane];
+  if (s < 0 || p < 0) return make_int2(-1, p);  // padding / synthetic entry: no write
+  const int page = locate(a, s, p, lane);
+  if (page < 0) return make_int2(-1, p);
+  const size_t row = (size_t)page * a.P + (p % a.P);
   uint4 *kd = a.k_pool + row * a.kv_vec;
   uint4 *vd = a.v_pool + row * a.kv_vec;
-  for (int i = lane; i < a.kv_vec; i += 32) {
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int i = lane + 32 * u;
+    if (i < a.kv_vec) {
+      kd[i] = kr[u];
+      vd[i] = vr[u];
+    }
+  }
+  for (int i = lane + 32 * U; i < a.kv_vec; i += 32) {  // wider rows than U vectors per lane
     kd[i] = ks[i];
     vd[i] = vs[i];
   }
-  const uint4 *xs = a.x_new + (size_t)tok * a.x_vec;
-  uint4 *xd = a.x_pool + row * a.x_vec;
-  for (int i = lane; i < a.x_vec; i += 32) xd[i] = xs[i];
+  if (lane < a.x_vec) a.x_pool[row * a.x_vec + lane] = xr;
+  return make_int2(page, p);
 }
 
-// Phase 2 for one token (one warp): if it closes a micro-block, store the
-// block's compressed key in the side pool.
-__device__ __forceinline__ void compress_block(const AppendArgs &a, int tok, int lane) {
-  const int s = a.tok_seq[tok], p = a.tok_pos[tok];
-  if (s < 0 || p < 0 || (p & 3) != 3) return;
-  const int page = locate(a, s, p, 32);  // errors were flagged by the first launch
-  if (page < 0) return;
+// Phase 2 for one token (one warp) that closes a micro-block (position p, on
+// page `page`): store the block's compressed key in the side pool. The four
+// indexer keys are read through L2 (phase 1 of this launch may have written
+// them from other SMs).
+__device__ __forceinline__ void compress_at(const AppendArgs &a, int p, int page, int lane) {
   const int slot = p % a.P;
   const uint32_t *x = reinterpret_cast<const uint32_t *>(a.x_pool) +
                       ((size_t)page * a.P + slot - 3) * (a.di / 2);
@@ -88,12 +108,22 @@ __device__ __forceinline__ void compress_block(const AppendArgs &a, int tok, int
                   ((size_t)page * (a.P / 4) + slot / 4) * (a.di / 2);
   const int half = a.di / 2;  // bf16 pairs per key
   for (int e = lane; e < half; e += 32) {
-    uint32_t v0 = x[e], v1 = x[half + e], v2 = x[2 * half + e], v3 = x[3 * half + e];
+    const uint32_t v0 = __ldcg(x + e), v1 = __ldcg(x + half + e);
+    const uint32_t v2 = __ldcg(x + 2 * half + e), v3 = __ldcg(x + 3 * half + e);
     // fp32 sum in token order, then IEEE division by 4, then RNE to bf16.
     float lo = __fadd_rn(__fadd_rn(__fadd_rn(bf16lo(v0), bf16lo(v1)), bf16lo(v2)), bf16lo(v3));
     float hi = __fadd_rn(__fadd_rn(__fadd_rn(bf16hi(v0), bf16hi(v1)), bf16hi(v2)), bf16hi(v3));
     out[e] = pack_bf16x2(__fdiv_rn(lo, 4.0f), __fdiv_rn(hi, 4.0f));
   }
+}
+
+// Phase 2 when the page has to be looked up again (separate launch).
+__device__ __forceinline__ void compress_block(const AppendArgs &a, int tok, int lane) {
+  const int s = a.tok_seq[tok], p = a.tok_pos[tok];
+  if (s < 0 || p < 0 || (p & 3) != 3) return;
+  const int page = locate(a, s, p, 32);  // errors were flagged by the first launch
+  if (page < 0) return;
+  compress_at(a, p, page, lane);
 }
 
 __global__ void __launch_bounds__(256) append_tokens_kernel(AppendArgs a) {
@@ -109,16 +139,25 @@ __global__ void __launch_bounds__(256) append_compress_kernel(AppendArgs a) {
 }
 
 // Both phases in one CTA (small N, e.g. one token per sequence in decode):
-// the barrier orders every phase-1 write before any phase-2 read.
-constexpr int SMALL_WARPS = 32;
-constexpr int SMALL_MAX_N = 4 * SMALL_WARPS;
-__global__ void __launch_bounds__(SMALL_WARPS * 32) append_small_kernel(AppendArgs a) {
+// the barrier orders every phase-1 write before any phase-2 read; a warp keeps
+// the position and page of its (at most SMALL_PER_WARP) tokens across it.
+constexpr int SMALL_WARPS = 16;
+constexpr int SMALL_PER_WARP = 8;
+constexpr int SMALL_MAX_N = SMALL_PER_WARP * SMALL_WARPS;
+__global__ void __launch_bounds__(SMALL_WARPS * 32, 1) append_small_kernel(AppendArgs a) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_wait();
-  for (int tok = warp; tok < a.N; tok += SMALL_WARPS) write_token(a, tok, lane);
+  int2 pp[SMALL_PER_WARP];  // (page, position) of this warp's tokens
+#pragma unroll
+  for (int u = 0; u < SMALL_PER_WARP; ++u) {
+    const int tok = warp + SMALL_WARPS * u;
+    pp[u] = tok < a.N ? write_token(a, tok, lane) : make_int2(-1, 0);
+  }
   __syncthreads();
   pdl_trigger();
-  for (int tok = warp; tok < a.N; tok += SMALL_WARPS) compress_block(a, tok, lane);
+#pragma unroll
+  for (int u = 0; u < SMALL_PER_WARP; ++u)
+    if (pp[u].x >= 0 && (pp[u].y & 3) == 3) compress_at(a, pp[u].y, pp[u].x, lane);
 }
 
 }  // namespace

@@ -176,10 +176,22 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a) {
     ctot[1] = te;
   }
   cluster.sync();
-  for (int r = 0; r < crank; ++r) {
-    const unsigned *rt = cluster.map_shared_rank(&ctot[0], r);
-    run_gt += rt[0];
-    run_eq += rt[1];
+  {
+    // the counts of every lower-ranked CTA, all loads in flight together
+    unsigned rg[TOPK_CLUSTER], re[TOPK_CLUSTER];
+#pragma unroll
+    for (int r = 0; r < TOPK_CLUSTER; ++r) {
+      const unsigned *rt = cluster.map_shared_rank(&ctot[0], r < crank ? r : crank);
+      rg[r] = rt[0];
+      re[r] = rt[1];
+    }
+#pragma unroll
+    for (int r = 0; r < TOPK_CLUSTER; ++r) {
+      if (r < crank) {
+        run_gt += rg[r];
+        run_eq += re[r];
+      }
+    }
   }
   cluster.sync();  // no CTA leaves while another still reads its counts
 
