@@ -58,6 +58,32 @@ unsigned *device_error_word(cudaError_t *status) {
 
 void set_last_error(const char *msg) { t_last_error = msg ? msg : ""; }
 
+cudaError_t ensure_dynamic_smem(const void *kernel, size_t bytes) {
+  struct Entry {
+    const void *fn;
+    int dev;
+    size_t bytes;
+  };
+  static std::mutex mu;
+  static Entry set[256];
+  static int nset = 0;
+  const int dev = current_device();
+  std::lock_guard<std::mutex> lk(mu);
+  int slot = -1;
+  for (int i = 0; i < nset; ++i)
+    if (set[i].fn == kernel && set[i].dev == dev) slot = i;
+  if (slot >= 0 && set[slot].bytes >= bytes) return cudaSuccess;
+  const cudaError_t e =
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e != cudaSuccess) return e;
+  if (slot >= 0) {
+    set[slot].bytes = bytes;
+  } else if (nset < 256) {
+    set[nset++] = Entry{kernel, dev, bytes};
+  }
+  return cudaSuccess;
+}
+
 int device_sm_count() {
   const int dev = current_device();
   if (dev < 0 || dev >= kMaxDevices) return 148;
@@ -275,6 +301,29 @@ qsa_status qsa_merge(int32_t R, int32_t B, int32_t Hq, int32_t D, const float *o
   } catch (...) {
     return fail(QSA_ERR_CUDA, "qsa_merge: internal exception");
   }
+}
+
+qsa_status qsa_decode_step(const qsa_dims *dims, const qsa_cache *cache, int32_t N,
+                           const int32_t *tok_seq, const int32_t *tok_pos, const void *k_new,
+                           const void *v_new, const void *kidx_new, int32_t B,
+                           const int32_t *seq_lens, const void *q, const void *q_idx,
+                           const float *w, int32_t k, int32_t R, float *scores, int32_t ld_scores,
+                           int32_t *sel, float *o_part, float *lse_part, void *ws,
+                           size_t ws_bytes, void *out, int32_t out_is_bf16, float *lse_out,
+                           qsa_stream_t stream) {
+  qsa_status st = QSA_OK;
+  if (N != 0)
+    st = qsa_append(dims, cache, N, tok_seq, tok_pos, k_new, v_new, kidx_new, stream);
+  if (st == QSA_OK)
+    st = qsa_index_score(dims, cache, B, seq_lens, q_idx, w, scores, ld_scores, stream);
+  if (st == QSA_OK)
+    st = qsa_topk_select(B, seq_lens, scores, ld_scores, k, sel, nullptr, 0, stream);
+  if (st == QSA_OK)
+    st = qsa_sparse_decode(dims, cache, B, seq_lens, q, sel, k, R, o_part, lse_part, ws, ws_bytes,
+                           stream);
+  if (st == QSA_OK && dims != nullptr)
+    st = qsa_merge(R, B, dims->Hq, dims->D, o_part, lse_part, out, out_is_bf16, lse_out, stream);
+  return st;
 }
 
 qsa_status qsa_check_device_errors(qsa_stream_t stream, int32_t *flags) {

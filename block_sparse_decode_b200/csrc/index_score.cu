@@ -600,7 +600,7 @@ cudaError_t launch_tc_t(const qsa_cache &c, TcArgs a, cudaStream_t st) {
     return cudaErrorInvalidValue;
   const size_t smem = 1024 + (size_t)a.stages * STAGE + meta;
   auto kern = index_score_tc_kernel<DI, N>;
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  e = ensure_dynamic_smem(reinterpret_cast<const void *>(kern), smem);
   if (e != cudaSuccess) return e;
   const long long tiles_bound = (long long)a.B * ((a.ld + TC_M - 1) / TC_M);
   const int grid =

@@ -29,6 +29,10 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
   return cudaLaunchKernelEx(&cfg, kern, static_cast<Args &&>(args)...);
 }
 
+// Raise a kernel's dynamic shared memory limit to at least `bytes` on the
+// current device; the driver is called only when the limit has to grow.
+cudaError_t ensure_dynamic_smem(const void *kernel, size_t bytes);
+
 // Device address of this device's error word (set up once per device).
 unsigned *device_error_word(cudaError_t *status);
 int device_sm_count();

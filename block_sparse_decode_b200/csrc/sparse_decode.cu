@@ -543,8 +543,8 @@ DecodePlan plan_decode(const qsa_dims &d, int B, int k, int R) {
 
 template <int ST>
 cudaError_t launch_st(const DecodeArgs &a, const DecodePlan &p, int B, cudaStream_t st) {
-  cudaError_t e = cudaFuncSetAttribute(sparse_decode_kernel<ST>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
+  cudaError_t e =
+      ensure_dynamic_smem(reinterpret_cast<const void *>(sparse_decode_kernel<ST>), p.smem);
   if (e != cudaSuccess) return e;
   e = launch_pdl(sparse_decode_kernel<ST>, dim3(p.ncb, p.nhg, B), DV_WARPS * 32, p.smem, st, a);
   if (e != cudaSuccess || p.ncb == 1) return e;  // one CTA per sequence: nothing to combine

@@ -219,8 +219,7 @@ cudaError_t launch_topk(int B, const int32_t *seq_lens, const float *scores, int
   TopkArgs a{scores, seq_lens, sel, ld, k, err};
   const int per_cta = (ld + TOPK_CLUSTER - 1) / TOPK_CLUSTER;
   const size_t smem = (size_t)per_cta * 4;
-  cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void *>(topk_kernel), smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(TOPK_CLUSTER, B, 1);

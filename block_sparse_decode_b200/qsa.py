@@ -30,7 +30,7 @@ QSA_ERR_TIMEOUT = 5
 EXPORTS = ("qsa_version", "qsa_last_error", "qsa_append", "qsa_index_score",
            "qsa_topk_workspace_size", "qsa_topk_select", "qsa_sparse_decode_workspace_size",
            "qsa_sparse_decode", "qsa_sparse_decode_static", "qsa_merge",
-           "qsa_check_device_errors")
+           "qsa_decode_step", "qsa_check_device_errors")
 
 
 class QsaError(RuntimeError):
@@ -77,6 +77,8 @@ def lib() -> ctypes.CDLL:
         "qsa_sparse_decode": (I32, [DP, CP, I32, P, P, P, I32, I32, P, P, P, SZ, P]),
         "qsa_sparse_decode_static": (I32, [DP, CP, I32, P, P, P, I32, I32, P, P, P]),
         "qsa_merge": (I32, [I32, I32, I32, I32, P, P, P, I32, P, P]),
+        "qsa_decode_step": (I32, [DP, CP, I32, P, P, P, P, P, I32, P, P, P, P, I32, I32, P, I32,
+                                  P, P, P, P, SZ, P, I32, P, P]),
         "qsa_check_device_errors": (I32, [P, ctypes.POINTER(I32)]),
     }
     for name, (res, args) in sig.items():
@@ -130,7 +132,11 @@ class QsaDims:
                    float(d.scale))
 
     def c(self) -> _Dims:
-        return _Dims(self.Hq, self.Hkv, self.D, self.Hi, self.di, self.P, self.scale)
+        c = self.__dict__.get("_c")
+        if c is None:  # built once (the dims are frozen)
+            c = _Dims(self.Hq, self.Hkv, self.D, self.Hi, self.di, self.P, self.scale)
+            object.__setattr__(self, "_c", c)
+        return c
 
 
 @dataclass
@@ -144,12 +150,21 @@ class QsaCache:
     block_table: torch.Tensor  # int32 [num_seqs, max_pages_per_seq]
 
     def c(self) -> _Cache:
+        # rebuilt only when a pool or the block table is replaced
+        key = (self.k_pool.data_ptr(), self.v_pool.data_ptr(), self.kidx_pool.data_ptr(),
+               self.side_pool.data_ptr(), self.block_table.data_ptr(),
+               tuple(self.block_table.shape), int(self.k_pool.shape[0]))
+        hit = self.__dict__.get("_c")
+        if hit is not None and hit[0] == key:
+            return hit[1]
         bf = torch.bfloat16
-        return _Cache(_ptr(self.k_pool, bf, "k_pool"), _ptr(self.v_pool, bf, "v_pool"),
+        c = _Cache(_ptr(self.k_pool, bf, "k_pool"), _ptr(self.v_pool, bf, "v_pool"),
                       _ptr(self.kidx_pool, bf, "kidx_pool"), _ptr(self.side_pool, bf, "side_pool"),
                       _ptr(self.block_table, torch.int32, "block_table"),
                       int(self.block_table.shape[0]), int(self.block_table.shape[1]),
                       int(self.k_pool.shape[0]))
+        self.__dict__["_c"] = (key, c)
+        return c
 
 
 def alloc_cache(dims: QsaDims, num_pages: int, block_table: torch.Tensor,
@@ -286,18 +301,31 @@ def alloc_step(dims: QsaDims, B: int, ld: int, k: int, R: int, device="cuda",
 
 def decode_step(dims: QsaDims, cache: QsaCache, seq_lens, q, q_idx, w, k: int, R: int,
                 buf: StepBuffers, stream=None, append=None):
-    """One QSA decode step: [append] -> score -> top-k -> split attention -> merge.
+    """One QSA decode step: [append] -> score -> top-k -> split attention -> merge,
+    issued by the library's single qsa_decode_step call.
 
     ``append`` is an optional (tok_seq, tok_pos, k_new, v_new, kidx_new) tuple
     written first. Results land in ``buf``.
     """
+    B = int(seq_lens.shape[0])
     if append is not None:
-        qsa_append(dims, cache, *append, stream=stream)
-    qsa_index_score(dims, cache, seq_lens, q_idx, w, buf.scores, stream=stream)
-    qsa_topk_select(seq_lens, buf.scores, k, buf.sel, stream=stream)
-    qsa_sparse_decode(dims, cache, seq_lens, q, buf.sel, k, R, buf.o_part, buf.lse_part, buf.ws,
-                      stream=stream)
-    qsa_merge(buf.o_part, buf.lse_part, buf.out, buf.lse, stream=stream)
+        tok_seq, tok_pos, k_new, v_new, kidx_new = append
+        N = int(tok_seq.shape[0])
+        app = (_ptr(tok_seq, torch.int32, "tok_seq"), _ptr(tok_pos, torch.int32, "tok_pos"),
+               _ptr(k_new, torch.bfloat16, "k_new"), _ptr(v_new, torch.bfloat16, "v_new"),
+               _ptr(kidx_new, torch.bfloat16, "kidx_new"))
+    else:
+        N, app = 0, (None,) * 5
+    _check(lib().qsa_decode_step(
+        ctypes.byref(dims.c()), ctypes.byref(cache.c()), N, *app, B,
+        _ptr(seq_lens, torch.int32, "seq_lens"), _ptr(q, torch.bfloat16, "q"),
+        _ptr(q_idx, torch.bfloat16, "q_idx"), _ptr(w, torch.float32, "w"), int(k), int(R),
+        _ptr(buf.scores, torch.float32, "scores"), int(buf.scores.shape[1]),
+        _ptr(buf.sel, torch.int32, "sel"), _ptr(buf.o_part, torch.float32, "o_part"),
+        _ptr(buf.lse_part, torch.float32, "lse_part"), _ptr(buf.ws, None, "ws"),
+        buf.ws.numel() * buf.ws.element_size(), _ptr(buf.out, None, "out"),
+        1 if buf.out.dtype == torch.bfloat16 else 0, _ptr(buf.lse, torch.float32, "lse"),
+        _stream(stream)))
 
 
 def ld_for(seq_lens) -> int:

@@ -225,6 +225,28 @@ qsa_status qsa_merge(int32_t R, int32_t B, int32_t Hq, int32_t D,
                      const float *o_part, const float *lse_part, void *out,
                      int32_t out_is_bf16, float *lse_out, qsa_stream_t stream);
 
+/* One decode step in one call: qsa_append of the N new tokens (skipped when
+ * N == 0), then qsa_index_score, qsa_topk_select (no workspace),
+ * qsa_sparse_decode and qsa_merge, enqueued in that order on `stream`, with
+ * the arguments documented at each of those calls (the merge writes `out`
+ * [B, Hq, D] and `lse_out` [B, Hq] from o_part / lse_part). The page orders
+ * the steps (section "What the pull request actually changes"); the single
+ * call is an interface convenience of this library that saves the caller
+ * four calls. The calls' own argument checks apply; the first failing call
+ * stops the sequence and its status is returned (calls before it stay
+ * enqueued). */
+qsa_status qsa_decode_step(const qsa_dims *dims, const qsa_cache *cache,
+                           int32_t N, const int32_t *tok_seq,
+                           const int32_t *tok_pos, const void *k_new,
+                           const void *v_new, const void *kidx_new, int32_t B,
+                           const int32_t *seq_lens, const void *q,
+                           const void *q_idx, const float *w, int32_t k,
+                           int32_t R, float *scores, int32_t ld_scores,
+                           int32_t *sel, float *o_part, float *lse_part,
+                           void *ws, size_t ws_bytes, void *out,
+                           int32_t out_is_bf16, float *lse_out,
+                           qsa_stream_t stream);
+
 /* Wait for `stream`, then read and clear the device error word of the
  * current device. *flags receives the bits that were set (0 if none):
  *   1 sequence row out of range    2 page id out of range
