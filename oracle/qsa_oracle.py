@@ -142,11 +142,13 @@ def slice_bounds(nb: int, R: int):
     return [((r * nb) // R, ((r + 1) * nb) // R) for r in range(R)]
 
 
-def attend_slices(q_bits, k_bits, v_bits, sel, L: int, scale: float, R: int):
+def attend_slices(q_bits, k_bits, v_bits, sel, L: int, scale: float, R: int, visible=None):
     """Per-slice partial attention over the selected blocks.
 
     q_bits [Hq, D]; k_bits, v_bits [>=L, Hkv, D]; sel: selected block indices
     (ascending, -1 padding ignored). Query head h reads KV head h // (Hq/Hkv).
+    The slices are those of the nb = ceil(L/4) blocks; the query sees tokens
+    t < L, or t < `visible` when given (a query placed before the end).
     Returns O [R, Hq, D] float64 and LSE [R, Hq] float64 (natural log,
     including the softmax scale).
     """
@@ -161,7 +163,8 @@ def attend_slices(q_bits, k_bits, v_bits, sel, L: int, scale: float, R: int):
     O = np.zeros((R, Hq, D), dtype=np.float64)
     LSE = np.full((R, Hq), NEG_INF, dtype=np.float64)
     for r, (lo, hi) in enumerate(slice_bounds(nb, R)):
-        toks = [t for j in blocks if lo <= j < hi for t in range(4 * j, 4 * j + 4) if t < L]
+        lim = L if visible is None else min(L, visible)
+        toks = [t for j in blocks if lo <= j < hi for t in range(4 * j, 4 * j + 4) if t < lim]
         if not toks:
             continue
         toks = np.asarray(toks)
@@ -174,6 +177,18 @@ def attend_slices(q_bits, k_bits, v_bits, sel, L: int, scale: float, R: int):
             O[r, h] = p @ Vf[toks, g, :]
             LSE[r, h] = lse
     return O, LSE
+
+
+def attend_slices_mq(q_bits, k_bits, v_bits, sel, L: int, scale: float, R: int):
+    """Several decode queries per sequence sharing one selection (multi-query
+    decode, e.g. draft tokens of multi-token prediction): q_bits [Q, Hq, D],
+    query j sits at position L - Q + j and sees the selected tokens
+    t <= L - Q + j. Returns O [R, Q, Hq, D] and LSE [R, Q, Hq] (float64)."""
+    q_all = np.asarray(q_bits)
+    Q = q_all.shape[0]
+    parts = [attend_slices(q_all[j], k_bits, v_bits, sel, L, scale, R, visible=L - Q + j + 1)
+             for j in range(Q)]
+    return (np.stack([o for o, _ in parts], axis=1), np.stack([l for _, l in parts], axis=1))
 
 
 def merge_partials(O, LSE):

@@ -394,3 +394,57 @@ def test_padding_tokens_write_nothing():
     oracle.append_paged(*pools, bt, d.P, [-1, 0, -1, 1], [3, -1, 7, -5], K, V, X)
     for a, b in zip(pools, before):
         assert np.array_equal(a, b)
+
+
+# ------------------------------------------------------------ multi-query decode
+
+def _mq_case(L, Q, seed, D=32, Hq=8, Hkv=2):
+    g = torch.Generator().manual_seed(seed)
+    K = torch.randn(L, Hkv, D, generator=g).to(torch.bfloat16)
+    V = torch.randn(L, Hkv, D, generator=g).to(torch.bfloat16)
+    q = torch.randn(Q, Hq, D, generator=g).to(torch.bfloat16)
+    return q, K, V
+
+
+@pytest.mark.parametrize("L,Q", [(37, 1), (37, 2), (40, 3), (5, 4), (1000, 2)])
+def test_multi_query_full_selection_equals_masked_sdpa_fp64(L, Q):
+    # every block selected, one slice: query j is dense attention over the
+    # tokens t <= L - Q + j (a bottom-right causal mask), by torch's SDPA
+    q, K, V = _mq_case(L, Q, seed=L * 10 + Q)
+    nb = (L + 3) // 4
+    scale = 0.17
+    O, LSE = oracle.attend_slices_mq(bits(q), bits(K), bits(V), np.arange(nb), L, scale, 1)
+    Hq, G = q.shape[1], q.shape[1] // K.shape[1]
+    qh = q.to(torch.float64).permute(1, 0, 2)[None]                          # [1, Hq, Q, D]
+    Kh = K.to(torch.float64).repeat_interleave(G, dim=1).permute(1, 0, 2)[None]
+    Vh = V.to(torch.float64).repeat_interleave(G, dim=1).permute(1, 0, 2)[None]
+    mask = torch.arange(L)[None, :] <= (L - Q + torch.arange(Q))[:, None]   # [Q, L]
+    ref = torch.nn.functional.scaled_dot_product_attention(qh, Kh, Vh, attn_mask=mask,
+                                                           scale=scale)
+    assert np.allclose(O[0], ref[0].permute(1, 0, 2).numpy(), atol=1e-10, rtol=0)
+    z = (qh @ Kh.transpose(-1, -2)) * scale
+    z = z.masked_fill(~mask, float("-inf"))
+    assert np.allclose(LSE[0], torch.logsumexp(z, dim=-1)[0].T.numpy(), atol=1e-10, rtol=0)
+
+
+def test_multi_query_split_merge_equals_unsplit_and_hides_future_blocks():
+    L, Q = 203, 3
+    q, K, V = _mq_case(L, Q, seed=5)
+    nb = (L + 3) // 4
+    sel = np.array([0, 3, 7, 20, 33, 49, nb - 1])  # the last block holds the queries' tokens
+    O1, L1 = oracle.attend_slices_mq(bits(q), bits(K), bits(V), sel, L, 0.2, 1)
+    for R in (2, 5, 51):
+        O, Ls = oracle.attend_slices_mq(bits(q), bits(K), bits(V), sel, L, 0.2, R)
+        for j in range(Q):
+            Om, Lm = oracle.merge_partials(O[:, j], Ls[:, j])
+            assert np.abs(Om - O1[0, j]).max() <= 1e-12
+            assert np.abs(Lm - L1[0, j]).max() <= 1e-12
+    # R = nb: the last slice is exactly the last block {200, 201, 202}: query 0
+    # (position 200) sees one token of it, query 2 all three; a slice holding
+    # only tokens after a query is empty for that query
+    O, Ls = oracle.attend_slices_mq(bits(q), bits(K), bits(V), np.array([nb - 1]), L, 0.2, nb)
+    assert np.all(Ls[: nb - 1] == -np.inf)
+    assert np.all(np.isfinite(Ls[nb - 1]))
+    Lq, Kq = 201, K[:201]
+    O0, L0 = oracle.attend_slices(bits(q[0]), bits(Kq), bits(V[:201]), np.array([50]), Lq, 0.2, 1)
+    assert np.abs(O[nb - 1, 0] - O0[0]).max() <= 1e-12   # query 0 = single query over t < 201
