@@ -54,6 +54,9 @@ def parse():
     ap.add_argument("--R", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--queries", type=int, default=1,
+                    help="decode queries per sequence (multi-query decode: each step appends "
+                         "this many tokens per sequence and decodes all of them)")
     return ap.parse_args()
 
 
@@ -186,7 +189,8 @@ def run_ours(args, rank, world, local_rank):
     dims = qsa.QsaDims.of(wl.dims)
     B = wl.B
 
-    # cache: prefill L-1 tokens in bulk; the step appends token L-1
+    Qn = args.queries
+    # cache: prefill L - Qn tokens in bulk; the step appends tokens L - Qn .. L - 1
     cache = qsa.alloc_cache(dims, wl.num_pages, wl.block_table, device=dev)
     T = sum(wl.cap_lens)
     tok_seq = torch.empty(T, dtype=torch.int32, device=dev)
@@ -195,24 +199,39 @@ def run_ours(args, rank, world, local_rank):
         o = wl.tok_off[b]
         tok_seq[o:o + L] = b
         tok_pos[o:o + L] = torch.arange(L, dtype=torch.int32, device=dev)
-        tok_seq[o + wl.seq_lens[b] - 1:o + L] = -1
+        tok_seq[o + wl.seq_lens[b] - Qn:o + L] = -1
     qsa.qsa_append(dims, cache, tok_seq, tok_pos, wl.k_tok, wl.v_tok, wl.kidx_tok)
     del tok_seq, tok_pos
-    rows = torch.tensor([wl.tok_off[b] + L - 1 for b, L in enumerate(wl.seq_lens)], device=dev)
+    rows = torch.tensor([wl.tok_off[b] + L - Qn + j for b, L in enumerate(wl.seq_lens)
+                         for j in range(Qn)], device=dev)
+    if Qn == 1:
+        q_step = wl.q.contiguous()
+    else:  # one decode query per new token
+        gq = torch.Generator(device=dev).manual_seed(seed + 17)
+        q_step = torch.randn((B, Qn, wl.dims.Hq, wl.dims.D), generator=gq,
+                             device=dev).to(torch.bfloat16)
     step_in = dict(
-        tok_seq=torch.arange(B, dtype=torch.int32, device=dev),
-        tok_pos=torch.tensor([L - 1 for L in wl.seq_lens], dtype=torch.int32, device=dev),
+        tok_seq=torch.arange(B, dtype=torch.int32, device=dev).repeat_interleave(Qn),
+        tok_pos=torch.tensor([L - Qn + j for L in wl.seq_lens for j in range(Qn)],
+                             dtype=torch.int32, device=dev),
         k_new=wl.k_tok[rows].contiguous(), v_new=wl.v_tok[rows].contiguous(),
         kidx_new=wl.kidx_tok[rows].contiguous(),
         seq_lens=torch.tensor(wl.seq_lens, dtype=torch.int32, device=dev),
-        q=wl.q.contiguous(), q_idx=wl.q_idx.contiguous(), w=wl.w.contiguous())
+        q=q_step, q_idx=wl.q_idx.contiguous(), w=wl.w.contiguous())
     ld = qsa.ld_for(wl.seq_lens)
     buf = qsa.alloc_step(dims, B, ld, k, R, device=dev)
+    if Qn > 1:  # partials, merged output and scratch with a query axis
+        buf.o_part = torch.empty((R, B, Qn, dims.Hq, dims.D), dtype=torch.float32, device=dev)
+        buf.lse_part = torch.empty((R, B, Qn, dims.Hq), dtype=torch.float32, device=dev)
+        buf.out = torch.empty((B * Qn, dims.Hq, dims.D), dtype=torch.bfloat16, device=dev)
+        buf.lse = torch.empty((B * Qn, dims.Hq), dtype=torch.float32, device=dev)
+        buf.ws = torch.empty(max(16, qsa.qsa_sparse_decode_mq_workspace_size(dims, B, Qn, k, R)),
+                             dtype=torch.uint8, device=dev)
     qsa.qsa_check_device_errors()
 
     # host-side copies for the oracle baseline (seq 0), then free the token arrays
     cpu_sample = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and Qn == 1:
         K0, V0, X0 = wl.seq_tokens(0)
         cpu_sample = dict(K=K0.cpu(), V=V0.cpu(), X=X0.cpu(), q=wl.q[0].cpu(),
                           q_idx=wl.q_idx[0].cpu(), w=wl.w[0].cpu(), L=wl.seq_lens[0])
@@ -227,10 +246,14 @@ def run_ours(args, rank, world, local_rank):
         "index_score": lambda: qsa.qsa_index_score(dims, cache, si["seq_lens"], si["q_idx"],
                                                    si["w"], buf.scores),
         "topk_select": lambda: qsa.qsa_topk_select(si["seq_lens"], buf.scores, k, buf.sel),
-        "sparse_decode": lambda: qsa.qsa_sparse_decode(dims, cache, si["seq_lens"], si["q"],
-                                                       buf.sel, k, R, buf.o_part, buf.lse_part,
-                                                       buf.ws),
-        "merge": lambda: qsa.qsa_merge(buf.o_part, buf.lse_part, buf.out, buf.lse),
+        "sparse_decode": (lambda: qsa.qsa_sparse_decode(dims, cache, si["seq_lens"], si["q"],
+                                                        buf.sel, k, R, buf.o_part, buf.lse_part,
+                                                        buf.ws)) if Qn == 1 else
+                         (lambda: qsa.qsa_sparse_decode_mq(dims, cache, si["seq_lens"], si["q"],
+                                                           buf.sel, k, R, buf.o_part,
+                                                           buf.lse_part, buf.ws)),
+        "merge": lambda: qsa.qsa_merge(buf.o_part.view(R, B * Qn, dims.Hq, dims.D),
+                                       buf.lse_part.view(R, B * Qn, dims.Hq), buf.out, buf.lse),
     }
 
     def step():
@@ -301,7 +324,7 @@ def run_ours(args, rank, world, local_rank):
     # e2e: host buffers in pinned memory, copies inside the timed region,
     # calls made eagerly through the binding (the user's API)
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and Qn == 1:
         # the step's inputs travel in one pinned staging buffer (one copy), the
         # merged output and its LSE in one device buffer (one copy back)
         def packed(tensors, device, pin):
@@ -353,7 +376,13 @@ def run_ours(args, rank, world, local_rank):
     dec_ms = kern_ms["sparse_decode"]
     achieved = side_b / (score_ms / 1e3) / 1e9
     traffic = profile_traffic("index_score.cu", "index_score_b8x256k.md")
-    attended = sum(min(4 * k, L) for L in wl.seq_lens)
+    attended = Qn * sum(min(4 * k, L) for L in wl.seq_lens)
+    # kernels per step: append, score, top-k, merge, and per group of two
+    # queries the decode plus (when sequences are split over CTAs) its combine
+    nhg = (dims.Hkv + 3) // 4
+    ntmax = (k + 3) // 4 + R - 1
+    ncb = max(1, min(296 // (B * nhg), ntmax), -(-ntmax // 256))
+    launches = 4 + ((Qn + 1) // 2) * (2 if ncb > 1 else 1)
     res = {
         "metric": METRIC,
         "value": job_rate(world, B, ms_per_step),
@@ -369,12 +398,15 @@ def run_ours(args, rank, world, local_rank):
         "data": "synthetic",
         "config": {"workload": f"{args.workload}: B={B} x L={max(wl.seq_lens)} tokens, "
                                f"32q/4kv heads x 128, indexer 16x128, top-{k} blocks of 4, "
-                               f"R={R}, paged P=64 (shuffled)",
-                   "batch": B, "context": max(wl.seq_lens), "k": k, "R": R,
+                               f"R={R}, paged P=64 (shuffled)"
+                               + (f", {Qn} decode queries per sequence (multi-query)"
+                                  if Qn > 1 else ""),
+                   "batch": B, "context": max(wl.seq_lens), "k": k, "R": R, "queries": Qn,
                    "l2": "flushed before every timed step (512 MiB write, then 512 MiB read)",
                    "step": "CUDA graph of append+score+topk+decode+merge",
                    "parallelism": f"replicas x{world}"},
         "attended_tokens_per_s": job_rate(world, attended, ms_per_step),
+        "query_tokens_per_s": job_rate(world, B * Qn, ms_per_step),
         "step_us_p10_p50_p90": [round(1e3 * float(np.percentile(step_ms, q)), 2)
                                 for q in (10, 50, 90)],
         "roofline": {"bound": "hbm", "kernel": "qsa_index_score", "achieved": achieved,
@@ -390,7 +422,7 @@ def run_ours(args, rank, world, local_rank):
             "gbs": (side_b + kv_b) / ((score_ms + dec_ms) / 1e3) / 1e9,
             "frac": (side_b + kv_b) / ((score_ms + dec_ms) / 1e3) / 1e9 / peak},
         "step_roofline_frac": (side_b + kv_b) / (ms_per_step / 1e3) / 1e9 / peak,
-        "gpu_launches": 5 * args.steps,
+        "gpu_launches": launches * args.steps,
         "clocks": clk.summary(),
         "e2e": e2e,
     }

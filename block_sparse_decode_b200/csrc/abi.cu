@@ -246,21 +246,36 @@ qsa_status qsa_topk_select(int32_t B, const int32_t *seq_lens, const float *scor
 }
 
 size_t qsa_sparse_decode_workspace_size(const qsa_dims *dims, int32_t B, int32_t k, int32_t R) {
-  if (dims == nullptr || B <= 0 || k <= 0 || R <= 0 || dims->Hkv <= 0 || dims->Hq <= 0)
+  return qsa_sparse_decode_mq_workspace_size(dims, B, 1, k, R);
+}
+
+size_t qsa_sparse_decode_mq_workspace_size(const qsa_dims *dims, int32_t B, int32_t Qn, int32_t k,
+                                           int32_t R) {
+  if (dims == nullptr || B <= 0 || Qn <= 0 || k <= 0 || R <= 0 || dims->Hkv <= 0 || dims->Hq <= 0)
     return 0;
-  return decode_ws_bytes(*dims, B, k, R);
+  return decode_ws_bytes(*dims, B, Qn, k, R);
 }
 
 qsa_status qsa_sparse_decode(const qsa_dims *dims, const qsa_cache *cache, int32_t B,
                              const int32_t *seq_lens, const void *q, const int32_t *sel,
                              int32_t k, int32_t R, float *o_part, float *lse_part, void *ws,
                              size_t ws_bytes, qsa_stream_t stream) {
+  return qsa_sparse_decode_mq(dims, cache, B, 1, seq_lens, q, sel, k, R, o_part, lse_part, ws,
+                              ws_bytes, stream);
+}
+
+qsa_status qsa_sparse_decode_mq(const qsa_dims *dims, const qsa_cache *cache, int32_t B,
+                                int32_t Qn, const int32_t *seq_lens, const void *q,
+                                const int32_t *sel, int32_t k, int32_t R, float *o_part,
+                                float *lse_part, void *ws, size_t ws_bytes,
+                                qsa_stream_t stream) {
   try {
     QSA_TRY(check_dims(dims));
     QSA_TRY(check_cache(cache, true, false));
     if (B < 0 || B > 65535) return fail(QSA_ERR_INVALID_ARG, "B=%d outside [0, 65535]", B);
     if (B > cache->num_seqs)
       return fail(QSA_ERR_INVALID_ARG, "B=%d exceeds block_table rows %d", B, cache->num_seqs);
+    if (Qn < 1 || Qn > 8) return fail(QSA_ERR_UNSUPPORTED, "Qn=%d outside [1, 8]", Qn);
     if (k < 1 || k > 4096) return fail(QSA_ERR_UNSUPPORTED, "k=%d outside [1, 4096]", k);
     if (R < 1 || R > 64) return fail(QSA_ERR_UNSUPPORTED, "R=%d outside [1, 64]", R);
     if (B == 0) return ok();
@@ -269,11 +284,11 @@ qsa_status qsa_sparse_decode(const qsa_dims *dims, const qsa_cache *cache, int32
       return fail(QSA_ERR_INVALID_ARG, "an argument array is NULL");
     if (!aligned16(q) || !aligned16(o_part) || !aligned16(ws))
       return fail(QSA_ERR_INVALID_ARG, "q / o_part / ws not 16-byte aligned");
-    const size_t need = decode_ws_bytes(*dims, B, k, R);
+    const size_t need = decode_ws_bytes(*dims, B, Qn, k, R);
     if (ws_bytes < need)
       return fail(QSA_ERR_INVALID_ARG, "workspace %zu bytes < %zu needed", ws_bytes, need);
     QSA_ERRWORD(err);
-    return cuda_status(launch_sparse_decode(*dims, *cache, B, seq_lens, q, sel, k, R, o_part,
+    return cuda_status(launch_sparse_decode(*dims, *cache, B, Qn, seq_lens, q, sel, k, R, o_part,
                                             lse_part, ws, err,
                                             reinterpret_cast<cudaStream_t>(stream)),
                        "qsa_sparse_decode launch");

@@ -52,8 +52,8 @@ constexpr int TOPK_MAX_KEYS_PER_CTA = 49152;  // 192 KiB of keys per CTA
 cudaError_t launch_topk(int B, const int32_t *seq_lens, const float *scores, int ld, int k,
                         int32_t *sel, unsigned *err, cudaStream_t st);
 
-size_t decode_ws_bytes(const qsa_dims &d, int B, int k, int R);
-cudaError_t launch_sparse_decode(const qsa_dims &d, const qsa_cache &c, int B,
+size_t decode_ws_bytes(const qsa_dims &d, int B, int Qn, int k, int R);
+cudaError_t launch_sparse_decode(const qsa_dims &d, const qsa_cache &c, int B, int Qn,
                                  const int32_t *seq_lens, const void *q, const int32_t *sel,
                                  int k, int R, float *o_part, float *lse_part, void *ws,
                                  unsigned *err, cudaStream_t st);

@@ -58,16 +58,18 @@ constexpr int DV_SLOTS = DV_CTAS_PER_SM * 148;  // CTAs in flight on a B200
 constexpr size_t DV_SMEM_LIMIT = 113 * 1024;    // shared memory per CTA so that two fit an SM
 constexpr int DV_CB_ROWS = 8;                   // query-head rows per combine CTA
 constexpr int DV_CB_BATCH = 8;                  // records loaded together by the combine
+constexpr int DV_QGROUP = 2;                    // queries of a sequence per pass over K/V
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 
 struct DecodeArgs {
-  const __nv_bfloat16 *k_pool, *v_pool, *q;
+  const __nv_bfloat16 *k_pool, *v_pool, *q;  // q [B, Qn, Hq, D]
   const int32_t *block_table, *seq_lens, *sel;
-  float *o_part, *lse_part;  // [R, B, Hq, D], [R, B, Hq]
-  float *rec_o, *rec_lse;    // [B, rb, Hq, D], [B, rb, Hq]: partials of shared slices
+  float *o_part, *lse_part;  // [R, B, Qn, Hq, D], [R, B, Qn, Hq]
+  float *rec_o, *rec_lse;    // [B, rb, QN, Hq, D], [B, rb, QN, Hq]: shared-slice partials
   int2 *span;                // [B, R]: contributors (c_lo, c_hi) of a shared slice
   int B, Hq, Hkv, G, P, max_pages, num_pages, k, k_pad, R, ncb, rb;
+  int Qn, q0, qn;            // queries per sequence; first query and size of this group
   int ring_bytes;            // DV_WARPS * ST * DV_STAGE
   float scale_log2;
   unsigned *err;
@@ -116,65 +118,86 @@ struct Acc {
   }
 };
 
-// One 16-token tile of one head: K rows at kbase, V rows at vbase (swizzled), token
-// i valid iff bit i of `valid`.
-__device__ __forceinline__ void attend_tile(Acc &s_, uint32_t kbase, uint32_t vbase, unsigned valid,
-                                            const uint32_t (&qf)[8][2], float scale_log2,
+// One 16-token tile of one head for QN queries of the same sequence: K rows
+// at kbase, V rows at vbase (swizzled); token i valid for query qq iff bit i
+// of valid[qq]. Each K and V fragment is loaded once for all queries.
+template <int QN>
+__device__ __forceinline__ void attend_tile(Acc (&st)[QN], uint32_t kbase, uint32_t vbase,
+                                            const unsigned (&valid)[QN],
+                                            const uint32_t (&qf)[QN][8][2], float scale_log2,
                                             int lane) {
   const int gq = lane >> 2;
   const int arow = (lane & 7) + ((lane >> 3) & 1) * 8;  // K: non-transposed x4
   const int akc = lane >> 4;
   const int vrow = (lane & 7) + ((lane >> 4) & 1) * 8;  // V: transposed x4
   const int vkc = (lane >> 3) & 1;
-  // S^T[16 tokens x 8 heads] in two independent accumulation chains
-  float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+  // S^T[16 tokens x 8 heads] per query, in two independent accumulation chains
+  float sa[QN][4], sb[QN][4];
+#pragma unroll
+  for (int qq = 0; qq < QN; ++qq)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) sa[qq][i] = sb[qq][i] = 0.f;
 #pragma unroll
   for (int ks = 0; ks < 4; ++ks) {
     uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
     ldsm_x4(kbase + swz(arow, 2 * ks + akc, DV_ROWB), a0, a1, a2, a3);
     ldsm_x4(kbase + swz(arow, 2 * (ks + 4) + akc, DV_ROWB), b0, b1, b2, b3);
-    mma_bf16_16816(sa, a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
-    mma_bf16_16816(sb, b0, b1, b2, b3, qf[ks + 4][0], qf[ks + 4][1]);
-  }
-  // s[0], s[1]: token gq, heads 2tq, 2tq+1; s[2], s[3]: token gq + 8
-  const bool v0 = (valid >> gq) & 1u, v1 = (valid >> (gq + 8)) & 1u;
-  const float x0 = v0 ? (sa[0] + sb[0]) * scale_log2 : -INFINITY;
-  const float x1 = v0 ? (sa[1] + sb[1]) * scale_log2 : -INFINITY;
-  const float x2 = v1 ? (sa[2] + sb[2]) * scale_log2 : -INFINITY;
-  const float x3 = v1 ? (sa[3] + sb[3]) * scale_log2 : -INFINITY;
-  float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
 #pragma unroll
-  for (int o_ = 4; o_ < 32; o_ <<= 1) {
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o_));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o_));
+    for (int qq = 0; qq < QN; ++qq) {
+      mma_bf16_16816(sa[qq], a0, a1, a2, a3, qf[qq][ks][0], qf[qq][ks][1]);
+      mma_bf16_16816(sb[qq], b0, b1, b2, b3, qf[qq][ks + 4][0], qf[qq][ks + 4][1]);
+    }
   }
-  const float mn0 = fmaxf(s_.m0, mx0), mn1 = fmaxf(s_.m1, mx1);
-  const float base0 = mn0 == -INFINITY ? 0.f : mn0, base1 = mn1 == -INFINITY ? 0.f : mn1;
-  const float c0 = exp2f(s_.m0 - base0), c1 = exp2f(s_.m1 - base1);
-  const float p0 = exp2f(x0 - base0), p1 = exp2f(x1 - base1);
-  const float p2 = exp2f(x2 - base0), p3 = exp2f(x3 - base1);
-  float r0 = p0 + p2, r1 = p1 + p3;
+  float c0[QN], c1[QN];
+  uint32_t pb0[QN], pb1[QN];
 #pragma unroll
-  for (int o_ = 4; o_ < 32; o_ <<= 1) {
-    r0 += __shfl_xor_sync(0xffffffffu, r0, o_);
-    r1 += __shfl_xor_sync(0xffffffffu, r1, o_);
+  for (int qq = 0; qq < QN; ++qq) {
+    Acc &s_ = st[qq];
+    // s[0], s[1]: token gq, heads 2tq, 2tq+1; s[2], s[3]: token gq + 8
+    const bool v0 = (valid[qq] >> gq) & 1u, v1 = (valid[qq] >> (gq + 8)) & 1u;
+    const float x0 = v0 ? (sa[qq][0] + sb[qq][0]) * scale_log2 : -INFINITY;
+    const float x1 = v0 ? (sa[qq][1] + sb[qq][1]) * scale_log2 : -INFINITY;
+    const float x2 = v1 ? (sa[qq][2] + sb[qq][2]) * scale_log2 : -INFINITY;
+    const float x3 = v1 ? (sa[qq][3] + sb[qq][3]) * scale_log2 : -INFINITY;
+    float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+    for (int o_ = 4; o_ < 32; o_ <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o_));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o_));
+    }
+    const float mn0 = fmaxf(s_.m0, mx0), mn1 = fmaxf(s_.m1, mx1);
+    const float base0 = mn0 == -INFINITY ? 0.f : mn0, base1 = mn1 == -INFINITY ? 0.f : mn1;
+    c0[qq] = exp2f(s_.m0 - base0);
+    c1[qq] = exp2f(s_.m1 - base1);
+    const float p0 = exp2f(x0 - base0), p1 = exp2f(x1 - base1);
+    const float p2 = exp2f(x2 - base0), p3 = exp2f(x3 - base1);
+    float r0 = p0 + p2, r1 = p1 + p3;
+#pragma unroll
+    for (int o_ = 4; o_ < 32; o_ <<= 1) {
+      r0 += __shfl_xor_sync(0xffffffffu, r0, o_);
+      r1 += __shfl_xor_sync(0xffffffffu, r1, o_);
+    }
+    s_.l0 = s_.l0 * c0[qq] + r0;
+    s_.l1 = s_.l1 * c1[qq] + r1;
+    s_.m0 = mn0;
+    s_.m1 = mn1;
+    // P^T (tokens x heads) in accumulator layout -> B operand (k = tokens, n = heads)
+    pb0[qq] = movmatrix_t(pack_bf16x2(p0, p1));
+    pb1[qq] = movmatrix_t(pack_bf16x2(p2, p3));
   }
-  s_.l0 = s_.l0 * c0 + r0;
-  s_.l1 = s_.l1 * c1 + r1;
-  s_.m0 = mn0;
-  s_.m1 = mn1;
-  // P^T (tokens x heads) in accumulator layout -> B operand (k = tokens, n = heads)
-  const uint32_t pb0 = movmatrix_t(pack_bf16x2(p0, p1));
-  const uint32_t pb1 = movmatrix_t(pack_bf16x2(p2, p3));
 #pragma unroll
   for (int mt = 0; mt < 8; ++mt) {
-    s_.o[mt][0] *= c0;
-    s_.o[mt][1] *= c1;
-    s_.o[mt][2] *= c0;
-    s_.o[mt][3] *= c1;
     uint32_t a0, a1, a2, a3;
     ldsm_x4_t(vbase + swz(vrow, 2 * mt + vkc, DV_ROWB), a0, a1, a2, a3);
-    mma_bf16_16816(s_.o[mt], a0, a1, a2, a3, pb0, pb1);
+#pragma unroll
+    for (int qq = 0; qq < QN; ++qq) {
+      Acc &s_ = st[qq];
+      s_.o[mt][0] *= c0[qq];
+      s_.o[mt][1] *= c1[qq];
+      s_.o[mt][2] *= c0[qq];
+      s_.o[mt][3] *= c1[qq];
+      mma_bf16_16816(s_.o[mt], a0, a1, a2, a3, pb0[qq], pb1[qq]);
+    }
   }
 }
 
@@ -214,7 +237,7 @@ __device__ __forceinline__ void tile_range(int c, int NT, int ncb, int &v0, int 
   n = (int)(((long long)(c + 1) * NT) / ncb) - v0;
 }
 
-template <int ST>
+template <int ST, int QN>
 __global__ void __launch_bounds__(DV_WARPS * 32, DV_CTAS_PER_SM) sparse_decode_kernel(DecodeArgs a) {
   extern __shared__ __align__(1024) unsigned char smem[];
   __shared__ int s_st[DV_RMAX], s_ct[DV_RMAX], s_pre[DV_RMAX + 1];
@@ -226,8 +249,9 @@ __global__ void __launch_bounds__(DV_WARPS * 32, DV_CTAS_PER_SM) sparse_decode_k
   const bool has_head = g < a.Hkv;
   // shared memory: ring | selection row | page table
   int32_t *s_sel = reinterpret_cast<int32_t *>(smem + a.ring_bytes);
-  int32_t *s_row = s_sel + a.k_pad;                                    // first pool row of a block
-  uint8_t *s_nv = reinterpret_cast<uint8_t *>(s_row + DV_TBL_BLOCKS);  // its valid tokens
+  int32_t *s_row = s_sel + a.k_pad;               // first pool row of a block
+  int32_t *s_blk = s_row + DV_TBL_BLOCKS;         // its block index (-1: none)
+  uint8_t *s_nv = reinterpret_cast<uint8_t *>(s_blk + DV_TBL_BLOCKS);  // its valid tokens
 
   // (1) L_b, the block-table row into L2, the query; then, once the top-k
   // kernel before this one has finished, the selection row
@@ -240,17 +264,18 @@ __global__ void __launch_bounds__(DV_WARPS * 32, DV_CTAS_PER_SM) sparse_decode_k
     for (int i = c + CL * tid; i < lines; i += CL * (int)blockDim.x)
       asm volatile("prefetch.global.L2 [%0];\n" ::"l"(bt_row + ((size_t)i << 7)));
   }
-  // query fragments (B operand of S^T = K Q^T): head g*G + lane/4
+  // query fragments (B operand of S^T = K Q^T): query a.q0 + qq, head g*G + lane/4
   const int gq = lane >> 2, tq = lane & 3;
-  uint32_t qf[8][2];
-  {
+  uint32_t qf[QN][8][2];
+#pragma unroll
+  for (int qq = 0; qq < QN; ++qq) {
     const bool hv = has_head && gq < a.G;
     const uint32_t *qrow = reinterpret_cast<const uint32_t *>(
-        a.q + ((size_t)b * a.Hq + (hv ? g * a.G + gq : 0)) * DV_D);
+        a.q + (((size_t)b * a.Qn + a.q0 + qq) * a.Hq + (hv ? g * a.G + gq : 0)) * DV_D);
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
-      qf[ks][0] = hv ? qrow[ks * 8 + tq] : 0u;
-      qf[ks][1] = hv ? qrow[ks * 8 + 4 + tq] : 0u;
+      qf[qq][ks][0] = hv ? qrow[ks * 8 + tq] : 0u;
+      qf[qq][ks][1] = hv ? qrow[ks * 8 + 4 + tq] : 0u;
     }
   }
   pdl_wait();
@@ -319,18 +344,18 @@ __global__ void __launch_bounds__(DV_WARPS * 32, DV_CTAS_PER_SM) sparse_decode_k
     ntile = DV_TBL_TILES;
   }
   const int nslot = 4 * ntile;
-  for (int q0 = 0; q0 < nslot; q0 += 4 * (int)blockDim.x) {
+  for (int base = 0; base < nslot; base += 4 * (int)blockDim.x) {
     long long idx[4];
     int jj[4], pg[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const int q = q0 + tid + u * (int)blockDim.x;
+      const int slot = base + tid + u * (int)blockDim.x;
       idx[u] = -1;
       jj[u] = 0;
-      if (q < nslot) {
-        const int v = v0 + (q >> 2);
+      if (slot < nslot) {
+        const int v = v0 + (slot >> 2);
         const int r = slice_of_tile(s_pre, a.R, v);
-        const int off = 4 * (v - s_pre[r]) + (q & 3);
+        const int off = 4 * (v - s_pre[r]) + (slot & 3);
         if (off < s_ct[r]) {
           const int j = s_sel[s_st[r] + off];
           if (j < 0 || j >= nb) {
@@ -351,8 +376,8 @@ __global__ void __launch_bounds__(DV_WARPS * 32, DV_CTAS_PER_SM) sparse_decode_k
     for (int u = 0; u < 4; ++u) pg[u] = idx[u] >= 0 ? __ldg(a.block_table + idx[u]) : -1;
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const int q = q0 + tid + u * (int)blockDim.x;
-      if (q < nslot) {
+      const int slot = base + tid + u * (int)blockDim.x;
+      if (slot < nslot) {
         int row = -1, nv = 0;
         if (idx[u] >= 0) {
           if (pg[u] < 0 || pg[u] >= a.num_pages) {
@@ -362,8 +387,9 @@ __global__ void __launch_bounds__(DV_WARPS * 32, DV_CTAS_PER_SM) sparse_decode_k
             nv = min(4, L - 4 * jj[u]);
           }
         }
-        s_row[q] = row;
-        s_nv[q] = (uint8_t)nv;
+        s_row[slot] = row;
+        s_blk[slot] = nv > 0 ? jj[u] : -1;
+        s_nv[slot] = (uint8_t)nv;
       }
     }
   }
@@ -387,10 +413,13 @@ __global__ void __launch_bounds__(DV_WARPS * 32, DV_CTAS_PER_SM) sparse_decode_k
   if (has_head && c == 0) {
     for (int r = 0; r < a.R; ++r) {
       if (s_ct[r] != 0) continue;
-      for (int h = 0; h < a.G; ++h) {
-        const size_t row = ((size_t)r * a.B + b) * a.Hq + g * a.G + h;
-        reinterpret_cast<float4 *>(a.o_part + row * DV_D)[lane] = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (lane == 0) a.lse_part[row] = -INFINITY;
+      for (int qq = 0; qq < QN; ++qq) {
+        for (int h = 0; h < a.G; ++h) {
+          const size_t row = (((size_t)r * a.B + b) * a.Qn + a.q0 + qq) * a.Hq + g * a.G + h;
+          reinterpret_cast<float4 *>(a.o_part + row * DV_D)[lane] =
+              make_float4(0.f, 0.f, 0.f, 0.f);
+          if (lane == 0) a.lse_part[row] = -INFINITY;
+        }
       }
     }
   }
@@ -422,20 +451,25 @@ __global__ void __launch_bounds__(DV_WARPS * 32, DV_CTAS_PER_SM) sparse_decode_k
 #pragma unroll
     for (int t = 0; t < ST - 1; ++t) issue(t);
 
-    Acc acc;
-    acc.reset();
+    Acc acc[QN];
+#pragma unroll
+    for (int qq = 0; qq < QN; ++qq) acc[qq].reset();
     int cur = -1;                            // slice of the running segment
     int rs = slice_of_tile(s_pre, a.R, v0);  // slice of the current tile
     // (5) partial of slice r over this CTA's tiles
     auto flush = [&](int r) {
       int c_lo, c_hi;
       contributors(r, c_lo, c_hi);
-      if (c_lo == c_hi) {  // the only contributor: the partial is slice r's result
-        const size_t row = ((size_t)r * a.B + b) * a.Hq + g * a.G;
-        store_partial(acc, a.o_part + row * DV_D, a.lse_part + row, a.G, lane);
-      } else {  // shared with neighbouring CTAs: a record for the combine kernel
-        const size_t row = ((size_t)b * a.rb + c + r) * a.Hq + g * a.G;
-        store_partial(acc, a.rec_o + row * DV_D, a.rec_lse + row, a.G, lane);
+#pragma unroll
+      for (int qq = 0; qq < QN; ++qq) {
+        if (c_lo == c_hi) {  // the only contributor: the partial is slice r's result
+          const size_t row =
+              (((size_t)r * a.B + b) * a.Qn + a.q0 + qq) * a.Hq + g * a.G;
+          store_partial(acc[qq], a.o_part + row * DV_D, a.lse_part + row, a.G, lane);
+        } else {  // shared with neighbouring CTAs: a record for the combine kernel
+          const size_t row = (((size_t)b * a.rb + c + r) * QN + qq) * a.Hq + g * a.G;
+          store_partial(acc[qq], a.rec_o + row * DV_D, a.rec_lse + row, a.G, lane);
+        }
       }
     };
     for (int t = 0; t < ntile; ++t) {
@@ -444,7 +478,8 @@ __global__ void __launch_bounds__(DV_WARPS * 32, DV_CTAS_PER_SM) sparse_decode_k
       if (rs != cur) {
         if (cur >= 0) {
           flush(cur);
-          acc.reset();
+#pragma unroll
+          for (int qq = 0; qq < QN; ++qq) acc[qq].reset();
         }
         cur = rs;
       }
@@ -453,10 +488,33 @@ __global__ void __launch_bounds__(DV_WARPS * 32, DV_CTAS_PER_SM) sparse_decode_k
       cp_async_wait<ST - 1>();
       __syncwarp();
       unsigned valid = 0;
+      int jlast = -1;
 #pragma unroll
-      for (int blk = 0; blk < 4; ++blk) valid |= ((1u << s_nv[4 * t + blk]) - 1u) << (4 * blk);
+      for (int blk = 0; blk < 4; ++blk) {
+        valid |= ((1u << s_nv[4 * t + blk]) - 1u) << (4 * blk);
+        jlast = max(jlast, s_blk[4 * t + blk]);
+      }
+      // query q0 + qq sits at position L - Qn + q0 + qq and sees the tokens up
+      // to it; only a tile reaching past the group's first query needs masks
+      const int lim0 = L - a.Qn + a.q0;
+      unsigned vq[QN];
+      unsigned any = 0u;
+#pragma unroll
+      for (int qq = 0; qq < QN; ++qq) {
+        vq[qq] = valid;
+        if (4 * jlast + 3 > lim0) {
+          unsigned m = 0u;
+#pragma unroll
+          for (int row = 0; row < DV_TOK; ++row) {
+            const int j = s_blk[4 * t + (row >> 2)];
+            if (j >= 0 && 4 * j + (row & 3) <= lim0 + qq) m |= 1u << row;
+          }
+          vq[qq] = valid & m;
+        }
+        any |= vq[qq];
+      }
       const uint32_t kbuf = ring + (t % ST) * DV_STAGE;
-      if (valid) attend_tile(acc, kbuf, kbuf + DV_TOK * DV_ROWB, valid, qf, a.scale_log2, lane);
+      if (any) attend_tile<QN>(acc, kbuf, kbuf + DV_TOK * DV_ROWB, vq, qf, a.scale_log2, lane);
     }
     cp_async_wait<0>();
     pdl_trigger();
@@ -471,17 +529,19 @@ __global__ void __launch_bounds__(DV_WARPS * 32, DV_CTAS_PER_SM) sparse_decode_k
 __global__ void __launch_bounds__(DV_CB_ROWS * 32) decode_combine_kernel(DecodeArgs a) {
   pdl_wait();  // the records come from the decode kernel before this one
   const int b = blockIdx.z, r = blockIdx.y;
+  // row = (query qq of the group, head h)
   const int q = blockIdx.x * DV_CB_ROWS + (threadIdx.x >> 5), d4 = threadIdx.x & 31;
   const int2 sp = a.span[(size_t)b * a.R + r];
-  if (sp.y <= sp.x || q >= a.Hq) return;  // written by the decode kernel itself
+  if (sp.y <= sp.x || q >= a.qn * a.Hq) return;  // written by the decode kernel itself
   const int n = sp.y - sp.x + 1;
-  const size_t row0 = ((size_t)b * a.rb + sp.x + r) * a.Hq + q;  // record i at row0 + i*Hq
+  const size_t stride = (size_t)a.qn * a.Hq;                         // between records
+  const size_t row0 = ((size_t)b * a.rb + sp.x + r) * stride + q;    // record i at row0 + i*stride
   float M = -INFINITY;
   for (int i0 = 0; i0 < n; i0 += DV_CB_BATCH) {
     float l[DV_CB_BATCH];
 #pragma unroll
     for (int u = 0; u < DV_CB_BATCH; ++u)
-      l[u] = __ldcg(a.rec_lse + row0 + (size_t)min(i0 + u, n - 1) * a.Hq);
+      l[u] = __ldcg(a.rec_lse + row0 + (size_t)min(i0 + u, n - 1) * stride);
 #pragma unroll
     for (int u = 0; u < DV_CB_BATCH; ++u) M = fmaxf(M, l[u]);
   }
@@ -492,7 +552,7 @@ __global__ void __launch_bounds__(DV_CB_ROWS * 32) decode_combine_kernel(DecodeA
       float4 v[DV_CB_BATCH];
 #pragma unroll
       for (int u = 0; u < DV_CB_BATCH; ++u) {
-        const size_t rr = row0 + (size_t)min(i0 + u, n - 1) * a.Hq;
+        const size_t rr = row0 + (size_t)min(i0 + u, n - 1) * stride;
         l[u] = __ldcg(a.rec_lse + rr);
         v[u] = __ldcg(reinterpret_cast<const float4 *>(a.rec_o + rr * DV_D) + d4);
       }
@@ -507,7 +567,8 @@ __global__ void __launch_bounds__(DV_CB_ROWS * 32) decode_combine_kernel(DecodeA
       }
     }
   }
-  const size_t orow = ((size_t)r * a.B + b) * a.Hq + q;
+  const int qq = q / a.Hq, h = q % a.Hq;
+  const size_t orow = (((size_t)r * a.B + b) * a.Qn + a.q0 + qq) * a.Hq + h;
   const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
   reinterpret_cast<float4 *>(a.o_part + orow * DV_D)[d4] =
       make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
@@ -523,7 +584,8 @@ DecodePlan plan_decode(const qsa_dims &d, int B, int k, int R) {
   DecodePlan p;
   p.nhg = (d.Hkv + DV_WARPS - 1) / DV_WARPS;
   p.k_pad = (k + 3) & ~3;
-  const size_t extra = (size_t)p.k_pad * 4 + (size_t)DV_TBL_BLOCKS * 5;
+  // selection row; per block slot: pool row, block index, valid tokens
+  const size_t extra = (size_t)p.k_pad * 4 + (size_t)DV_TBL_BLOCKS * 9;
   const size_t static_smem = 1024;
   const size_t fit = (DV_SMEM_LIMIT - static_smem - extra) / ((size_t)DV_WARPS * DV_STAGE);
   p.stages = fit >= 4 ? 4 : (fit >= 3 ? 3 : 2);
@@ -541,26 +603,37 @@ DecodePlan plan_decode(const qsa_dims &d, int B, int k, int R) {
   return p;
 }
 
-template <int ST>
+template <int ST, int QN>
 cudaError_t launch_st(const DecodeArgs &a, const DecodePlan &p, int B, cudaStream_t st) {
   cudaError_t e =
-      ensure_dynamic_smem(reinterpret_cast<const void *>(sparse_decode_kernel<ST>), p.smem);
+      ensure_dynamic_smem(reinterpret_cast<const void *>(sparse_decode_kernel<ST, QN>), p.smem);
   if (e != cudaSuccess) return e;
-  e = launch_pdl(sparse_decode_kernel<ST>, dim3(p.ncb, p.nhg, B), DV_WARPS * 32, p.smem, st, a);
+  e = launch_pdl(sparse_decode_kernel<ST, QN>, dim3(p.ncb, p.nhg, B), DV_WARPS * 32, p.smem, st,
+                 a);
   if (e != cudaSuccess || p.ncb == 1) return e;  // one CTA per sequence: nothing to combine
-  return launch_pdl(decode_combine_kernel, dim3((a.Hq + DV_CB_ROWS - 1) / DV_CB_ROWS, a.R, B),
-                    DV_CB_ROWS * 32, 0, st, a);
+  return launch_pdl(decode_combine_kernel,
+                    dim3((QN * a.Hq + DV_CB_ROWS - 1) / DV_CB_ROWS, a.R, B), DV_CB_ROWS * 32, 0,
+                    st, a);
+}
+
+template <int QN>
+cudaError_t launch_qn(const DecodeArgs &a, const DecodePlan &p, int B, cudaStream_t st) {
+  switch (p.stages) {
+    case 4: return launch_st<4, QN>(a, p, B, st);
+    case 3: return launch_st<3, QN>(a, p, B, st);
+    default: return launch_st<2, QN>(a, p, B, st);
+  }
 }
 
 }  // namespace
 
-size_t decode_ws_bytes(const qsa_dims &d, int B, int k, int R) {
+size_t decode_ws_bytes(const qsa_dims &d, int B, int Qn, int k, int R) {
   const DecodePlan p = plan_decode(d, B, k, R);
-  const size_t rows = (size_t)B * p.rb * d.Hq;
+  const size_t rows = (size_t)B * p.rb * (Qn < DV_QGROUP ? Qn : DV_QGROUP) * d.Hq;
   return rows * (DV_D + 1) * sizeof(float) + (size_t)B * R * sizeof(int2);
 }
 
-cudaError_t launch_sparse_decode(const qsa_dims &d, const qsa_cache &c, int B,
+cudaError_t launch_sparse_decode(const qsa_dims &d, const qsa_cache &c, int B, int Qn,
                                  const int32_t *seq_lens, const void *q, const int32_t *sel,
                                  int k, int R, float *o_part, float *lse_part, void *ws,
                                  unsigned *err, cudaStream_t st) {
@@ -575,10 +648,6 @@ cudaError_t launch_sparse_decode(const qsa_dims &d, const qsa_cache &c, int B,
   a.sel = sel;
   a.o_part = o_part;
   a.lse_part = lse_part;
-  const size_t rows = (size_t)B * p.rb * d.Hq;
-  a.rec_o = static_cast<float *>(ws);
-  a.rec_lse = a.rec_o + rows * DV_D;
-  a.span = reinterpret_cast<int2 *>(a.rec_lse + rows);
   a.B = B;
   a.Hq = d.Hq;
   a.Hkv = d.Hkv;
@@ -591,14 +660,22 @@ cudaError_t launch_sparse_decode(const qsa_dims &d, const qsa_cache &c, int B,
   a.R = R;
   a.ncb = p.ncb;
   a.rb = p.rb;
+  a.Qn = Qn;
   a.ring_bytes = DV_WARPS * p.stages * DV_STAGE;
   a.scale_log2 = d.scale * LOG2E;
   a.err = err;
-  switch (p.stages) {
-    case 4: return launch_st<4>(a, p, B, st);
-    case 3: return launch_st<3>(a, p, B, st);
-    default: return launch_st<2>(a, p, B, st);
+  // query groups of up to DV_QGROUP, each one pass over the selected K/V
+  for (int q0 = 0; q0 < Qn; q0 += DV_QGROUP) {
+    a.q0 = q0;
+    a.qn = Qn - q0 < DV_QGROUP ? Qn - q0 : DV_QGROUP;
+    const size_t rows = (size_t)B * p.rb * a.qn * d.Hq;
+    a.rec_o = static_cast<float *>(ws);
+    a.rec_lse = a.rec_o + rows * DV_D;
+    a.span = reinterpret_cast<int2 *>(a.rec_lse + rows);
+    const cudaError_t e = a.qn == 2 ? launch_qn<2>(a, p, B, st) : launch_qn<1>(a, p, B, st);
+    if (e != cudaSuccess) return e;
   }
+  return cudaSuccess;
 }
 
 }  // namespace qsa

@@ -30,7 +30,8 @@ QSA_ERR_TIMEOUT = 5
 EXPORTS = ("qsa_version", "qsa_last_error", "qsa_append", "qsa_index_score",
            "qsa_topk_workspace_size", "qsa_topk_select", "qsa_sparse_decode_workspace_size",
            "qsa_sparse_decode", "qsa_sparse_decode_static", "qsa_merge",
-           "qsa_decode_step", "qsa_check_device_errors")
+           "qsa_decode_step", "qsa_sparse_decode_mq_workspace_size", "qsa_sparse_decode_mq",
+           "qsa_check_device_errors")
 
 
 class QsaError(RuntimeError):
@@ -76,6 +77,8 @@ def lib() -> ctypes.CDLL:
         "qsa_sparse_decode_workspace_size": (SZ, [DP, I32, I32, I32]),
         "qsa_sparse_decode": (I32, [DP, CP, I32, P, P, P, I32, I32, P, P, P, SZ, P]),
         "qsa_sparse_decode_static": (I32, [DP, CP, I32, P, P, P, I32, I32, P, P, P]),
+        "qsa_sparse_decode_mq_workspace_size": (SZ, [DP, I32, I32, I32, I32]),
+        "qsa_sparse_decode_mq": (I32, [DP, CP, I32, I32, P, P, P, I32, I32, P, P, P, SZ, P]),
         "qsa_merge": (I32, [I32, I32, I32, I32, P, P, P, I32, P, P]),
         "qsa_decode_step": (I32, [DP, CP, I32, P, P, P, P, P, I32, P, P, P, P, I32, I32, P, I32,
                                   P, P, P, P, SZ, P, I32, P, P]),
@@ -235,6 +238,23 @@ def qsa_sparse_decode(dims: QsaDims, cache: QsaCache, seq_lens, q, sel, k: int, 
                                    _ptr(lse_part, torch.float32, "lse_part"),
                                    _ptr(ws, None, "ws"), ws.numel() * ws.element_size(),
                                    _stream(stream)))
+
+
+def qsa_sparse_decode_mq_workspace_size(dims: QsaDims, B: int, Qn: int, k: int, R: int) -> int:
+    return int(lib().qsa_sparse_decode_mq_workspace_size(ctypes.byref(dims.c()), B, Qn, k, R))
+
+
+def qsa_sparse_decode_mq(dims: QsaDims, cache: QsaCache, seq_lens, q, sel, k: int, R: int,
+                         o_part, lse_part, ws, stream=None):
+    """Multi-query decode: q [B, Qn, Hq, D] -> o_part [R, B, Qn, Hq, D]."""
+    B, Qn = int(q.shape[0]), int(q.shape[1])
+    _check(lib().qsa_sparse_decode_mq(ctypes.byref(dims.c()), ctypes.byref(cache.c()), B, Qn,
+                                      _ptr(seq_lens, torch.int32, "seq_lens"),
+                                      _ptr(q, torch.bfloat16, "q"), _ptr(sel, torch.int32, "sel"),
+                                      int(k), int(R), _ptr(o_part, torch.float32, "o_part"),
+                                      _ptr(lse_part, torch.float32, "lse_part"),
+                                      _ptr(ws, None, "ws"), ws.numel() * ws.element_size(),
+                                      _stream(stream)))
 
 
 def qsa_sparse_decode_static(dims: QsaDims, cache: QsaCache, seq_lens, q, sel, k: int, R: int,

@@ -188,6 +188,30 @@ qsa_status qsa_sparse_decode(const qsa_dims *dims, const qsa_cache *cache,
                              int32_t R, float *o_part, float *lse_part,
                              void *ws, size_t ws_bytes, qsa_stream_t stream);
 
+/* Scratch bytes of qsa_sparse_decode_mq (Qn queries per sequence). */
+size_t qsa_sparse_decode_mq_workspace_size(const qsa_dims *dims, int32_t B,
+                                           int32_t Qn, int32_t k, int32_t R);
+
+/* Multi-query decode: Qn decode queries per sequence share the sequence's
+ * one selection and one gather of its K/V (several new tokens per step, as
+ * in multi-token prediction or speculative decoding). The page names such a
+ * workload (section "Why a serving PR ... is still worth your time") without
+ * defining it; this library's reading: the Qn new tokens are the last Qn
+ * positions of the sequence (already appended), and query j sits at position
+ * L_b - Qn + j and attends to the selected tokens t <= L_b - Qn + j.
+ *   q         bf16 [B, Qn, Hq, D]
+ *   o_part    fp32 [R, B, Qn, Hq, D];  lse_part  fp32 [R, B, Qn, Hq]
+ * Slices, selection and empty-slice rule as in qsa_sparse_decode (a slice
+ * whose selected tokens all lie after a query is empty for that query);
+ * qsa_merge combines the result with B * Qn rows. Queries are processed in
+ * groups of two per pass over the selected K/V. Supported: 1 <= Qn <= 8;
+ * qsa_sparse_decode is this call with Qn = 1. */
+qsa_status qsa_sparse_decode_mq(const qsa_dims *dims, const qsa_cache *cache,
+                                int32_t B, int32_t Qn, const int32_t *seq_lens,
+                                const void *q, const int32_t *sel, int32_t k,
+                                int32_t R, float *o_part, float *lse_part,
+                                void *ws, size_t ws_bytes, qsa_stream_t stream);
+
 /* Size of the static device scratch of qsa_sparse_decode_static (32 MiB). */
 #define QSA_STATIC_SCRATCH_BYTES (32u << 20)
 

@@ -393,3 +393,41 @@ def test_steady128x64k_append_steps():
     for b in range(wl.B):
         _, _, X = wl.seq_tokens(b, L)
         assert np.array_equal(run.side_rows(b, L), oracle.side_cache(bits(X), L)), b
+
+
+# ------------------------------------------------------------ multi-query decode
+
+@pytest.mark.parametrize("Qn,R", [(1, 4), (2, 1), (2, 4), (3, 8), (5, 2)])
+def test_multi_query_decode_matches_oracle(Qn, R):
+    # the Qn queries are the sequence's last Qn positions (all appended); each
+    # sees the shared selection's tokens up to its own position. Lengths below
+    # Qn leave the first queries with nothing to see (zeros, LSE = -inf).
+    lens = [9001, 2050, 3, 40003, 1026, 13]
+    wl = make_custom(DIMS_FULL, lens, k=256, R=R, seed=300 + 10 * Qn + R, device=DEV)
+    run = GpuRun(wl)
+    run.step()  # cache complete, selection of every sequence in run.buf.sel
+    d = run.dims
+    g = torch.Generator(device=DEV).manual_seed(Qn)
+    q = torch.randn((wl.B, Qn, d.Hq, d.D), generator=g, device=DEV).to(torch.bfloat16)
+    o = torch.full((R, wl.B, Qn, d.Hq, d.D), float("nan"), device=DEV)
+    lse = torch.full((R, wl.B, Qn, d.Hq), float("nan"), device=DEV)
+    ws = torch.empty(max(16, qsa.qsa_sparse_decode_mq_workspace_size(d, wl.B, Qn, wl.k, R)),
+                     dtype=torch.uint8, device=DEV)
+    qsa.qsa_sparse_decode_mq(d, run.cache, run.seq_lens, q, run.buf.sel, wl.k, R, o, lse, ws)
+    out = torch.empty((wl.B * Qn, d.Hq, d.D), dtype=torch.float32, device=DEV)
+    lse_m = torch.empty((wl.B * Qn, d.Hq), dtype=torch.float32, device=DEV)
+    qsa.qsa_merge(o.view(R, wl.B * Qn, d.Hq, d.D), lse.view(R, wl.B * Qn, d.Hq), out, lse_m)
+    assert qsa.qsa_check_device_errors() == 0
+    o_np, l_np = o.cpu().numpy(), lse.cpu().numpy()
+    om_np, lm_np = out.view(wl.B, Qn, d.Hq, d.D).cpu().numpy(), lse_m.view(wl.B, Qn, d.Hq).cpu().numpy()
+    for b, L in enumerate(lens):
+        K, V, _ = wl.seq_tokens(b)
+        sel = run.buf.sel[b].cpu().numpy()
+        O_ref, L_ref = oracle.attend_slices_mq(bits(q[b]), bits(K), bits(V), sel, L,
+                                               wl.dims.scale, R)
+        for j in range(Qn):
+            check_attention(o_np[:, b, j], l_np[:, b, j], O_ref[:, j], L_ref[:, j],
+                            what=f"Qn={Qn} R={R} b={b} query {j}")
+            Om, Lm = oracle.merge_partials(O_ref[:, j], L_ref[:, j])
+            check_attention(om_np[b, j], lm_np[b, j], Om, Lm,
+                            what=f"merged Qn={Qn} R={R} b={b} query {j}")
