@@ -452,18 +452,37 @@ def _oracle_one(sample, dims, k, R):
                                   k, R, dims.scale)
 
 
-def cpu_baseline(sample, dims, k, R, budget_s=12.0):
-    """The oracle, as it stands, on whole sequences of the same workload."""
+def _oracle_rate(sample, dims, k, R, budget_s):
     n, t0 = 0, time.perf_counter()
     while True:
         _oracle_one(sample, dims, k, R)
         n += 1
         el = time.perf_counter() - t0
         if el >= budget_s or n >= 20:
-            break
-    return {"value": n / el, "unit": "seqs/s", "cores": _threads(), "kind": "oracle",
-            "sample": f"{n} full decode(s) of one {sample['L']}-token sequence of the same "
-                      f"workload (score, top-{k}, R={R} attention, merge), numpy fp64"}
+            return n, n / el
+
+
+def cpu_baseline(sample, dims, k, R, budget_s=12.0, single_budget_s=8.0):
+    """The oracle, as it stands, on whole sequences of the same workload: with
+    the BLAS threads numpy brings (all host cores), and on one thread."""
+    n, rate = _oracle_rate(sample, dims, k, R, budget_s)
+    res = {"value": rate, "unit": "seqs/s", "cores": _threads(), "kind": "oracle",
+           "sample": f"{n} full decode(s) of one {sample['L']}-token sequence of the same "
+                     f"workload (score, top-{k}, R={R} attention, merge), numpy fp64"}
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            n1, rate1 = _oracle_rate(sample, dims, k, R, single_budget_s)
+        res["single_thread"] = {"value": rate1, "unit": "seqs/s", "cores": 1,
+                                "sample": f"{n1} full decode(s), BLAS limited to one thread"}
+    except Exception as e:  # threadpoolctl missing: report the multi-thread figure only
+        res["single_thread"] = {"unavailable": str(e)[:120]}
+    try:
+        res["cpu_model"] = open("/proc/cpuinfo").read().split("model name")[1].split(
+            "\n")[0].strip(" :\t")
+    except Exception:
+        pass
+    return res
 
 
 # ------------------------------------------------------------ reference arm
