@@ -191,6 +191,15 @@ def attend_slices_mq(q_bits, k_bits, v_bits, sel, L: int, scale: float, R: int):
     return (np.stack([o for o, _ in parts], axis=1), np.stack([l for _, l in parts], axis=1))
 
 
+def owned_blocks(sel, P: int, W: int, r: int) -> np.ndarray:
+    """Decode context parallelism over W ranks: the selected blocks whose page
+    (block j lies on page 4j // P of its sequence) belongs to rank r, page p
+    belonging to rank p mod W. Same order as `sel`, -1 padded to len(sel)."""
+    sel = np.asarray(sel)
+    own = [int(j) for j in sel if j >= 0 and ((4 * int(j)) // P) % W == r]
+    return np.array(own + [-1] * (len(sel) - len(own)), dtype=np.int64)
+
+
 def merge_partials(O, LSE):
     """LSE-weighted combine of R partials: O [R, H, D], LSE [R, H] -> O [H, D], LSE [H].
     Slices with LSE = -inf contribute nothing."""

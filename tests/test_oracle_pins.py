@@ -448,3 +448,37 @@ def test_multi_query_split_merge_equals_unsplit_and_hides_future_blocks():
     Lq, Kq = 201, K[:201]
     O0, L0 = oracle.attend_slices(bits(q[0]), bits(Kq), bits(V[:201]), np.array([50]), Lq, 0.2, 1)
     assert np.abs(O[nb - 1, 0] - O0[0]).max() <= 1e-12   # query 0 = single query over t < 201
+
+
+# ------------------------------------------------------------ context parallel
+
+@pytest.mark.parametrize("W,P", [(2, 64), (4, 64), (3, 32), (8, 16)])
+def test_owned_blocks_partition_the_selection(W, P):
+    g = np.random.default_rng(W * 100 + P)
+    sel = np.sort(g.choice(5000, size=300, replace=False))
+    sel = np.concatenate([sel, -np.ones(20, dtype=np.int64)])
+    parts = [oracle.owned_blocks(sel, P, W, r) for r in range(W)]
+    got = np.sort(np.concatenate([p[p >= 0] for p in parts]))
+    assert np.array_equal(got, sel[sel >= 0])          # every block on exactly one rank
+    for r, p in enumerate(parts):
+        live = p[p >= 0]
+        assert np.all(np.diff(live) > 0) and np.all(p[len(live):] == -1)
+        assert np.all(((4 * live) // P) % W == r)      # by its page
+
+
+def test_context_parallel_merge_equals_single_rank_attention():
+    # each rank attends over its own pages' share of the one selection; the
+    # LSE-weighted merge of the W partials is the attention over all of it
+    d = Dims(Hq=8, Hkv=2, D=32, Hi=4, di=32, P=16, scale=0.2)
+    wl = make_custom(d, [1501], k=64, R=1, seed=21, paged=False)
+    K, V, X = wl.seq_tokens(0)
+    args = (bits(wl.q[0]), bits(K), bits(V))
+    sel = oracle.topk_blocks(oracle.index_scores(oracle.block_keys(bits(X), 1501),
+                                                 bits(wl.q_idx[0]), wl.w[0].numpy()), 64)
+    O1, L1 = oracle.attend_slices(*args, sel, 1501, d.scale, 1)
+    for W in (2, 3, 4):
+        parts = [oracle.attend_slices(*args, oracle.owned_blocks(sel, d.P, W, r), 1501,
+                                      d.scale, 1) for r in range(W)]
+        Om, Lm = oracle.merge_partials(np.stack([o[0] for o, _ in parts]),
+                                       np.stack([l[0] for _, l in parts]))
+        assert np.abs(Om - O1[0]).max() <= 1e-12 and np.abs(Lm - L1[0]).max() <= 1e-12
