@@ -297,6 +297,25 @@ qsa_status qsa_sparse_decode_mq(const qsa_dims *dims, const qsa_cache *cache, in
   }
 }
 
+qsa_status qsa_select_owned(int32_t B, const int32_t *sel, int32_t k, int32_t P, int32_t W,
+                            int32_t r, int32_t *sel_out, qsa_stream_t stream) {
+  try {
+    if (B < 0 || B > 65535) return fail(QSA_ERR_INVALID_ARG, "B=%d outside [0, 65535]", B);
+    if (k < 1 || k > 4096) return fail(QSA_ERR_UNSUPPORTED, "k=%d outside [1, 4096]", k);
+    if (P <= 0 || P % 4 != 0) return fail(QSA_ERR_INVALID_ARG, "P=%d not a positive multiple of 4", P);
+    if (W < 1 || W > 1024 || r < 0 || r >= W)
+      return fail(QSA_ERR_INVALID_ARG, "rank %d of %d outside the supported range", r, W);
+    if (B > 0 && (sel == nullptr || sel_out == nullptr))
+      return fail(QSA_ERR_INVALID_ARG, "an argument array is NULL");
+    if (B > 0 && sel == sel_out) return fail(QSA_ERR_INVALID_ARG, "sel_out must not alias sel");
+    return cuda_status(launch_select_owned(sel, B, k, P, W, r, sel_out,
+                                           reinterpret_cast<cudaStream_t>(stream)),
+                       "qsa_select_owned launch");
+  } catch (...) {
+    return fail(QSA_ERR_CUDA, "qsa_select_owned: internal exception");
+  }
+}
+
 qsa_status qsa_merge(int32_t R, int32_t B, int32_t Hq, int32_t D, const float *o_part,
                      const float *lse_part, void *out, int32_t out_is_bf16, float *lse_out,
                      qsa_stream_t stream) {

@@ -58,6 +58,9 @@ cudaError_t launch_sparse_decode(const qsa_dims &d, const qsa_cache &c, int B, i
                                  int k, int R, float *o_part, float *lse_part, void *ws,
                                  unsigned *err, cudaStream_t st);
 
+cudaError_t launch_select_owned(const int32_t *sel, int B, int k, int P, int W, int r,
+                                int32_t *out, cudaStream_t st);
+
 cudaError_t launch_merge(int R, int B, int Hq, int D, const float *o_part, const float *lse_part,
                          void *out, int out_is_bf16, float *lse_out, cudaStream_t st);
 

@@ -291,7 +291,18 @@ __global__ void __launch_bounds__(DV_WARPS * 32, DV_CTAS_PER_SM) sparse_decode_k
   // its tiles are [pre[r], pre[r+1]) of the sequence's NT = pre[R] tiles
   const int L = s_L;
   const int nb = L <= 0 ? 0 : (L + 3) >> 2;
-  const int kb = min(a.k, nb);
+  int kb = min(a.k, nb);
+  {
+    // the list ends at its first -1 (a selection may hold fewer than
+    // min(k, nb) blocks, e.g. one rank's share): valid ids come first, so the
+    // predicate "entry < 0" is monotone over the row
+    int lo = 0, hi = kb;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (s_sel[mid] < 0) hi = mid; else lo = mid + 1;
+    }
+    kb = lo;
+  }
   if (warp == 0) {
     int st[2], ct[2], nt[2];
 #pragma unroll

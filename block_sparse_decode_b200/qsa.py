@@ -31,7 +31,7 @@ EXPORTS = ("qsa_version", "qsa_last_error", "qsa_append", "qsa_index_score",
            "qsa_topk_workspace_size", "qsa_topk_select", "qsa_sparse_decode_workspace_size",
            "qsa_sparse_decode", "qsa_sparse_decode_static", "qsa_merge",
            "qsa_decode_step", "qsa_sparse_decode_mq_workspace_size", "qsa_sparse_decode_mq",
-           "qsa_check_device_errors")
+           "qsa_select_owned", "qsa_check_device_errors")
 
 
 class QsaError(RuntimeError):
@@ -79,6 +79,7 @@ def lib() -> ctypes.CDLL:
         "qsa_sparse_decode_static": (I32, [DP, CP, I32, P, P, P, I32, I32, P, P, P]),
         "qsa_sparse_decode_mq_workspace_size": (SZ, [DP, I32, I32, I32, I32]),
         "qsa_sparse_decode_mq": (I32, [DP, CP, I32, I32, P, P, P, I32, I32, P, P, P, SZ, P]),
+        "qsa_select_owned": (I32, [I32, P, I32, I32, I32, I32, P, P]),
         "qsa_merge": (I32, [I32, I32, I32, I32, P, P, P, I32, P, P]),
         "qsa_decode_step": (I32, [DP, CP, I32, P, P, P, P, P, I32, P, P, P, P, I32, I32, P, I32,
                                   P, P, P, P, SZ, P, I32, P, P]),
@@ -269,6 +270,15 @@ def qsa_sparse_decode_static(dims: QsaDims, cache: QsaCache, seq_lens, q, sel, k
                                           _ptr(o_part, torch.float32, "o_part"),
                                           _ptr(lse_part, torch.float32, "lse_part"),
                                           _stream(stream)))
+
+
+def qsa_select_owned(sel, P: int, world: int, rank: int, sel_out, stream=None):
+    """The selected blocks whose page rank ``rank`` of ``world`` holds (page p
+    on rank p mod world), same order, -1 padded."""
+    B, k = (int(x) for x in sel.shape)
+    _check(lib().qsa_select_owned(B, _ptr(sel, torch.int32, "sel"), k, int(P), int(world),
+                                  int(rank), _ptr(sel_out, torch.int32, "sel_out"),
+                                  _stream(stream)))
 
 
 def qsa_merge(o_part, lse_part, out, lse_out=None, stream=None):

@@ -177,7 +177,9 @@ size_t qsa_sparse_decode_workspace_size(const qsa_dims *dims, int32_t B,
  * the selector replicated, results combined afterwards).
  *   q         bf16 [B, Hq, D]
  *   sel       int32 [B, k] as produced by qsa_topk_select (ascending, -1
- *             padded); the same selection serves all R slices
+ *             padded); the same selection serves all R slices. The list ends
+ *             at its first -1 or after min(k, nb_b) entries, so a shorter
+ *             selection (e.g. qsa_select_owned's) is accepted
  *   o_part    fp32 [R, B, Hq, D];  lse_part  fp32 [R, B, Hq]
  * Slice r holds the attention of each query head over the tokens t < L_b of
  * the selected blocks in [floor(r*nb/R), floor((r+1)*nb/R)); an empty slice
@@ -237,6 +239,21 @@ qsa_status qsa_sparse_decode_static(const qsa_dims *dims, const qsa_cache *cache
                                     const void *q, const int32_t *sel, int32_t k,
                                     int32_t R, float *o_part, float *lse_part,
                                     qsa_stream_t stream);
+
+/* Decode context parallelism (page section "What the pull request actually
+ * changes": each rank reads only its slice of the main KV cache, the
+ * selector stays replicated; "Questions worth answering directly": partial
+ * attention results are merged afterwards). This library's reading of a
+ * rank's slice: page p of every sequence is held by rank p mod W (balanced,
+ * and stable as sequences grow). Every rank scores and selects on the
+ * replicated side cache, keeps with this call the selected blocks of the
+ * pages it holds (sel_out [B, k], same order, -1 padded; block j lies on page
+ * 4j / P), attends over them with qsa_sparse_decode, gathers the W partials
+ * from the other ranks and combines them with qsa_merge (R = W).
+ * Supported: 1 <= W <= 1024, 0 <= r < W, P a positive multiple of 4. */
+qsa_status qsa_select_owned(int32_t B, const int32_t *sel, int32_t k, int32_t P,
+                            int32_t W, int32_t r, int32_t *sel_out,
+                            qsa_stream_t stream);
 
 /* LSE-weighted combine of R partial results (page sections "What the pull
  * request actually changes", second bullet, and "Questions worth answering

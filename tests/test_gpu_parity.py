@@ -431,3 +431,48 @@ def test_multi_query_decode_matches_oracle(Qn, R):
             Om, Lm = oracle.merge_partials(O_ref[:, j], L_ref[:, j])
             check_attention(om_np[b, j], lm_np[b, j], Om, Lm,
                             what=f"merged Qn={Qn} R={R} b={b} query {j}")
+
+
+# ------------------------------------------------------------ context parallel
+
+@pytest.mark.parametrize("W", [2, 4])
+def test_context_parallel_ranks_merge_to_full_attention(W):
+    # one process emulates W ranks: rank r maps only the pages p = r mod W of
+    # every sequence (the others -1), filters the shared selection to them,
+    # decodes one slice over its own pages; the merge of the W partials is the
+    # attention over the whole selection
+    lens = [30001, 5000, 77, 12345, 2048]
+    wl = make_custom(DIMS_FULL, lens, k=512, R=1, seed=400 + W, device=DEV)
+    run = GpuRun(wl)
+    run.step()
+    d, B = run.dims, wl.B
+    sel = run.buf.sel
+    cols = torch.arange(run.cache.block_table.shape[1], device=DEV)
+    O, L = [], []
+    for r in range(W):
+        bt = run.cache.block_table.clone()
+        bt[:, (cols % W) != r] = -1
+        cache_r = qsa.QsaCache(run.cache.k_pool, run.cache.v_pool, run.cache.kidx_pool,
+                               run.cache.side_pool, bt)
+        sel_r = torch.full_like(sel, -7)
+        qsa.qsa_select_owned(sel, d.P, W, r, sel_r)
+        for b in range(B):
+            assert np.array_equal(sel_r[b].cpu().numpy(),
+                                  oracle.owned_blocks(sel[b].cpu().numpy(), d.P, W, r)), (r, b)
+        o_r = torch.empty((1, B, d.Hq, d.D), dtype=torch.float32, device=DEV)
+        l_r = torch.empty((1, B, d.Hq), dtype=torch.float32, device=DEV)
+        ws = torch.empty(max(16, qsa.qsa_sparse_decode_workspace_size(d, B, wl.k, 1)),
+                         dtype=torch.uint8, device=DEV)
+        qsa.qsa_sparse_decode(d, cache_r, run.seq_lens, wl.q, sel_r, wl.k, 1, o_r, l_r, ws)
+        assert qsa.qsa_check_device_errors() == 0  # no page outside the rank's share was read
+        O.append(o_r[0])
+        L.append(l_r[0])
+    out = torch.empty((B, d.Hq, d.D), dtype=torch.float32, device=DEV)
+    lse = torch.empty((B, d.Hq), dtype=torch.float32, device=DEV)
+    qsa.qsa_merge(torch.stack(O), torch.stack(L), out, lse)
+    for b, Lb in enumerate(lens):
+        K, V, _ = wl.seq_tokens(b)
+        ref_o, ref_l = oracle.attend_slices(bits(wl.q[b]), bits(K), bits(V),
+                                            sel[b].cpu().numpy(), Lb, wl.dims.scale, 1)
+        check_attention(out[b].cpu().numpy(), lse[b].cpu().numpy(), ref_o[0], ref_l[0],
+                        what=f"DCP W={W} b={b}")

@@ -63,6 +63,64 @@ def test_two_gloo_ranks_take_the_max_and_draw_distinct_batches():
         assert len(set(seeds)) == world  # each replica its own batch
 
 
+def _dcp_worker(rank, world, port, out_q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=__import__("datetime").timedelta(seconds=60))
+    try:
+        import numpy as np
+        import oracle
+        from block_sparse_decode_b200 import dcp
+        from synth import make_custom
+        from synth.workloads import Dims
+        from tests.helpers import bits
+        d = Dims(Hq=8, Hkv=2, D=32, Hi=4, di=32, P=16, scale=0.2)
+        wl = make_custom(d, [2001, 517], k=48, R=1, seed=77, paged=False)
+        O_r, L_r, full = [], [], []
+        for b, L in enumerate(wl.seq_lens):
+            K, V, X = wl.seq_tokens(b)
+            sel = oracle.topk_blocks(oracle.index_scores(oracle.block_keys(bits(X), L),
+                                                         bits(wl.q_idx[b]), wl.w[b].numpy()), 48)
+            args = (bits(wl.q[b]), bits(K), bits(V))
+            o, l = oracle.attend_slices(*args, oracle.owned_blocks(sel, d.P, world, rank), L,
+                                        d.scale, 1)
+            O_r.append(o[0])
+            L_r.append(l[0])
+            full.append(oracle.attend_slices(*args, sel, L, d.scale, 1))
+        # the product's exchange step, on CPU tensors over gloo
+        O, Ls = dcp.exchange_partials(torch.from_numpy(np.stack(O_r)),
+                                      torch.from_numpy(np.stack(L_r)))
+        worst = 0.0
+        for b in range(len(wl.seq_lens)):
+            Om, Lm = oracle.merge_partials(O[:, b].numpy(), Ls[:, b].numpy())
+            worst = max(worst, float(np.abs(Om - full[b][0][0]).max()),
+                        float(np.abs(Lm - full[b][1][0]).max()))
+        out_q.put((rank, tuple(O.shape), worst))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_context_parallel_exchange_over_two_gloo_ranks():
+    # each rank holds the partial over its own pages' share of the selection;
+    # the gathered, merged partials equal the attention over the whole
+    # selection on every rank
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_dcp_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    results = [q.get(timeout=180) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, shape, worst in results:
+        assert shape == (world, 2, 8, 32)
+        assert worst <= 1e-12, (rank, worst)
+
+
 def test_single_process_max_is_identity():
     assert not dist.is_initialized()
     assert bench.max_over_ranks(3.25, torch.device("cpu")) == 3.25
