@@ -54,6 +54,9 @@ def parse():
     ap.add_argument("--R", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--dcp-world", type=int, default=0,
+                    help="also time, on this GPU, rank 0's share of a decode-context-parallel "
+                         "step over this many ranks (page p on rank p mod W)")
     ap.add_argument("--queries", type=int, default=1,
                     help="decode queries per sequence (multi-query decode: each step appends "
                          "this many tokens per sequence and decodes all of them)")
@@ -321,6 +324,40 @@ def run_ours(args, rank, world, local_rank):
         kern_ms[n] = statistics.mean(timed(g) for _ in range(args.steps))
     qsa.qsa_check_device_errors()
 
+    # decode context parallelism, emulated on one GPU: rank 0 maps only its
+    # pages (p = 0 mod W), filters the selection to them and decodes one slice
+    dcp_res = None
+    if args.dcp_world > 1 and Qn == 1:
+        Wd = args.dcp_world
+        bt0 = cache.block_table.clone()
+        cols = torch.arange(bt0.shape[1], device=dev)
+        bt0[:, (cols % Wd) != 0] = -1
+        cache0 = qsa.QsaCache(cache.k_pool, cache.v_pool, cache.kidx_pool, cache.side_pool, bt0)
+        sel0 = torch.empty_like(buf.sel)
+        o0 = torch.empty((1, B, dims.Hq, dims.D), dtype=torch.float32, device=dev)
+        l0 = torch.empty((1, B, dims.Hq), dtype=torch.float32, device=dev)
+        ws0 = torch.empty(max(16, qsa.qsa_sparse_decode_workspace_size(dims, B, k, 1)),
+                          dtype=torch.uint8, device=dev)
+
+        def rank0():
+            qsa.qsa_select_owned(buf.sel, dims.P, Wd, 0, sel0)
+            qsa.qsa_sparse_decode(dims, cache0, si["seq_lens"], si["q"], sel0, k, 1, o0, l0, ws0)
+
+        g0 = capture(rank0)
+        for _ in range(3):
+            timed(g0)
+        r0_ms = statistics.mean(timed(g0) for _ in range(args.steps))
+        qsa.qsa_check_device_errors()
+        kept = int((sel0 >= 0).sum())
+        dcp_res = {"world": Wd, "rank0_select_and_decode_us": 1e3 * r0_ms,
+                   "rank0_selected_blocks": kept,
+                   "rank0_kv_bytes": kept * 4 * dims.Hkv * dims.D * 2 * 2,
+                   "exchange_bytes_per_rank": B * dims.Hq * (dims.D + 1) * 4,
+                   "note": "one GPU: rank 0's filter + one-slice decode over its pages, in a "
+                           "graph after an L2 flush; the all-gather and the merge of W "
+                           "partials are not timed here"}
+        g0.reset()
+
     # e2e: host buffers in pinned memory, copies inside the timed region,
     # calls made eagerly through the binding (the user's API)
     e2e = None
@@ -426,6 +463,8 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clk.summary(),
         "e2e": e2e,
     }
+    if dcp_res is not None:
+        res["dcp_emulated"] = dcp_res
     graph.reset()
     for g in kgraphs.values():
         g.reset()
