@@ -57,7 +57,7 @@ constexpr int DV_CTAS_PER_SM = 2;
 constexpr int DV_SLOTS = DV_CTAS_PER_SM * 148;  // CTAs in flight on a B200
 constexpr size_t DV_SMEM_LIMIT = 113 * 1024;    // shared memory per CTA so that two fit an SM
 constexpr int DV_CB_ROWS = 8;                   // query-head rows per combine CTA
-constexpr int DV_CB_BATCH = 8;                  // records loaded together by the combine
+constexpr int DV_CB_BATCH = 16;                 // records' outputs loaded together (combine)
 constexpr int DV_QGROUP = 2;                    // queries of a sequence per pass over K/V
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
@@ -533,57 +533,63 @@ __global__ void __launch_bounds__(DV_WARPS * 32, DV_CTAS_PER_SM) sparse_decode_k
   }
 }
 
-// (6) One CTA per (group of DV_CB_ROWS query heads, slice, sequence); thread
-// (row, d4) combines dims 4*d4..4*d4+3 of one query head over the records of
-// the slice's contributors: first the max of their LSEs, then the weighted
-// sum, DV_CB_BATCH records' loads in flight at a time.
+// (6) One CTA per (group of DV_CB_ROWS query rows, slice, sequence); warp =
+// one (query, head) row, lane l owns dims 4l..4l+3. Lane i holds the weight
+// of record i of each group of 32 (its LSE loaded in one round trip per 32
+// records, the max taken across the warp); the outputs are then read
+// DV_CB_BATCH records at a time, their weights broadcast from the lanes.
 __global__ void __launch_bounds__(DV_CB_ROWS * 32) decode_combine_kernel(DecodeArgs a) {
   pdl_wait();  // the records come from the decode kernel before this one
   const int b = blockIdx.z, r = blockIdx.y;
   // row = (query qq of the group, head h)
-  const int q = blockIdx.x * DV_CB_ROWS + (threadIdx.x >> 5), d4 = threadIdx.x & 31;
+  const int q = blockIdx.x * DV_CB_ROWS + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   const int2 sp = a.span[(size_t)b * a.R + r];
   if (sp.y <= sp.x || q >= a.qn * a.Hq) return;  // written by the decode kernel itself
   const int n = sp.y - sp.x + 1;
   const size_t stride = (size_t)a.qn * a.Hq;                         // between records
   const size_t row0 = ((size_t)b * a.rb + sp.x + r) * stride + q;    // record i at row0 + i*stride
   float M = -INFINITY;
-  for (int i0 = 0; i0 < n; i0 += DV_CB_BATCH) {
-    float l[DV_CB_BATCH];
-#pragma unroll
-    for (int u = 0; u < DV_CB_BATCH; ++u)
-      l[u] = __ldcg(a.rec_lse + row0 + (size_t)min(i0 + u, n - 1) * stride);
-#pragma unroll
-    for (int u = 0; u < DV_CB_BATCH; ++u) M = fmaxf(M, l[u]);
+  for (int i0 = 0; i0 < n; i0 += 32) {
+    const float l = i0 + lane < n ? __ldcg(a.rec_lse + row0 + (size_t)(i0 + lane) * stride)
+                                  : -INFINITY;
+    M = fmaxf(M, l);
   }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   float acc[4] = {0.f, 0.f, 0.f, 0.f}, wsum = 0.f;
   if (M != -INFINITY) {
-    for (int i0 = 0; i0 < n; i0 += DV_CB_BATCH) {
-      float l[DV_CB_BATCH];
-      float4 v[DV_CB_BATCH];
+    for (int i0 = 0; i0 < n; i0 += 32) {
+      const float l = i0 + lane < n ? __ldcg(a.rec_lse + row0 + (size_t)(i0 + lane) * stride)
+                                    : -INFINITY;
+      const float wl = l == -INFINITY ? 0.f : __expf(l - M);  // weight of record i0 + lane
+      const int m = min(32, n - i0);
+      for (int u0 = 0; u0 < m; u0 += DV_CB_BATCH) {
+        float4 v[DV_CB_BATCH];
 #pragma unroll
-      for (int u = 0; u < DV_CB_BATCH; ++u) {
-        const size_t rr = row0 + (size_t)min(i0 + u, n - 1) * stride;
-        l[u] = __ldcg(a.rec_lse + rr);
-        v[u] = __ldcg(reinterpret_cast<const float4 *>(a.rec_o + rr * DV_D) + d4);
-      }
+        for (int u = 0; u < DV_CB_BATCH; ++u) {
+          const size_t rr = row0 + (size_t)(i0 + min(u0 + u, m - 1)) * stride;
+          v[u] = __ldcg(reinterpret_cast<const float4 *>(a.rec_o + rr * DV_D) + lane);
+        }
 #pragma unroll
-      for (int u = 0; u < DV_CB_BATCH; ++u) {
-        const float w = i0 + u < n ? __expf(l[u] - M) : 0.f;
-        wsum += w;
-        acc[0] += w * v[u].x;
-        acc[1] += w * v[u].y;
-        acc[2] += w * v[u].z;
-        acc[3] += w * v[u].w;
+        for (int u = 0; u < DV_CB_BATCH; ++u) {
+          const float w = __shfl_sync(0xffffffffu, wl, (u0 + u) & 31);
+          if (u0 + u < m && w != 0.f) {  // a record of a query that saw nothing holds zeros
+            wsum += w;
+            acc[0] += w * v[u].x;
+            acc[1] += w * v[u].y;
+            acc[2] += w * v[u].z;
+            acc[3] += w * v[u].w;
+          }
+        }
       }
     }
   }
   const int qq = q / a.Hq, h = q % a.Hq;
   const size_t orow = (((size_t)r * a.B + b) * a.Qn + a.q0 + qq) * a.Hq + h;
   const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-  reinterpret_cast<float4 *>(a.o_part + orow * DV_D)[d4] =
+  reinterpret_cast<float4 *>(a.o_part + orow * DV_D)[lane] =
       make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
-  if (d4 == 0) a.lse_part[orow] = wsum > 0.f ? M + logf(wsum) : -INFINITY;
+  if (lane == 0) a.lse_part[orow] = wsum > 0.f ? M + logf(wsum) : -INFINITY;
 }
 
 struct DecodePlan {
