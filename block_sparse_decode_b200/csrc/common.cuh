@@ -29,7 +29,9 @@ __device__ __forceinline__ void raise_err(unsigned *err, unsigned bit) {
 // finishes, but every CTA executes pdl_wait() before it touches anything an
 // earlier kernel wrote (and before it exits), so the completion of a grid
 // still implies the completion of all work before it. pdl_trigger() lets the
-// next kernel start launching; CTAs call it once their main work is done.
+// next kernel start launching (its CTAs then wait in pdl_wait for this whole
+// grid). A kernel whose CTAs occupy the SMs calls it only once its main work
+// is done: dependents placed on the SMs of early finishers slowed the step.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() {
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");

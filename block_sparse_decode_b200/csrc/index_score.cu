@@ -265,6 +265,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   int *prefix = reinterpret_cast<int *>(smem_raw + pad + (size_t)S * STAGE + TBL * 4);
   int *lens = prefix + (a.B + 1);
 
+  // the CTAs pull the block-table rows of the batch into L2 together, so the
+  // page-table fill below (which first needs the tile prefix) hits L2
+  {
+    const char *bt = reinterpret_cast<const char *>(a.block_table);
+    const long long lines = ((long long)a.B * a.max_pages * 4 + 127) >> 7;
+    for (long long i = blockIdx.x + (long long)gridDim.x * threadIdx.x; i < lines;
+         i += (long long)gridDim.x * blockDim.x)
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(bt + (i << 7)));
+  }
+
   // ---- per-CTA tile prefix over sequences
   __shared__ int carry;
   __shared__ int wsum[TC_THREADS / 32];

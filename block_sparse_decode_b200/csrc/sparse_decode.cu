@@ -540,6 +540,7 @@ __global__ void __launch_bounds__(DV_WARPS * 32, DV_CTAS_PER_SM) sparse_decode_k
 // DV_CB_BATCH records at a time, their weights broadcast from the lanes.
 __global__ void __launch_bounds__(DV_CB_ROWS * 32) decode_combine_kernel(DecodeArgs a) {
   pdl_wait();  // the records come from the decode kernel before this one
+  pdl_trigger();  // the merge kernel waits for this whole grid
   const int b = blockIdx.z, r = blockIdx.y;
   // row = (query qq of the group, head h)
   const int q = blockIdx.x * DV_CB_ROWS + (threadIdx.x >> 5), lane = threadIdx.x & 31;
