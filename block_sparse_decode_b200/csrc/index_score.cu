@@ -49,6 +49,7 @@
 
 #include "common.cuh"
 #include "launch.h"
+#include "tc_util.cuh"
 #include "umma_desc.h"
 
 namespace qsa {
@@ -61,8 +62,6 @@ constexpr int TC_PROD_WARPS = 3;                          // producers take tile
 constexpr int TC_MMA_WARP = TC_PROD_WARPS;                // warp 3
 constexpr int TC_EPI0 = TC_PROD_WARPS + 1;                // first epilogue warp
 constexpr int TC_THREADS = 32 * (TC_PROD_WARPS + 1 + TC_EPI_WARPS);
-constexpr uint32_t TC_SPIN_LIMIT = 1u << 22;  // try_wait rounds before giving up
-constexpr uint32_t TC_DRAIN_LIMIT = 1u << 20;
 constexpr int TBL = 4096;  // shared page-table entries (two halves)
 __device__ const int32_t k_no_page = -1;
 
@@ -92,95 +91,6 @@ struct TcCtrl {
   int consumed;  // tiles the MMA warp consumed
   int done;      // tiles the epilogue finished
 };
-
-// ------------------------------------------------------------ PTX helpers
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-      " selp.b32 %0, 1, 0, p;\n}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Bounded wait; on timeout (or once another role gave up) returns false. The
-// drain after an abort passes honor_abort = false: it must still wait for its
-// own copies and MMAs.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
-                                          unsigned *err, uint32_t limit = TC_SPIN_LIMIT,
-                                          bool honor_abort = true) {
-  for (uint32_t i = 0; i < limit; ++i) {
-    if (mbar_try(bar, parity)) return true;
-    if (honor_abort && (i & 255u) == 255u && *abort_flag) return false;
-  }
-  *abort_flag = 1;
-  raise_err(err, ERR_TIMEOUT);
-  return false;
-}
-__device__ __forceinline__ void mbar_arrive_expect(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, uint32_t bar,
-                                            int c0, int c1, int c2) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
-      "l"(map), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
-      : "memory");
-}
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar,
-                                            int c0, int c1) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
-      "l"(map), "r"(bar), "r"(c0), "r"(c1)
-      : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-// Arrive on `bar` once every cp.async this thread issued so far has landed
-// (the arrival counts toward the barrier's expected count).
-__device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc,
-                                       uint32_t accumulate) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(tmem_d),
-      "l"(da), "l"(db), "r"(idesc), "r"(accumulate));
-}
-__device__ __forceinline__ void tc_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   bar)
-               : "memory");
-}
-__device__ __forceinline__ void tc_ld16(uint32_t taddr, float (&v)[16]) {
-  uint32_t r[16];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
-      "%14,%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
-}
 
 __device__ __forceinline__ int tc_find_seq(const int *prefix, int B, int t) {
   int lo = 0, hi = B - 1;
@@ -549,13 +459,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   }
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
-                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
-                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+}  // namespace
 
-// cuTensorMapEncodeTiled from the driver (no link-time libcuda dependency).
-EncodeTiledFn encode_fn(cudaError_t *status) {
+EncodeTiledFn encode_tiled_fn(cudaError_t *status) {
   static std::once_flag once;
   static EncodeTiledFn fn = nullptr;
   static cudaError_t st = cudaSuccess;
@@ -570,10 +476,12 @@ EncodeTiledFn encode_fn(cudaError_t *status) {
   return fn;
 }
 
+namespace {
+
 template <int DI, int N>
 cudaError_t launch_tc_t(const qsa_cache &c, TcArgs a, cudaStream_t st) {
   cudaError_t e;
-  EncodeTiledFn enc = encode_fn(&e);
+  EncodeTiledFn enc = encode_tiled_fn(&e);
   if (e != cudaSuccess) return e;
   if (enc == nullptr) return cudaErrorNotSupported;
   // side pool viewed as [num_pages][rpp rows][DI]; q_idx as [B*Hi][DI]

@@ -34,7 +34,11 @@ CUDA library follows, are:
   blocks, LSE_r = ln sum_t exp z_t, O_r = sum_t softmax(z)_t V_t, and an empty
   slice gives O_r = 0, LSE_r = -inf;
 * merge: O = sum_r e^(LSE_r - m) O_r / sum_r e^(LSE_r - m), LSE = m +
-  ln sum_r e^(LSE_r - m), m = max_r LSE_r.
+  ln sum_r e^(LSE_r - m), m = max_r LSE_r;
+* sparse prefill (listed on the page beside the decode path, with no steps
+  given): every token of an appended chunk queries like a decode step over
+  its own causal prefix, i.e. the decode step of the sequence cut right
+  after that token.
 
 Floating point: fp64 for every dot product, softmax and merge; exact fp32
 (IEEE round-to-nearest adds and division) plus round-to-nearest-even to bf16
@@ -235,6 +239,46 @@ def decode_sequence(kidx_bits, k_bits, v_bits, q_bits, q_idx_bits, w, L: int, k:
     O_part, LSE_part = attend_slices(q_bits, k_bits, v_bits, use_sel, L, scale, R)
     O, LSE = merge_partials(O_part, LSE_part)
     return dict(scores=scores, sel=own_sel, O_part=O_part, LSE_part=LSE_part, O=O, LSE=LSE)
+
+
+# -------------------------------------------------------- sparse prefill
+
+def prefill_rows(seq_lens, row_start):
+    """Query rows of a chunked prefill (this library's reading of the sparse
+    prefill the page lists beside the decode path; the page describes no
+    step of it). Sequence s holds rows [row_start[s], row_start[s+1]): its
+    T_s newest tokens, already appended, so L_s = seq_lens[s] counts them.
+    Row i of sequence s is the token at position L_s - T_s + i; it queries
+    like a decode step of a sequence of length row_len = L_s - T_s + i + 1.
+    Returns (row_seq, row_len) as int64 arrays over all rows."""
+    seq_lens = [int(x) for x in seq_lens]
+    row_start = [int(x) for x in row_start]
+    assert len(row_start) == len(seq_lens) + 1 and row_start[0] == 0
+    row_seq, row_len = [], []
+    for s, L in enumerate(seq_lens):
+        T = row_start[s + 1] - row_start[s]
+        assert 0 <= T <= L
+        for i in range(T):
+            row_seq.append(s)
+            row_len.append(L - T + i + 1)
+    return np.asarray(row_seq, dtype=np.int64), np.asarray(row_len, dtype=np.int64)
+
+
+def prefill_sequence(kidx_bits, k_bits, v_bits, q_bits, q_idx_bits, w, L: int, T: int, k: int,
+                     R: int, scale: float, sels=None):
+    """The T chunk rows of one sequence of length L (after the chunk): row i is
+    the decode step (score -> top-k -> R-way split attention -> merge) of the
+    sequence cut to its first L - T + i + 1 tokens, with the row's own
+    q [Hq, D], q_idx [Hi, di] and w [Hi] (q_bits [T, Hq, D], q_idx_bits
+    [T, Hi, di], w [T, Hi]). ``sels`` [T, k], when given, replaces each row's
+    own selection in the attention. Returns one decode_sequence dict per row."""
+    out = []
+    for i in range(T):
+        ell = L - T + i + 1
+        out.append(decode_sequence(kidx_bits, k_bits, v_bits, np.asarray(q_bits)[i],
+                                   np.asarray(q_idx_bits)[i], np.asarray(w)[i], ell, k, R, scale,
+                                   sel=None if sels is None else np.asarray(sels)[i]))
+    return out
 
 
 # ------------------------------------------------------ paged cache append

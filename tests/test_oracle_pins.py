@@ -482,3 +482,97 @@ def test_context_parallel_merge_equals_single_rank_attention():
         Om, Lm = oracle.merge_partials(np.stack([o[0] for o, _ in parts]),
                                        np.stack([l[0] for _, l in parts]))
         assert np.abs(Om - O1[0]).max() <= 1e-12 and np.abs(Lm - L1[0]).max() <= 1e-12
+
+
+# ------------------------------------------------------------ sparse prefill
+
+def test_prefill_rows_hand():
+    # sequence 0: L=10, 3 chunk rows at positions 7, 8, 9; sequence 1: L=7,
+    # rows at 5, 6; sequence 2: no rows; sequence 3: the whole context is the chunk
+    row_seq, row_len = oracle.prefill_rows([10, 7, 3, 3], [0, 3, 5, 5, 8])
+    assert row_seq.tolist() == [0, 0, 0, 1, 1, 3, 3, 3]
+    assert row_len.tolist() == [8, 9, 10, 6, 7, 1, 2, 3]
+
+
+def _prefill_case(L, T, seed, D=32, Hq=8, Hkv=2, Hi=3, di=16):
+    g = torch.Generator().manual_seed(seed)
+    K = torch.randn(L, Hkv, D, generator=g).to(torch.bfloat16)
+    V = torch.randn(L, Hkv, D, generator=g).to(torch.bfloat16)
+    X = torch.randn(L, di, generator=g).to(torch.bfloat16)
+    q = torch.randn(T, Hq, D, generator=g).to(torch.bfloat16)
+    qi = torch.randn(T, Hi, di, generator=g).to(torch.bfloat16)
+    w = torch.rand(T, Hi, generator=g)
+    return K, V, X, q, qi, w
+
+
+@pytest.mark.parametrize("L,T", [(45, 9), (13, 13), (40, 1), (7, 3)])
+def test_prefill_dense_when_k_covers_the_context(L, T):
+    # k >= every row's block count: each row attends densely over its own
+    # causal prefix, i.e. a bottom-right causal mask over the chunk, by SDPA
+    K, V, X, q, qi, w = _prefill_case(L, T, seed=L * 100 + T)
+    scale = 0.21
+    rows = oracle.prefill_sequence(bits(X), bits(K), bits(V), bits(q), bits(qi), w.numpy(), L, T,
+                                   k=64, R=1, scale=scale)
+    G = q.shape[1] // K.shape[1]
+    qh = q.to(torch.float64).permute(1, 0, 2)[None]                          # [1, Hq, T, D]
+    Kh = K.to(torch.float64).repeat_interleave(G, dim=1).permute(1, 0, 2)[None]
+    Vh = V.to(torch.float64).repeat_interleave(G, dim=1).permute(1, 0, 2)[None]
+    mask = torch.arange(L)[None, :] <= (L - T + torch.arange(T))[:, None]   # [T, L]
+    ref = torch.nn.functional.scaled_dot_product_attention(qh, Kh, Vh, attn_mask=mask, scale=scale)
+    z = ((qh @ Kh.transpose(-1, -2)) * scale).masked_fill(~mask, float("-inf"))
+    lse = torch.logsumexp(z, dim=-1)[0].T.numpy()                           # [T, Hq]
+    for i, r in enumerate(rows):
+        assert np.allclose(r["O"], ref[0, :, i].numpy(), atol=1e-10, rtol=0)
+        assert np.allclose(r["LSE"], lse[i], atol=1e-10, rtol=0)
+        assert r["sel"][r["sel"] >= 0].tolist() == list(range((L - T + i + 1 + 3) // 4))
+
+
+def _brute_row_scores(X, qi_row, w_row, ell):
+    # the score definition written out with loops: block b holds tokens
+    # 4b..4b+3 that are < ell; its key is the bf16 rounding of the fp32
+    # left-to-right sum of those keys divided by their count
+    Xf = X.to(torch.float32)
+    out = []
+    for b in range((ell + 3) // 4):
+        toks = [t for t in range(4 * b, 4 * b + 4) if t < ell]
+        acc = Xf[toks[0]].clone()
+        for t in toks[1:]:
+            acc = acc + Xf[t]
+        kc = (acc / float(len(toks))).to(torch.bfloat16).to(torch.float64)
+        s = 0.0
+        for h in range(qi_row.shape[0]):
+            dot = float((qi_row[h].to(torch.float64) * kc).sum())
+            s += float(w_row[h]) * max(0.0, dot)
+        out.append(s)
+    return np.array(out)
+
+
+def test_prefill_row_scores_by_brute_force():
+    L, T = 23, 6   # rows see 18..23 tokens: partial blocks of every size
+    K, V, X, q, qi, w = _prefill_case(L, T, seed=99)
+    rows = oracle.prefill_sequence(bits(X), bits(K), bits(V), bits(q), bits(qi), w.numpy(), L, T,
+                                   k=3, R=2, scale=0.3)
+    for i, r in enumerate(rows):
+        ref = _brute_row_scores(X, qi[i], w[i], L - T + i + 1)
+        assert r["scores"].shape == ref.shape
+        assert np.allclose(r["scores"], ref, rtol=1e-12, atol=1e-12)
+
+
+def test_prefill_rows_ignore_later_tokens():
+    L, T = 61, 5
+    K, V, X, q, qi, w = _prefill_case(L, T, seed=7)
+    args = dict(L=L, T=T, k=4, R=3, scale=0.25)
+    base = oracle.prefill_sequence(bits(X), bits(K), bits(V), bits(q), bits(qi), w.numpy(), **args)
+    for i in range(T):
+        pos = L - T + i
+        K2, V2, X2 = K.clone(), V.clone(), X.clone()
+        K2[pos + 1:] = -K2[pos + 1:] * 3
+        V2[pos + 1:] = V2[pos + 1:] + 5
+        X2[pos + 1:] = -X2[pos + 1:]
+        got = oracle.prefill_sequence(bits(X2), bits(K2), bits(V2), bits(q), bits(qi), w.numpy(),
+                                      **args)
+        assert np.array_equal(got[i]["sel"], base[i]["sel"])
+        assert np.array_equal(got[i]["scores"], base[i]["scores"])
+        assert np.array_equal(got[i]["O"], base[i]["O"])
+        if i + 1 < T:   # a later row sees the change
+            assert not np.array_equal(got[T - 1]["O"], base[T - 1]["O"])
