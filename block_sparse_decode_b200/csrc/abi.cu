@@ -360,6 +360,120 @@ qsa_status qsa_decode_step(const qsa_dims *dims, const qsa_cache *cache, int32_t
   return st;
 }
 
+size_t qsa_prefill_index_score_workspace_size(const qsa_dims *dims, int32_t S, int32_t Nq) {
+  if (dims == nullptr || S < 0 || Nq < 0 || !prefill_supported(*dims)) return 0;
+  return prefill_plan_ws_bytes(*dims, S, Nq);
+}
+
+qsa_status qsa_prefill_index_score(const qsa_dims *dims, const qsa_cache *cache, int32_t S,
+                                   const int32_t *seq_lens, const int32_t *row_start, int32_t Nq,
+                                   const void *q_idx, const float *w, float *scores,
+                                   int32_t ld_scores, int32_t *row_len, void *ws,
+                                   size_t ws_bytes, qsa_stream_t stream) {
+  try {
+    QSA_TRY(check_dims(dims));
+    QSA_TRY(check_cache(cache, false, true));
+    if (S < 0 || S > cache->num_seqs)
+      return fail(QSA_ERR_INVALID_ARG, "S=%d outside [0, block_table rows %d]", S,
+                  cache->num_seqs);
+    if (Nq < 0 || Nq > 65535) return fail(QSA_ERR_INVALID_ARG, "Nq=%d outside [0, 65535]", Nq);
+    if (ld_scores <= 0) return fail(QSA_ERR_INVALID_ARG, "ld_scores must be positive");
+    if (!prefill_supported(*dims))
+      return fail(QSA_ERR_UNSUPPORTED,
+                  "qsa_prefill_index_score needs Hi in {4, 8, 16, 32} and the page size P a "
+                  "power of two in [32, 1024]");
+    if (S == 0 || Nq == 0) return ok();
+    if (seq_lens == nullptr || row_start == nullptr || q_idx == nullptr || w == nullptr ||
+        scores == nullptr || row_len == nullptr || ws == nullptr)
+      return fail(QSA_ERR_INVALID_ARG, "an argument array is NULL");
+    if (!aligned16(q_idx) || !aligned16(ws))
+      return fail(QSA_ERR_INVALID_ARG, "q_idx / ws not 16-byte aligned");
+    const size_t need = prefill_plan_ws_bytes(*dims, S, Nq);
+    if (ws_bytes < need)
+      return fail(QSA_ERR_INVALID_ARG, "workspace %zu bytes < %zu needed", ws_bytes, need);
+    QSA_ERRWORD(err);
+    return cuda_status(launch_prefill_index_score(*dims, *cache, S, seq_lens, row_start, Nq,
+                                                  q_idx, w, scores, ld_scores, row_len, ws, err,
+                                                  reinterpret_cast<cudaStream_t>(stream)),
+                       "qsa_prefill_index_score launch");
+  } catch (...) {
+    return fail(QSA_ERR_CUDA, "qsa_prefill_index_score: internal exception");
+  }
+}
+
+qsa_status qsa_prefill_sparse_decode(const qsa_dims *dims, const qsa_cache *cache, int32_t S,
+                                     const int32_t *seq_lens, const int32_t *row_start,
+                                     int32_t Nq, const void *q, const int32_t *sel, int32_t k,
+                                     int32_t R, float *o_part, float *lse_part, void *ws,
+                                     size_t ws_bytes, qsa_stream_t stream) {
+  try {
+    QSA_TRY(check_dims(dims));
+    QSA_TRY(check_cache(cache, true, false));
+    if (S < 0 || S > cache->num_seqs)
+      return fail(QSA_ERR_INVALID_ARG, "S=%d outside [0, block_table rows %d]", S,
+                  cache->num_seqs);
+    if (Nq < 0 || Nq > 65535) return fail(QSA_ERR_INVALID_ARG, "Nq=%d outside [0, 65535]", Nq);
+    if (k < 1 || k > 4096) return fail(QSA_ERR_UNSUPPORTED, "k=%d outside [1, 4096]", k);
+    if (R < 1 || R > 64) return fail(QSA_ERR_UNSUPPORTED, "R=%d outside [1, 64]", R);
+    if (S == 0 || Nq == 0) return ok();
+    if (seq_lens == nullptr || row_start == nullptr || q == nullptr || sel == nullptr ||
+        o_part == nullptr || lse_part == nullptr || ws == nullptr)
+      return fail(QSA_ERR_INVALID_ARG, "an argument array is NULL");
+    if (!aligned16(q) || !aligned16(o_part) || !aligned16(ws))
+      return fail(QSA_ERR_INVALID_ARG, "q / o_part / ws not 16-byte aligned");
+    const size_t need = decode_ws_bytes(*dims, Nq, 1, k, R);
+    if (ws_bytes < need)
+      return fail(QSA_ERR_INVALID_ARG, "workspace %zu bytes < %zu needed", ws_bytes, need);
+    QSA_ERRWORD(err);
+    return cuda_status(launch_sparse_decode(*dims, *cache, Nq, 1, seq_lens, q, sel, k, R, o_part,
+                                            lse_part, ws, err,
+                                            reinterpret_cast<cudaStream_t>(stream), row_start, S),
+                       "qsa_prefill_sparse_decode launch");
+  } catch (...) {
+    return fail(QSA_ERR_CUDA, "qsa_prefill_sparse_decode: internal exception");
+  }
+}
+
+namespace {
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+}  // namespace
+
+size_t qsa_sparse_prefill_workspace_size(const qsa_dims *dims, int32_t S, int32_t Nq, int32_t k,
+                                         int32_t R) {
+  if (dims == nullptr || S < 0 || Nq <= 0 || k <= 0 || R <= 0 || dims->Hkv <= 0 ||
+      dims->Hq <= 0 || !prefill_supported(*dims))
+    return 0;
+  return align256(prefill_plan_ws_bytes(*dims, S, Nq)) + decode_ws_bytes(*dims, Nq, 1, k, R);
+}
+
+qsa_status qsa_sparse_prefill(const qsa_dims *dims, const qsa_cache *cache, int32_t S,
+                              const int32_t *seq_lens, const int32_t *row_start, int32_t Nq,
+                              const void *q, const void *q_idx, const float *w, int32_t k,
+                              int32_t R, float *scores, int32_t ld_scores, int32_t *row_len,
+                              int32_t *sel, float *o_part, float *lse_part, void *ws,
+                              size_t ws_bytes, void *out, int32_t out_is_bf16, float *lse_out,
+                              qsa_stream_t stream) {
+  if (dims == nullptr) return fail(QSA_ERR_INVALID_ARG, "dims is NULL");
+  if (S < 0 || Nq < 0) return fail(QSA_ERR_INVALID_ARG, "S or Nq negative");
+  if (S == 0 || Nq == 0) return ok();
+  if (!prefill_supported(*dims))
+    return fail(QSA_ERR_UNSUPPORTED, "qsa_sparse_prefill needs Hi in {4, 8, 16, 32}");
+  const size_t plan = align256(prefill_plan_ws_bytes(*dims, S, Nq));
+  if (ws == nullptr || ws_bytes < plan)
+    return fail(QSA_ERR_INVALID_ARG, "workspace of %zu bytes is too small", ws_bytes);
+  unsigned char *wd = static_cast<unsigned char *>(ws) + plan;
+  qsa_status st = qsa_prefill_index_score(dims, cache, S, seq_lens, row_start, Nq, q_idx, w,
+                                          scores, ld_scores, row_len, ws, plan, stream);
+  if (st == QSA_OK)
+    st = qsa_topk_select(Nq, row_len, scores, ld_scores, k, sel, nullptr, 0, stream);
+  if (st == QSA_OK)
+    st = qsa_prefill_sparse_decode(dims, cache, S, seq_lens, row_start, Nq, q, sel, k, R, o_part,
+                                   lse_part, wd, ws_bytes - plan, stream);
+  if (st == QSA_OK)
+    st = qsa_merge(R, Nq, dims->Hq, dims->D, o_part, lse_part, out, out_is_bf16, lse_out, stream);
+  return st;
+}
+
 qsa_status qsa_check_device_errors(qsa_stream_t stream, int32_t *flags) {
   try {
     if (flags) *flags = 0;

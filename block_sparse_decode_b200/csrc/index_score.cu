@@ -102,54 +102,12 @@ __device__ __forceinline__ int tc_find_seq(const int *prefix, int B, int t) {
 }
 
 // Score of the trailing partial block of sequence b (whole warp; every lane
-// returns it). The key is the bf16-rounded mean of its L mod 4 indexer keys,
-// built exactly as the side cache builds complete blocks.
+// returns it).
 template <int DI>
 __device__ float partial_block_score(const TcArgs &a, int b, int L, bool *ok_out) {
-  const int lane = threadIdx.x & 31;
-  const int nfull = L >> 2, n = L - 4 * nfull, pos = 4 * nfull;
-  const int col = pos / a.P;
-  int page = -1;
-  if (col < a.max_pages) page = a.block_table[(size_t)b * a.max_pages + col];
-  const bool ok = page >= 0 && page < a.num_pages;
-  *ok_out = ok;
-  if (!ok) {
-    if (lane == 0) raise_err(a.err, col < a.max_pages ? ERR_PAGE : ERR_BT);
-    return 0.f;
-  }
-  const uint32_t *x = reinterpret_cast<const uint32_t *>(a.kidx_pool) +
-                      ((size_t)page * a.P + pos % a.P) * (DI / 2);
-  float klo[DI / 64], khi[DI / 64];
-#pragma unroll
-  for (int i = 0; i < DI / 64; ++i) {
-    const int e = lane + 32 * i;
-    uint32_t v = x[e];
-    float lo = bf16lo(v), hi = bf16hi(v);
-    for (int u = 1; u < n; ++u) {
-      v = x[u * (DI / 2) + e];
-      lo = __fadd_rn(lo, bf16lo(v));
-      hi = __fadd_rn(hi, bf16hi(v));
-    }
-    const uint32_t kc = pack_bf16x2(__fdiv_rn(lo, (float)n), __fdiv_rn(hi, (float)n));
-    klo[i] = bf16lo(kc);
-    khi[i] = bf16hi(kc);
-  }
-  float score = 0.f;
-  for (int h = 0; h < a.Hi; ++h) {
-    const uint32_t *qrow =
-        reinterpret_cast<const uint32_t *>(a.q_idx + ((size_t)b * a.Hi + h) * DI);
-    float part = 0.f;
-#pragma unroll
-    for (int i = 0; i < DI / 64; ++i) {
-      const uint32_t q = qrow[lane + 32 * i];
-      part = fmaf(klo[i], bf16lo(q), part);
-      part = fmaf(khi[i], bf16hi(q), part);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-    score = fmaf(a.w[(size_t)b * a.Hi + h], fmaxf(part, 0.f), score);
-  }
-  return score;
+  return partial_block_score_row<DI>(a.kidx_pool, a.P, a.block_table + (size_t)b * a.max_pages,
+                                     a.max_pages, a.num_pages, L, a.q_idx + (size_t)b * a.Hi * DI,
+                                     a.w + (size_t)b * a.Hi, a.Hi, a.err, ok_out);
 }
 
 template <int DI, int N>

@@ -53,13 +53,27 @@ cudaError_t launch_topk(int B, const int32_t *seq_lens, const float *scores, int
                         int32_t *sel, unsigned *err, cudaStream_t st);
 
 size_t decode_ws_bytes(const qsa_dims &d, int B, int Qn, int k, int R);
+// row_start != nullptr: B prefill rows of S chunks (sequence s holds rows
+// [row_start[s], row_start[s+1]), seq_lens[s] counts its chunk), Qn = 1.
 cudaError_t launch_sparse_decode(const qsa_dims &d, const qsa_cache &c, int B, int Qn,
                                  const int32_t *seq_lens, const void *q, const int32_t *sel,
                                  int k, int R, float *o_part, float *lse_part, void *ws,
-                                 unsigned *err, cudaStream_t st);
+                                 unsigned *err, cudaStream_t st,
+                                 const int32_t *row_start = nullptr, int S = 0);
 
 cudaError_t launch_select_owned(const int32_t *sel, int B, int k, int P, int W, int r,
                                 int32_t *out, cudaStream_t st);
+
+// Sparse prefill scoring (prefill.cu): query rows of appended chunks, groups
+// of prefill_group_rows(d) rows of one sequence sharing each side-cache tile.
+bool prefill_supported(const qsa_dims &d);
+int prefill_group_rows(const qsa_dims &d);
+size_t prefill_plan_ws_bytes(const qsa_dims &d, int S, int Nq);
+cudaError_t launch_prefill_index_score(const qsa_dims &d, const qsa_cache &c, int S,
+                                       const int32_t *seq_lens, const int32_t *row_start, int Nq,
+                                       const void *q_idx, const float *w, float *scores, int ld,
+                                       int32_t *row_len, void *ws, unsigned *err,
+                                       cudaStream_t st);
 
 cudaError_t launch_merge(int R, int B, int Hq, int D, const float *o_part, const float *lse_part,
                          void *out, int out_is_bf16, float *lse_out, cudaStream_t st);

@@ -65,6 +65,11 @@ constexpr float LN2 = 0.6931471805599453f;
 struct DecodeArgs {
   const __nv_bfloat16 *k_pool, *v_pool, *q;  // q [B, Qn, Hq, D]
   const int32_t *block_table, *seq_lens, *sel;
+  // prefill rows (nullptr for decode): row b belongs to the sequence s with
+  // row_start[s] <= b < row_start[s+1] and sees L_s - T_s + (b - row_start[s]) + 1
+  // tokens (T_s its chunk rows), through block-table row s
+  const int32_t *row_start;
+  int S;
   float *o_part, *lse_part;  // [R, B, Qn, Hq, D], [R, B, Qn, Hq]
   float *rec_o, *rec_lse;    // [B, rb, QN, Hq, D], [B, rb, QN, Hq]: shared-slice partials
   int2 *span;                // [B, R]: contributors (c_lo, c_hi) of a shared slice
@@ -255,11 +260,31 @@ __global__ void __launch_bounds__(DV_WARPS * 32, DV_CTAS_PER_SM) sparse_decode_k
 
   // (1) L_b, the block-table row into L2, the query; then, once the top-k
   // kernel before this one has finished, the selection row
+  int bs = b;  // block-table row
   {
-    if (tid == 0) s_L = a.seq_lens[b];
+    int L;
+    if (a.row_start == nullptr) {
+      L = a.seq_lens[b];
+    } else {  // prefill row: the chunk holding it (every thread; S is small)
+      int lo = 0, hi = a.S - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (__ldg(a.row_start + mid) <= b) lo = mid; else hi = mid - 1;
+      }
+      const int r0 = __ldg(a.row_start + lo), r1 = __ldg(a.row_start + lo + 1);
+      const int Ls = __ldg(a.seq_lens + lo);
+      L = 0;  // a row outside every chunk attends to nothing
+      if (r0 <= b && b < r1 && r1 - r0 <= Ls) {
+        L = Ls - (r1 - r0) + (b - r0) + 1;
+        bs = lo;
+      } else if (tid == 0) {
+        raise_err(a.err, ERR_LEN);
+      }
+    }
+    if (tid == 0) s_L = L;
     // the CTAs of a sequence pull its block-table row into L2 together, so
     // the page lookups after the slice search hit L2
-    const char *bt_row = reinterpret_cast<const char *>(a.block_table + (size_t)b * a.max_pages);
+    const char *bt_row = reinterpret_cast<const char *>(a.block_table + (size_t)bs * a.max_pages);
     const int lines = (a.max_pages * 4 + 127) >> 7;
     for (int i = c + CL * tid; i < lines; i += CL * (int)blockDim.x)
       asm volatile("prefetch.global.L2 [%0];\n" ::"l"(bt_row + ((size_t)i << 7)));
@@ -376,7 +401,7 @@ __global__ void __launch_bounds__(DV_WARPS * 32, DV_CTAS_PER_SM) sparse_decode_k
             if (col >= a.max_pages) {
               raise_err(a.err, ERR_BT);
             } else {
-              idx[u] = (long long)b * a.max_pages + col;
+              idx[u] = (long long)bs * a.max_pages + col;
               jj[u] = j;
             }
           }
@@ -654,7 +679,8 @@ size_t decode_ws_bytes(const qsa_dims &d, int B, int Qn, int k, int R) {
 cudaError_t launch_sparse_decode(const qsa_dims &d, const qsa_cache &c, int B, int Qn,
                                  const int32_t *seq_lens, const void *q, const int32_t *sel,
                                  int k, int R, float *o_part, float *lse_part, void *ws,
-                                 unsigned *err, cudaStream_t st) {
+                                 unsigned *err, cudaStream_t st, const int32_t *row_start,
+                                 int S) {
   if (B == 0) return cudaSuccess;
   const DecodePlan p = plan_decode(d, B, k, R);
   DecodeArgs a;
@@ -664,6 +690,8 @@ cudaError_t launch_sparse_decode(const qsa_dims &d, const qsa_cache &c, int B, i
   a.block_table = c.block_table;
   a.seq_lens = seq_lens;
   a.sel = sel;
+  a.row_start = row_start;
+  a.S = S;
   a.o_part = o_part;
   a.lse_part = lse_part;
   a.B = B;

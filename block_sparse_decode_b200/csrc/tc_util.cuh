@@ -1,6 +1,7 @@
 // Device helpers shared by the tensor-core scoring kernels (decode and
 // prefill): mbarriers with bounded waits, TMA tile loads, tcgen05 MMA issue,
-// commit and TMEM loads, and the host lookup of cuTensorMapEncodeTiled.
+// commit and TMEM loads, the partial-block score on CUDA cores, and the host
+// lookup of cuTensorMapEncodeTiled.
 #pragma once
 
 #include <cuda.h>
@@ -97,6 +98,77 @@ __device__ __forceinline__ void tc_ld16(uint32_t taddr, float (&v)[16]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tc_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Score of the trailing partial block of a query whose context is the first
+// L tokens of the sequence with block-table row bt_row (whole warp; every
+// lane returns it). The key is the bf16-rounded mean of its L mod 4 indexer
+// keys, built exactly as the side cache builds complete blocks; q_rows holds
+// the query's Hi indexer rows of DI elements, w_row its Hi head weights.
+template <int DI>
+__device__ float partial_block_score_row(const __nv_bfloat16 *kidx_pool, int P,
+                                         const int32_t *bt_row, int max_pages, int num_pages,
+                                         int L, const __nv_bfloat16 *q_rows, const float *w_row,
+                                         int Hi, unsigned *err, bool *ok_out) {
+  const int lane = threadIdx.x & 31;
+  const int nfull = L >> 2, n = L - 4 * nfull, pos = 4 * nfull;
+  const int col = pos / P;
+  int page = -1;
+  if (col < max_pages) page = bt_row[col];
+  const bool ok = page >= 0 && page < num_pages;
+  *ok_out = ok;
+  if (!ok) {
+    if (lane == 0) raise_err(err, col < max_pages ? ERR_PAGE : ERR_BT);
+    return 0.f;
+  }
+  const uint32_t *x = reinterpret_cast<const uint32_t *>(kidx_pool) +
+                      ((size_t)page * P + pos % P) * (DI / 2);
+  float klo[DI / 64], khi[DI / 64];
+#pragma unroll
+  for (int i = 0; i < DI / 64; ++i) {
+    const int e = lane + 32 * i;
+    uint32_t v = x[e];
+    float lo = bf16lo(v), hi = bf16hi(v);
+    for (int u = 1; u < n; ++u) {
+      v = x[u * (DI / 2) + e];
+      lo = __fadd_rn(lo, bf16lo(v));
+      hi = __fadd_rn(hi, bf16hi(v));
+    }
+    const uint32_t kc = pack_bf16x2(__fdiv_rn(lo, (float)n), __fdiv_rn(hi, (float)n));
+    klo[i] = bf16lo(kc);
+    khi[i] = bf16hi(kc);
+  }
+  float score = 0.f;
+  for (int h = 0; h < Hi; ++h) {
+    const uint32_t *qrow = reinterpret_cast<const uint32_t *>(q_rows + (size_t)h * DI);
+    float part = 0.f;
+#pragma unroll
+    for (int i = 0; i < DI / 64; ++i) {
+      const uint32_t q = qrow[lane + 32 * i];
+      part = fmaf(klo[i], bf16lo(q), part);
+      part = fmaf(khi[i], bf16hi(q), part);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    score = fmaf(w_row[h], fmaxf(part, 0.f), score);
+  }
+  return score;
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,

@@ -31,7 +31,10 @@ EXPORTS = ("qsa_version", "qsa_last_error", "qsa_append", "qsa_index_score",
            "qsa_topk_workspace_size", "qsa_topk_select", "qsa_sparse_decode_workspace_size",
            "qsa_sparse_decode", "qsa_sparse_decode_static", "qsa_merge",
            "qsa_decode_step", "qsa_sparse_decode_mq_workspace_size", "qsa_sparse_decode_mq",
-           "qsa_select_owned", "qsa_check_device_errors")
+           "qsa_select_owned", "qsa_check_device_errors",
+           "qsa_prefill_index_score_workspace_size", "qsa_prefill_index_score",
+           "qsa_prefill_sparse_decode", "qsa_sparse_prefill_workspace_size",
+           "qsa_sparse_prefill")
 
 
 class QsaError(RuntimeError):
@@ -84,6 +87,13 @@ def lib() -> ctypes.CDLL:
         "qsa_decode_step": (I32, [DP, CP, I32, P, P, P, P, P, I32, P, P, P, P, I32, I32, P, I32,
                                   P, P, P, P, SZ, P, I32, P, P]),
         "qsa_check_device_errors": (I32, [P, ctypes.POINTER(I32)]),
+        "qsa_prefill_index_score_workspace_size": (SZ, [DP, I32, I32]),
+        "qsa_prefill_index_score": (I32, [DP, CP, I32, P, P, I32, P, P, P, I32, P, P, SZ, P]),
+        "qsa_prefill_sparse_decode": (I32, [DP, CP, I32, P, P, I32, P, P, I32, I32, P, P, P, SZ,
+                                            P]),
+        "qsa_sparse_prefill_workspace_size": (SZ, [DP, I32, I32, I32, I32]),
+        "qsa_sparse_prefill": (I32, [DP, CP, I32, P, P, I32, P, P, P, I32, I32, P, I32, P, P, P,
+                                     P, P, SZ, P, I32, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -361,3 +371,85 @@ def decode_step(dims: QsaDims, cache: QsaCache, seq_lens, q, q_idx, w, k: int, R
 def ld_for(seq_lens) -> int:
     """Smallest score row length that holds every sequence's blocks."""
     return max(1, max(int(math.ceil(int(L) / 4)) for L in seq_lens))
+
+
+# ------------------------------------------------------------ sparse prefill
+
+def qsa_prefill_index_score_workspace_size(dims: QsaDims, S: int, Nq: int) -> int:
+    return int(lib().qsa_prefill_index_score_workspace_size(ctypes.byref(dims.c()), S, Nq))
+
+
+def qsa_prefill_index_score(dims: QsaDims, cache: QsaCache, seq_lens, row_start, q_idx, w,
+                            scores, row_len, ws, stream=None):
+    """Scores of every prefill row: q_idx [Nq, Hi, di] -> scores [Nq, ld], row_len [Nq]."""
+    S, Nq = int(seq_lens.shape[0]), int(q_idx.shape[0])
+    _check(lib().qsa_prefill_index_score(
+        ctypes.byref(dims.c()), ctypes.byref(cache.c()), S,
+        _ptr(seq_lens, torch.int32, "seq_lens"), _ptr(row_start, torch.int32, "row_start"), Nq,
+        _ptr(q_idx, torch.bfloat16, "q_idx"), _ptr(w, torch.float32, "w"),
+        _ptr(scores, torch.float32, "scores"), int(scores.shape[1]),
+        _ptr(row_len, torch.int32, "row_len"), _ptr(ws, None, "ws"),
+        ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def qsa_prefill_sparse_decode(dims: QsaDims, cache: QsaCache, seq_lens, row_start, q, sel,
+                              k: int, R: int, o_part, lse_part, ws, stream=None):
+    """Split attention of every prefill row: q [Nq, Hq, D] -> o_part [R, Nq, Hq, D]."""
+    S, Nq = int(seq_lens.shape[0]), int(q.shape[0])
+    _check(lib().qsa_prefill_sparse_decode(
+        ctypes.byref(dims.c()), ctypes.byref(cache.c()), S,
+        _ptr(seq_lens, torch.int32, "seq_lens"), _ptr(row_start, torch.int32, "row_start"), Nq,
+        _ptr(q, torch.bfloat16, "q"), _ptr(sel, torch.int32, "sel"), int(k), int(R),
+        _ptr(o_part, torch.float32, "o_part"), _ptr(lse_part, torch.float32, "lse_part"),
+        _ptr(ws, None, "ws"), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def qsa_sparse_prefill_workspace_size(dims: QsaDims, S: int, Nq: int, k: int, R: int) -> int:
+    return int(lib().qsa_sparse_prefill_workspace_size(ctypes.byref(dims.c()), S, Nq, k, R))
+
+
+@dataclass
+class PrefillBuffers:
+    """Outputs and scratch of one sparse prefill for fixed (S, Nq, k, R, ld)."""
+
+    scores: torch.Tensor     # fp32 [Nq, ld]
+    row_len: torch.Tensor    # int32 [Nq]
+    sel: torch.Tensor        # int32 [Nq, k]
+    o_part: torch.Tensor     # fp32 [R, Nq, Hq, D]
+    lse_part: torch.Tensor   # fp32 [R, Nq, Hq]
+    out: torch.Tensor        # bf16 [Nq, Hq, D]
+    lse: torch.Tensor        # fp32 [Nq, Hq]
+    ws: torch.Tensor         # uint8 scratch of qsa_sparse_prefill
+
+
+def alloc_prefill(dims: QsaDims, S: int, Nq: int, ld: int, k: int, R: int, device="cuda",
+                  out_dtype=torch.bfloat16) -> PrefillBuffers:
+    ws_bytes = max(16, qsa_sparse_prefill_workspace_size(dims, S, Nq, k, R))
+    return PrefillBuffers(
+        scores=torch.empty((Nq, ld), dtype=torch.float32, device=device),
+        row_len=torch.empty((Nq,), dtype=torch.int32, device=device),
+        sel=torch.empty((Nq, k), dtype=torch.int32, device=device),
+        o_part=torch.empty((R, Nq, dims.Hq, dims.D), dtype=torch.float32, device=device),
+        lse_part=torch.empty((R, Nq, dims.Hq), dtype=torch.float32, device=device),
+        out=torch.empty((Nq, dims.Hq, dims.D), dtype=out_dtype, device=device),
+        lse=torch.empty((Nq, dims.Hq), dtype=torch.float32, device=device),
+        ws=torch.empty((ws_bytes,), dtype=torch.uint8, device=device))
+
+
+def sparse_prefill(dims: QsaDims, cache: QsaCache, seq_lens, row_start, q, q_idx, w, k: int,
+                   R: int, buf: PrefillBuffers, stream=None):
+    """Sparse prefill of the chunk rows (already appended): score -> top-k ->
+    split attention -> merge per row, by the library's single qsa_sparse_prefill
+    call. Results land in ``buf``."""
+    S, Nq = int(seq_lens.shape[0]), int(q.shape[0])
+    _check(lib().qsa_sparse_prefill(
+        ctypes.byref(dims.c()), ctypes.byref(cache.c()), S,
+        _ptr(seq_lens, torch.int32, "seq_lens"), _ptr(row_start, torch.int32, "row_start"), Nq,
+        _ptr(q, torch.bfloat16, "q"), _ptr(q_idx, torch.bfloat16, "q_idx"),
+        _ptr(w, torch.float32, "w"), int(k), int(R), _ptr(buf.scores, torch.float32, "scores"),
+        int(buf.scores.shape[1]), _ptr(buf.row_len, torch.int32, "row_len"),
+        _ptr(buf.sel, torch.int32, "sel"), _ptr(buf.o_part, torch.float32, "o_part"),
+        _ptr(buf.lse_part, torch.float32, "lse_part"), _ptr(buf.ws, None, "ws"),
+        buf.ws.numel() * buf.ws.element_size(), _ptr(buf.out, None, "out"),
+        1 if buf.out.dtype == torch.bfloat16 else 0, _ptr(buf.lse, torch.float32, "lse"),
+        _stream(stream)))

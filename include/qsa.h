@@ -288,6 +288,86 @@ qsa_status qsa_decode_step(const qsa_dims *dims, const qsa_cache *cache,
                            int32_t out_is_bf16, float *lse_out,
                            qsa_stream_t stream);
 
+/* ---------------------------------------------------------- sparse prefill
+ * Page "Qwen 4 QSA gets decode context parallelism" (orcarouter.ai), section
+ * "Why a serving PR about an unreleased architecture is still worth your
+ * time": the engine work around the decode path includes a native sparse
+ * prefill kernel for the QSA path; the page gives none of its steps. This
+ * library's reading: every token of an appended chunk queries like a decode
+ * step over its own causal prefix.
+ * Chunks: sequence s (0 <= s < S, block-table row s) holds the query rows
+ * [row_start[s], row_start[s+1]) (int32 [S + 1], non-decreasing, row_start[0]
+ * = 0, row_start[S] = Nq): its T_s = row_start[s+1] - row_start[s] newest
+ * tokens, already appended (qsa_append), so that seq_lens[s] = L_s >= T_s
+ * counts them. Row i of sequence s is the token at position L_s - T_s + i;
+ * its causal length is row_len = L_s - T_s + i + 1, and its result is the
+ * decode step of a sequence of that length (score its ceil(row_len / 4)
+ * blocks, keep the min(k, .) best, attend over their tokens < row_len, split
+ * R ways, merge). Rows are in chunk order: q, q_idx, w, scores, sel and the
+ * partials are indexed by row. Supported: as qsa_index_score, and Hi in
+ * {4, 8, 16, 32}; 0 <= Nq <= 65535. A chunk whose rows overrun Nq, whose
+ * T_s exceeds L_s or whose ceil(L_s / 4) blocks exceed ld_scores is skipped
+ * (its rows get row_len 0 and attend to nothing) and raises device error
+ * flag 16. */
+
+/* Scratch bytes of qsa_prefill_index_score. */
+size_t qsa_prefill_index_score_workspace_size(const qsa_dims *dims, int32_t S,
+                                              int32_t Nq);
+
+/* Indexer scores of every prefill row (qsa_index_score per row):
+ *   q_idx   bf16 [Nq, Hi, di] (16-byte aligned);  w  fp32 [Nq, Hi]
+ *   scores  fp32 [Nq, ld_scores]: row r's blocks j < ceil(row_len[r] / 4)
+ *           are written, nothing else
+ *   row_len int32 [Nq] (out): each row's causal length, the sequence
+ *           lengths qsa_topk_select takes for the rows (0 for a row of a
+ *           skipped chunk)
+ *   ws      scratch of qsa_prefill_index_score_workspace_size bytes,
+ *           16-byte aligned, no initialisation needed; used until the call's
+ *           kernels finish.
+ * Up to 256 / Hi consecutive rows of one chunk share each 128-block tile of
+ * the side cache in one tensor-core MMA. */
+qsa_status qsa_prefill_index_score(const qsa_dims *dims, const qsa_cache *cache,
+                                   int32_t S, const int32_t *seq_lens,
+                                   const int32_t *row_start, int32_t Nq,
+                                   const void *q_idx, const float *w,
+                                   float *scores, int32_t ld_scores,
+                                   int32_t *row_len, void *ws, size_t ws_bytes,
+                                   qsa_stream_t stream);
+
+/* Split sparse attention of every prefill row over its own selection
+ * (qsa_sparse_decode per row, at the row's causal length):
+ *   q        bf16 [Nq, Hq, D];  sel  int32 [Nq, k] (e.g. qsa_topk_select over
+ *            the rows with row_len as sequence lengths)
+ *   o_part   fp32 [R, Nq, Hq, D];  lse_part  fp32 [R, Nq, Hq]
+ *   ws       qsa_sparse_decode_workspace_size(dims, Nq, k, R) bytes.
+ * qsa_merge with B = Nq combines the partials. */
+qsa_status qsa_prefill_sparse_decode(const qsa_dims *dims, const qsa_cache *cache,
+                                     int32_t S, const int32_t *seq_lens,
+                                     const int32_t *row_start, int32_t Nq,
+                                     const void *q, const int32_t *sel, int32_t k,
+                                     int32_t R, float *o_part, float *lse_part,
+                                     void *ws, size_t ws_bytes, qsa_stream_t stream);
+
+/* Scratch bytes of qsa_sparse_prefill. */
+size_t qsa_sparse_prefill_workspace_size(const qsa_dims *dims, int32_t S, int32_t Nq,
+                                         int32_t k, int32_t R);
+
+/* The whole sparse prefill of the rows: qsa_prefill_index_score,
+ * qsa_topk_select (rows, row_len), qsa_prefill_sparse_decode and qsa_merge
+ * (B = Nq: out [Nq, Hq, D], lse_out [Nq, Hq]) enqueued in that order, with
+ * the arguments documented there; ws holds
+ * qsa_sparse_prefill_workspace_size bytes (16-byte aligned). The chunk's
+ * tokens must already be appended. An interface convenience of this library
+ * (one call instead of four); the first failing call stops the sequence. */
+qsa_status qsa_sparse_prefill(const qsa_dims *dims, const qsa_cache *cache, int32_t S,
+                              const int32_t *seq_lens, const int32_t *row_start,
+                              int32_t Nq, const void *q, const void *q_idx,
+                              const float *w, int32_t k, int32_t R, float *scores,
+                              int32_t ld_scores, int32_t *row_len, int32_t *sel,
+                              float *o_part, float *lse_part, void *ws,
+                              size_t ws_bytes, void *out, int32_t out_is_bf16,
+                              float *lse_out, qsa_stream_t stream);
+
 /* Wait for `stream`, then read and clear the device error word of the
  * current device. *flags receives the bits that were set (0 if none):
  *   1 sequence row out of range    2 page id out of range

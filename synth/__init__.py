@@ -15,5 +15,6 @@ from .workloads import (  # noqa: F401
     make_workload,
     make_custom,
     step_queries,
+    prefill_queries,
     seed_for,
 )

@@ -39,6 +39,7 @@ BASE_SEED = 20261202
 # RNG stream ids, in the fixed order the tensors are drawn.
 _S_LENS, _S_K, _S_V, _S_KIDX, _S_Q, _S_QIDX, _S_W, _S_PAGES, _S_NEEDLE, _S_MIX = range(10)
 _S_STEP = 100  # + step index: per-step queries of the append workload
+_S_PREFILL = 90  # query rows of a prefill chunk
 
 
 def seed_for(preset: str) -> int:
@@ -282,3 +283,24 @@ def step_queries(wl: Workload, t: int):
     q_idx = torch.randn((B, d.Hi, d.di), generator=g, device=dev).to(torch.bfloat16)
     w = torch.rand((B, d.Hi), generator=g, device=dev)
     return q, q_idx, w
+
+
+def prefill_queries(wl: Workload, chunk_lens, seed: int | None = None):
+    """Query rows of a sparse prefill whose chunks are the chunk_lens[s]
+    newest tokens of each sequence (already part of seq_lens[s]): returns
+    (row_start int32 [S + 1], q [Nq, Hq, D], q_idx [Nq, Hi, di], w [Nq, Hi]),
+    rows in chunk order, one draw per tensor (N(0, 1) rounded to bf16, w from
+    U(0, 1) as for decode queries)."""
+    d, dev = wl.dims, wl.q.device
+    chunk_lens = [int(x) for x in chunk_lens]
+    assert len(chunk_lens) == wl.B
+    assert all(0 <= T <= L for T, L in zip(chunk_lens, wl.seq_lens))
+    row_start = [0]
+    for T in chunk_lens:
+        row_start.append(row_start[-1] + T)
+    Nq = row_start[-1]
+    g = _gen(dev, wl.seed if seed is None else seed, _S_PREFILL)
+    q = torch.randn((Nq, d.Hq, d.D), generator=g, device=dev).to(torch.bfloat16)
+    q_idx = torch.randn((Nq, d.Hi, d.di), generator=g, device=dev).to(torch.bfloat16)
+    w = torch.rand((Nq, d.Hi), generator=g, device=dev)
+    return torch.tensor(row_start, dtype=torch.int32, device=dev), q, q_idx, w
