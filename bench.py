@@ -38,6 +38,7 @@ sys.path.insert(0, ROOT)
 METRIC = "QSA decode seqs/s & attended tokens/s at 256K ctx; HBM GB/s as % of roofline"
 L2_FLUSH_BYTES = 512 << 20
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 
 
 def parse():
@@ -57,6 +58,9 @@ def parse():
     ap.add_argument("--dcp-world", type=int, default=0,
                     help="also time, on this GPU, rank 0's share of a decode-context-parallel "
                          "step over this many ranks (page p on rank p mod W)")
+    ap.add_argument("--prefill-rows", type=int, default=32,
+                    help="also time a sparse prefill of each sequence's this many newest "
+                         "tokens (one query row per token) on the step's cache; 0: skip")
     ap.add_argument("--queries", type=int, default=1,
                     help="decode queries per sequence (multi-query decode: each step appends "
                          "this many tokens per sequence and decodes all of them)")
@@ -72,6 +76,17 @@ def load_peaks():
             d = json.load(f)
         return float(d["hbm_gbs"]), "measured"
     return FALLBACK_HBM_GBS, "fallback"
+
+
+def load_tensor_peak():
+    """Dense bf16 TFLOP/s (burst: a kernel timed alone) and its source."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        if "bf16_tflops" in d:
+            return float(d["bf16_tflops"]), "measured"
+    return FALLBACK_BF16_TFLOPS, "fallback"
 
 
 def profile_traffic(kernel_src: str, summary: str):
@@ -358,6 +373,13 @@ def run_ours(args, rank, world, local_rank):
                            "partials are not timed here"}
         g0.reset()
 
+    # sparse prefill on the same cache: the chunk is each sequence's newest
+    # prefill_rows tokens (appended by the step), one query row per token
+    prefill_res = None
+    if args.prefill_rows > 0 and Qn == 1:
+        prefill_res = time_prefill(args, qsa, wl, dims, cache, si["seq_lens"], k, R, ld, dev,
+                                   capture, timed)
+
     # e2e: host buffers in pinned memory, copies inside the timed region,
     # calls made eagerly through the binding (the user's API)
     e2e = None
@@ -465,12 +487,82 @@ def run_ours(args, rank, world, local_rank):
     }
     if dcp_res is not None:
         res["dcp_emulated"] = dcp_res
+    if prefill_res is not None:
+        res["prefill"] = prefill_res
     graph.reset()
     for g in kgraphs.values():
         g.reset()
     if cpu_sample is not None:
         res["cpu_baseline"] = cpu_baseline(cpu_sample, dims, k, R)
     return res
+
+
+def time_prefill(args, qsa, wl, dims, cache, seq_lens, k, R, ld, dev, capture, timed):
+    """Sparse prefill of every sequence's newest rows: the whole call and each
+    of its four calls in their own graphs (L2 flushed before each launch)."""
+    from synth import prefill_queries
+
+    T = min(args.prefill_rows, min(wl.seq_lens))
+    B = wl.B
+    row_start, q, q_idx, w = prefill_queries(wl, [T] * B)
+    Nq = B * T
+    pb = qsa.alloc_prefill(dims, B, Nq, ld, k, R, device=dev)
+    ws1 = torch.empty(max(16, qsa.qsa_prefill_index_score_workspace_size(dims, B, Nq)),
+                      dtype=torch.uint8, device=dev)
+    ws2 = torch.empty(max(16, qsa.qsa_sparse_decode_workspace_size(dims, Nq, k, R)),
+                      dtype=torch.uint8, device=dev)
+    calls = {
+        "prefill_index_score": lambda: qsa.qsa_prefill_index_score(
+            dims, cache, seq_lens, row_start, q_idx, w, pb.scores, pb.row_len, ws1),
+        "topk_select": lambda: qsa.qsa_topk_select(pb.row_len, pb.scores, k, pb.sel),
+        "prefill_sparse_decode": lambda: qsa.qsa_prefill_sparse_decode(
+            dims, cache, seq_lens, row_start, q, pb.sel, k, R, pb.o_part, pb.lse_part, ws2),
+        "merge": lambda: qsa.qsa_merge(pb.o_part, pb.lse_part, pb.out, pb.lse),
+    }
+    whole = capture(lambda: qsa.sparse_prefill(dims, cache, seq_lens, row_start, q, q_idx, w,
+                                               k, R, pb))
+    graphs = {n: capture(fn) for n, fn in calls.items()}
+    n_rep = max(10, min(args.steps, 100))
+    for _ in range(3):
+        timed(whole)
+    all_ms = statistics.mean(timed(whole) for _ in range(n_rep))
+    us = {}
+    for n, g in graphs.items():
+        for _ in range(3):
+            timed(g)
+        us[n] = 1e3 * statistics.mean(timed(g) for _ in range(n_rep))
+    qsa.qsa_check_device_errors()
+    whole.reset()
+    for g in graphs.values():
+        g.reset()
+    lens = [L - T + i + 1 for L in wl.seq_lens for i in range(T)]
+    flops = 2.0 * dims.Hi * dims.di * sum(ell // 4 for ell in lens)
+    kv = sum(min(4 * k, ell) for ell in lens) * dims.Hkv * dims.D * 2 * 2
+    tpk, tpk_src = load_tensor_peak()
+    hbm, hbm_src = load_peaks()
+    s_tf = flops / (us["prefill_index_score"] * 1e-6) / 1e12
+    d_gb = kv / (us["prefill_sparse_decode"] * 1e-6) / 1e9
+    return {
+        "workload": f"the decode cache; each of the {B} sequences' newest {T} tokens as "
+                    f"query rows ({Nq} rows, context {min(wl.seq_lens) - T + 1}.."
+                    f"{max(wl.seq_lens)}), top-{k}, R={R}",
+        "rows": Nq,
+        "rows_per_s": Nq / (all_ms / 1e3),
+        "us": 1e3 * all_ms,
+        "kernels_us": us,
+        "timing": "qsa_sparse_prefill and each of its calls alone in a CUDA graph, L2 "
+                  "flushed before every launch, CUDA events, mean of %d" % n_rep,
+        "roofline": {
+            "prefill_index_score": {"bound": "tensor", "achieved": s_tf, "peak": tpk,
+                                    "unit": "TFLOP/s", "frac": s_tf / tpk,
+                                    "peak_source": tpk_src, "flops": flops},
+            "prefill_sparse_decode": {"bound": "hbm", "achieved": d_gb, "peak": hbm,
+                                      "unit": "GB/s", "frac": d_gb / hbm,
+                                      "peak_source": hbm_src, "algorithmic_bytes": kv,
+                                      "note": "rows of a sequence share selected blocks "
+                                              "through L2, so frac can exceed 1"},
+        },
+    }
 
 
 def _threads():

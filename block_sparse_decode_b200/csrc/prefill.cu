@@ -34,10 +34,11 @@
 //                        query rows into one shared buffer when the group
 //                        changes (after the MMAs on the old rows completed)
 //                        and issues the MMAs into one of two accumulators
-//              warps 4-7 epilogue: tcgen05.ld of 32 blocks x 256 columns,
-//                        per row the head-weighted ReLU sum, one coalesced
-//                        store per (row, 32 blocks), masked to the blocks
-//                        complete within the row's own prefix.
+//              warps 4-11 epilogue: two warps per TMEM lane quadrant, each
+//                        tcgen05.ld of 32 blocks x 128 columns (half the
+//                        group's rows), per row the head-weighted ReLU sum,
+//                        one coalesced store per (row, 32 blocks), masked to
+//                        the blocks complete within the row's own prefix.
 // Every mbarrier wait is bounded, with the drain of the decode scoring kernel.
 #include <cuda.h>
 
@@ -57,7 +58,8 @@ constexpr int PF_MAX_STAGES = 6;
 constexpr int PF_PROD_WARPS = 3;
 constexpr int PF_MMA_WARP = PF_PROD_WARPS;
 constexpr int PF_EPI0 = PF_PROD_WARPS + 1;
-constexpr int PF_EPI_WARPS = 4;
+constexpr int PF_EPI_WARPS = 8;  // two per TMEM lane quadrant, each half the columns
+constexpr int PF_EPI_COLS = PF_N / 2;
 constexpr int PF_THREADS = 32 * (PF_PROD_WARPS + 1 + PF_EPI_WARPS);
 constexpr int PL_THREADS = 1024;
 
@@ -226,8 +228,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
 
   extern __shared__ unsigned char smem_raw[];
   __shared__ PfCtrl ctl;
-  __shared__ float w_s[PF_EPI_WARPS][PF_N];  // per epilogue warp: the group's head weights
-  __shared__ int nf_s[PF_EPI_WARPS][QG];     // and each row's complete blocks
+  __shared__ float w_s[PF_EPI_WARPS][PF_EPI_COLS];  // per epilogue warp: its rows' head weights
+  __shared__ int nf_s[PF_EPI_WARPS][QG / 2];        // and their complete blocks
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = a.stages;
 
@@ -393,7 +395,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q4 = warp & 3;  // TMEM lane quadrant this warp may access
+    const int e = warp - PF_EPI0;
+    const int q4 = warp & 3;             // TMEM lane quadrant this warp may access
+    const int half = e >> 2;             // columns [half * 128, half * 128 + 128)
+    constexpr int QH = QG / 2;           // group rows per half
     int acc = 0, g = g_first, cur_g = -1, row0 = 0;
     uint32_t aph = 0;
     int done = 0;
@@ -401,12 +406,13 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
       g = pf_advance(a.gtile, g, t0 + ti);
       if (g != cur_g) {
         const int4 gi = __ldg(a.ginfo + g);
-        row0 = gi.y;
-        for (int i = lane; i < PF_N; i += 32) {
+        row0 = gi.y + half * QH;  // first row of this warp's half
+        const int nr = gi.z - half * QH;
+        for (int i = lane; i < PF_EPI_COLS; i += 32) {
           const int qi = i / HI, h = i % HI;
-          w_s[q4][i] = qi < gi.z ? __ldg(a.w + (size_t)(row0 + qi) * HI + h) : 0.f;
+          w_s[e][i] = qi < nr ? __ldg(a.w + (size_t)(row0 + qi) * HI + h) : 0.f;
         }
-        for (int i = lane; i < QG; i += 32) nf_s[q4][i] = i < gi.z ? a.row_len[row0 + i] >> 2 : 0;
+        for (int i = lane; i < QH; i += 32) nf_s[e][i] = i < nr ? a.row_len[row0 + i] >> 2 : 0;
         __syncwarp();
         cur_g = g;
       }
@@ -416,23 +422,27 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       __syncwarp();
       tc_fence_after();
-      const uint32_t taddr = tmem + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(acc * PF_N);
+      const uint32_t taddr = tmem + ((uint32_t)(q4 * 32) << 16) +
+                             (uint32_t)(acc * PF_N + half * PF_EPI_COLS);
       float part = 0.f;
 #pragma unroll
-      for (int c0 = 0; c0 < PF_N; c0 += 32) {
-        float v[32];
-        tc_ld32(taddr + c0, v);
-        if (c0 + 32 == PF_N) {  // every column read: the accumulator may be overwritten
+      for (int c0 = 0; c0 < PF_EPI_COLS; c0 += 64) {
+        uint32_t r0[32], r1[32];
+        tc_ld32_nowait(taddr + c0, r0);
+        tc_ld32_nowait(taddr + c0 + 32, r1);
+        tc_wait_ld();
+        if (c0 + 64 == PF_EPI_COLS) {  // every column read: the accumulator may be overwritten
           tc_fence_before();
           mbar_arrive(tempty0 + 8 * acc);
         }
 #pragma unroll
-        for (int u = 0; u < 32; ++u) {
+        for (int u = 0; u < 64; ++u) {
           const int col = c0 + u;
-          part = fmaf(w_s[q4][col], fmaxf(v[u], 0.f), part);
+          const float v = __uint_as_float(u < 32 ? r0[u] : r1[u - 32]);
+          part = fmaf(w_s[e][col], fmaxf(v, 0.f), part);
           if (col % HI == HI - 1) {
             const int qi = col / HI;
-            if (j < nf_s[q4][qi]) a.scores[(size_t)(row0 + qi) * a.ld + j] = part;
+            if (j < nf_s[e][qi]) a.scores[(size_t)(row0 + qi) * a.ld + j] = part;
             part = 0.f;
           }
         }

@@ -211,12 +211,359 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// One CTA per sequence (rows of a prefill, or any batch whose score rows fit):
+// the upper 16 bits of every key in shared memory (2 bytes per block), two
+// 8-bit radix passes over them, then two over the low 16 bits of only the
+// keys equal to the 16-bit threshold, re-read from global memory (the score
+// row is L2-resident right after scoring). The passes synchronise with block
+// barriers only; a pass over a whole row costs a few microseconds of issue
+// time on one SM, so the kernel makes three: the load (with the first
+// digit's counts), the second digit's counts, and a gather of every key at
+// or above the 16-bit threshold into a list (the k winners plus the keys
+// tied with the threshold on the upper half, a few hundred beyond k). The
+// low-half passes and the index tie-break run on that list, and the winners
+// reach the output in ascending order through a bitmap of the row and one
+// block-wide scan of its word counts. A list that overflows TR_GATHER (a
+// row of largely equal scores) takes the slow path: the tied keys' low
+// halves are listed (or, beyond TR_CAND, re-read from global memory in every
+// pass) and two more passes over the row count and compact the winners;
+// each warp owns a contiguous segment of the row, so that compaction writes
+// ascending indices with one block-wide count exchange.
+constexpr int TR_THREADS = 1024;
+constexpr int TR_WARPS = TR_THREADS / 32;
+constexpr int TR_LOADS = 16;   // score loads per lane issued together
+constexpr int TR_CAND = 2048;    // keys tied on the upper half kept as a list (slow path)
+constexpr int TR_GATHER = 4096;  // keys at or above the upper-half threshold (fast path)
+
+__host__ __device__ inline size_t tr_k16_bytes(int ld) { return ((size_t)ld * 2 + 15) / 16 * 16; }
+__host__ __device__ inline size_t tr_bit_bytes(int ld) {
+  return (((size_t)ld + 31) / 32 * 4 + 15) / 16 * 16;
+}
+
+// Digit with cum >= need > cum - count over 256 descending bins, chosen by
+// the CTA's first 256 threads from the per-warp histograms; every thread
+// returns (digit, keys above it, keys in it) through pick.
+__device__ __forceinline__ void tr_pick(unsigned (*whist)[256], unsigned *wtot, int *pick,
+                                        int need) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  unsigned c = 0u, cum = 0u;
+  if (tid < 256) {
+#pragma unroll 8
+    for (int w = 0; w < TR_WARPS; ++w) c += whist[w][255 - tid];
+    cum = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned y = __shfl_up_sync(0xffffffffu, cum, o);
+      if (lane >= o) cum += y;
+    }
+    if (lane == 31) wtot[warp] = cum;
+  }
+  __syncthreads();
+  if (tid < 256) {
+    for (int w = 0; w < warp; ++w) cum += wtot[w];
+    if (cum >= (unsigned)need && cum - c < (unsigned)need) {
+      pick[0] = 255 - tid;
+      pick[1] = (int)(cum - c);
+      pick[2] = (int)c;
+    }
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(TR_THREADS, 1) topk_row_kernel(TopkArgs a) {
+  // dynamic: [upper key halves of the row][bitmap of the row][gather list:
+  // indices, keys] (the slow path's tied-key list reuses the indices)
+  extern __shared__ __align__(16) unsigned char tr_dyn[];
+  __shared__ unsigned whist[TR_WARPS][256];     // per-warp digit counts
+  __shared__ unsigned wtot[8];
+  __shared__ int pick[3];
+  __shared__ unsigned wgt[TR_WARPS], weq[TR_WARPS];
+  __shared__ int ncand;
+  const int b = blockIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const unsigned lower = (1u << lane) - 1u;
+  const int L = a.seq_lens[b];
+  const int nb = L < 0 ? 0 : (L + 3) >> 2;
+  int32_t *out = a.sel + (size_t)b * a.k;
+  uint16_t *k16 = reinterpret_cast<uint16_t *>(tr_dyn);
+  uint32_t *cbit = reinterpret_cast<uint32_t *>(tr_dyn + tr_k16_bytes(a.ld));
+  int *gidx = reinterpret_cast<int *>(tr_dyn + tr_k16_bytes(a.ld) + tr_bit_bytes(a.ld));
+  uint32_t *gkey = reinterpret_cast<uint32_t *>(gidx + TR_GATHER);
+  int *clist = gidx;
+  pdl_wait();  // the scores come from the kernel before this one
+  if (L < 0 || nb > a.ld) {
+    if (tid == 0) raise_err(a.err, ERR_LEN);
+    for (int i = tid; i < a.k; i += TR_THREADS) out[i] = -1;
+    return;
+  }
+  if (nb <= a.k) {
+    for (int i = tid; i < a.k; i += TR_THREADS) out[i] = i < nb ? i : -1;
+    return;
+  }
+  const float *src = a.scores + (size_t)b * a.ld;
+  // warp segments: whole 32-key rounds, so every ballot sees a full warp
+  const int seg = ((nb + TR_WARPS - 1) / TR_WARPS + 31) & ~31;
+  const int s0 = min(nb, warp * seg), s1 = min(nb, s0 + seg);
+  for (int i = lane; i < 256; i += 32) whist[warp][i] = 0u;
+  __syncwarp();
+  // load: keys' upper halves to shared memory, first-digit counts
+  for (int i0 = s0; i0 < s1; i0 += 32 * TR_LOADS) {
+    float v[TR_LOADS];
+#pragma unroll
+    for (int u = 0; u < TR_LOADS; ++u) {
+      const int i = i0 + 32 * u + lane;
+      v[u] = i < s1 ? src[i] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < TR_LOADS; ++u) {
+      const int i = i0 + 32 * u + lane;
+      const bool valid = i < s1;
+      const uint32_t key = score_key(v[u]), d = key >> 24;
+      if (valid) k16[i] = (uint16_t)(key >> 16);
+      // the top digits of a warp's keys mostly span a few values: count each
+      // with a ballot instead of 32 same-address atomics
+      const uint32_t dlo = __reduce_min_sync(0xffffffffu, valid ? d : 255u);
+      const uint32_t dhi = __reduce_max_sync(0xffffffffu, valid ? d : 0u);
+      if (dlo <= dhi && dhi - dlo < 4u) {
+        for (uint32_t dd = dlo; dd <= dhi; ++dd) {
+          const unsigned m = __ballot_sync(0xffffffffu, valid && d == dd);
+          if (lane == 0 && m != 0u) atomicAdd(&whist[warp][dd], (unsigned)__popc(m));
+        }
+      } else if (valid) {
+        atomicAdd(&whist[warp][d], 1u);
+      }
+    }
+  }
+  __syncthreads();
+  int need = a.k;
+  tr_pick(whist, wtot, pick, need);
+  const uint32_t d1 = (uint32_t)pick[0];
+  need -= pick[1];
+  uint32_t prefix = d1 << 24, mask = 0xFF000000u;
+  bool done = pick[2] == need;
+  if (!done) {  // second digit: bits 23..16
+    for (int i = lane; i < 256; i += 32) whist[warp][i] = 0u;
+    __syncwarp();
+    for (int i = s0 + lane; i < s1; i += 32) {
+      const uint32_t h = k16[i];
+      if ((h >> 8) == d1) atomicAdd(&whist[warp][h & 255u], 1u);
+    }
+    __syncthreads();
+    tr_pick(whist, wtot, pick, need);
+    prefix |= (uint32_t)pick[0] << 16;
+    mask = 0xFFFF0000u;
+    need -= pick[1];
+    done = pick[2] == need;
+  }
+  const uint32_t t16 = prefix >> 16;
+  {
+    // ---- fast path: the keys whose upper bits (under the mask) are at or
+    // above the threshold's: every winner, plus the ties still open
+    const uint32_t pm = prefix & 0xFFFF0000u, mu = mask & 0xFFFF0000u;
+    const int nw = (nb + 31) / 32;
+    for (int i = tid; i < nw; i += TR_THREADS) cbit[i] = 0u;
+    if (tid == 0) ncand = 0;
+    __syncthreads();
+    for (int base = s0; base < s1; base += 32) {
+      const int i = base + lane;
+      const bool c = i < s1 && (((uint32_t)k16[i] << 16) & mu) >= pm;
+      const unsigned m = __ballot_sync(0xffffffffu, c);
+      if (m != 0u) {
+        int off = 0;
+        if (lane == 0) off = atomicAdd(&ncand, __popc(m));
+        off = __shfl_sync(0xffffffffu, off, 0);
+        const int p = off + __popc(m & lower);
+        if (c && p < TR_GATHER) gidx[p] = i;
+      }
+    }
+    __syncthreads();
+    const int ng = ncand;
+    if (ng <= TR_GATHER) {
+      const bool open = !done;  // ties on the upper half still to resolve
+      if (open) {
+        for (int j = tid; j < ng; j += TR_THREADS) {
+          const int i = gidx[j];
+          gkey[j] = k16[i] == t16 ? score_key(src[i]) : 0xFFFFFFFFu;
+        }
+        __syncthreads();
+        for (int pass = 0; pass < 2 && !done; ++pass) {  // bits 15..8, then 7..0
+          const int shift = 8 - 8 * pass;
+          for (int i = lane; i < 256; i += 32) whist[warp][i] = 0u;
+          __syncwarp();
+          for (int j = tid; j < ng; j += TR_THREADS) {
+            if (k16[gidx[j]] != t16) continue;
+            const uint32_t key = gkey[j];
+            if ((key & mask) == prefix) atomicAdd(&whist[warp][(key >> shift) & 255u], 1u);
+          }
+          __syncthreads();
+          tr_pick(whist, wtot, pick, need);
+          prefix |= (uint32_t)pick[0] << shift;
+          mask |= 255u << shift;
+          need -= pick[1];
+          done = pick[2] == need;
+        }
+      }
+      pdl_trigger();
+      // winners: every listed key above the threshold under the final mask,
+      // and the first `need` (by index) equal to it
+      auto state = [&](int j) -> int {  // +1 above, 0 equal, -1 below
+        if (!open || k16[gidx[j]] != t16) return 1;
+        const uint32_t m = gkey[j] & mask;
+        return m > prefix ? 1 : (m == prefix ? 0 : -1);
+      };
+      // the equal keys' indices listed once (the per-warp histograms are
+      // free now), each ranked against that short list only
+      int *eql = reinterpret_cast<int *>(&whist[0][0]);
+      if (tid == 0) ncand = 0;
+      __syncthreads();
+      for (int j = tid; j < ng; j += TR_THREADS) {
+        const int st = state(j);
+        if (st > 0) atomicOr(&cbit[gidx[j] >> 5], 1u << (gidx[j] & 31));
+        if (st == 0) eql[atomicAdd(&ncand, 1)] = gidx[j];
+      }
+      __syncthreads();
+      const int ne = ncand;
+      for (int e = tid; e < ne; e += TR_THREADS) {
+        const int i = eql[e];
+        int before = 0;  // equal keys with a lower index
+        for (int f = 0; f < ne; ++f) before += eql[f] < i ? 1 : 0;
+        if (before < need) atomicOr(&cbit[i >> 5], 1u << (i & 31));
+      }
+      __syncthreads();
+      // the bitmap's words in contiguous runs per thread, one scan of counts
+      const int wpt = (nw + TR_THREADS - 1) / TR_THREADS;
+      const int w0 = min(nw, tid * wpt), w1 = min(nw, w0 + wpt);
+      unsigned cnt = 0u;
+      for (int w = w0; w < w1; ++w) cnt += __popc(cbit[w]);
+      unsigned incl = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (lane == 31) wgt[warp] = incl;
+      __syncthreads();
+      unsigned pos = incl - cnt;
+      for (int w = 0; w < warp; ++w) pos += wgt[w];
+      for (int w = w0; w < w1; ++w) {
+        unsigned bits = cbit[w];
+        while (bits != 0u) {
+          const int bit = __ffs(bits) - 1;
+          if (pos < (unsigned)a.k) out[pos] = 32 * w + bit;
+          ++pos;
+          bits &= bits - 1u;
+        }
+      }
+      return;
+    }
+  }
+  // ---- slow path (more than TR_GATHER keys at or above the upper threshold)
+  bool have_low = false;  // the tied keys' low halves are in k16 (marked in cbit)
+  int nc = 0;
+  if (!done) {
+    for (int i = tid; i < (nb + 31) / 32; i += TR_THREADS) cbit[i] = 0u;
+    if (tid == 0) ncand = 0;
+    __syncthreads();
+    for (int base = s0; base < s1; base += 32) {
+      const int i = base + lane;
+      const bool c = i < s1 && k16[i] == t16;
+      const unsigned m = __ballot_sync(0xffffffffu, c);
+      if (m != 0u) {
+        int off = 0;
+        if (lane == 0) off = atomicAdd(&ncand, __popc(m));
+        off = __shfl_sync(0xffffffffu, off, 0);
+        const int p = off + __popc(m & lower);
+        if (c && p < TR_CAND) clist[p] = i;
+      }
+    }
+    __syncthreads();
+    nc = ncand;
+    if (nc <= TR_CAND) {
+      for (int j = tid; j < nc; j += TR_THREADS) {
+        const int i = clist[j];
+        k16[i] = (uint16_t)(score_key(src[i]) & 0xFFFFu);
+        atomicOr(&cbit[i >> 5], 1u << (i & 31));
+      }
+      have_low = true;
+    }
+    __syncthreads();
+  }
+  for (int pass = 0; pass < 2 && !done; ++pass) {  // bits 15..8, then 7..0
+    const int shift = 8 - 8 * pass;
+    for (int i = lane; i < 256; i += 32) whist[warp][i] = 0u;
+    __syncwarp();
+    if (have_low) {
+      for (int j = tid; j < nc; j += TR_THREADS) {
+        const uint32_t key = (t16 << 16) | k16[clist[j]];
+        if ((key & mask) == prefix) atomicAdd(&whist[warp][(key >> shift) & 255u], 1u);
+      }
+    } else {
+      for (int i = s0 + lane; i < s1; i += 32) {
+        if (k16[i] == t16) {
+          const uint32_t key = score_key(src[i]);
+          if ((key & mask) == prefix) atomicAdd(&whist[warp][(key >> shift) & 255u], 1u);
+        }
+      }
+    }
+    __syncthreads();
+    tr_pick(whist, wtot, pick, need);
+    prefix |= (uint32_t)pick[0] << shift;
+    mask |= 255u << shift;
+    need -= pick[1];
+    done = pick[2] == need;
+  }
+  pdl_trigger();
+  const int take_eq = need;
+  // (masked key vs prefix) of block i: +1 above, 0 equal, -1 below; the
+  // low half is read from global memory only when the upper halves tie
+  auto cmp = [&](int i) -> int {
+    if (have_low && ((cbit[i >> 5] >> (i & 31)) & 1u)) {
+      const uint32_t m = ((t16 << 16) | k16[i]) & mask;
+      return m > prefix ? 1 : (m == prefix ? 0 : -1);
+    }
+    const uint32_t hm = ((uint32_t)k16[i] << 16) & mask, pm = prefix & 0xFFFF0000u;
+    if (hm != pm) return hm > pm ? 1 : -1;
+    if ((mask & 0xFFFFu) == 0u) return 0;
+    const uint32_t m = score_key(src[i]) & mask;
+    return m > prefix ? 1 : (m == prefix ? 0 : -1);
+  };
+  unsigned gt = 0u, eq = 0u;
+  for (int base = s0; base < s1; base += 32) {
+    const int i = base + lane;
+    const int c = i < s1 ? cmp(i) : -1;
+    gt += __popc(__ballot_sync(0xffffffffu, c > 0));
+    eq += __popc(__ballot_sync(0xffffffffu, c == 0));
+  }
+  if (lane == 0) { wgt[warp] = gt; weq[warp] = eq; }
+  __syncthreads();
+  unsigned run_gt = 0u, run_eq = 0u;
+  for (int w = 0; w < warp; ++w) { run_gt += wgt[w]; run_eq += weq[w]; }
+  for (int base = s0; base < s1; base += 32) {
+    const int i = base + lane;
+    const int c = i < s1 ? cmp(i) : -1;
+    const unsigned bg = __ballot_sync(0xffffffffu, c > 0);
+    const unsigned be = __ballot_sync(0xffffffffu, c == 0);
+    const unsigned gb = run_gt + __popc(bg & lower), eb = run_eq + __popc(be & lower);
+    const unsigned pos = c > 0 ? gb + min(eb, (unsigned)take_eq) : gb + eb;
+    if ((c > 0 || (c == 0 && eb < (unsigned)take_eq)) && pos < (unsigned)a.k) out[pos] = i;
+    run_gt += __popc(bg);
+    run_eq += __popc(be);
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_topk(int B, const int32_t *seq_lens, const float *scores, int ld, int k,
                         int32_t *sel, unsigned *err, cudaStream_t st) {
   if (B == 0) return cudaSuccess;
   TopkArgs a{scores, seq_lens, sel, ld, k, err};
+  if (B >= TOPK_ROW_MIN_B && ld <= TOPK_ROW_MAX_KEYS) {
+    const size_t smem = tr_k16_bytes(ld) + tr_bit_bytes(ld) + (size_t)TR_GATHER * 8;
+    cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void *>(topk_row_kernel), smem);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(topk_row_kernel, B, TR_THREADS, smem, st, a);
+  }
   const int per_cta = (ld + TOPK_CLUSTER - 1) / TOPK_CLUSTER;
   const size_t smem = (size_t)per_cta * 4;
   cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void *>(topk_kernel), smem);

@@ -114,11 +114,13 @@ def _topk_gpu(scores_np, k, lens=None):
     return sel.cpu().numpy()
 
 
+@pytest.mark.parametrize("rows", [6, 66])  # clusters per row; one CTA per row
 @pytest.mark.parametrize("case", ["random", "ties", "allzero", "negzero", "negative", "few",
                                   "heavy"])
-def test_topk_exact(case):
+def test_topk_exact(case, rows):
     g = np.random.default_rng(sum(map(ord, case)))
-    B, ld, k = 6, 70001, 512
+    # one CTA per row takes rows of at most 65,536 blocks
+    B, ld, k = 6, (70001 if rows <= 6 else 65536), 512
     if case == "random":
         s = g.standard_normal((B, ld)).astype(np.float32) ** 2
     elif case == "ties":
@@ -138,6 +140,11 @@ def test_topk_exact(case):
     lens = [4 * ld - 3, 4 * ld, 2049, 2048, 4 * 513, 1]
     if case == "few":
         lens = [5, 4 * 511 + 1, 4 * 512, 4 * 512 + 1, 4 * 65536, 4 * 70001]
+    lens = [min(x, 4 * ld) for x in lens]
+    if rows > B:  # the same rows again, each with a shifted copy of its scores
+        s = np.concatenate([np.roll(s, 7 * r, axis=1) for r in range(rows // B)], axis=0)
+        lens = lens * (rows // B)
+        B = rows
     got = _topk_gpu(s, k, lens)
     for b in range(B):
         nb = (lens[b] + 3) // 4
@@ -145,15 +152,28 @@ def test_topk_exact(case):
         assert np.array_equal(got[b], ref), f"{case} b={b} nb={nb}"
 
 
+@pytest.mark.parametrize("rows", [3, 66])
 @pytest.mark.parametrize("k", [1, 2, 255, 256, 1024, 4096])
-def test_topk_k_sweep(k):
+def test_topk_k_sweep(k, rows):
     g = np.random.default_rng(k)
-    s = (g.integers(0, 1000, (3, 30000)) * 0.25).astype(np.float32)
-    lens = [4 * 30000, 4 * 4097 - 2, 4 * k + 4]
+    s = (g.integers(0, 1000, (rows, 30000)) * 0.25).astype(np.float32)
+    lens = ([4 * 30000, 4 * 4097 - 2, 4 * k + 4] * rows)[:rows]
     got = _topk_gpu(s, k, lens)
-    for b in range(3):
+    for b in range(rows):
         nb = (lens[b] + 3) // 4
         assert np.array_equal(got[b], oracle.topk_blocks(s[b, :nb].astype(np.float64), k))
+
+
+def test_topk_many_rows_long_score_rows_use_clusters():
+    # rows longer than the one-CTA kernel's shared-memory key array
+    g = np.random.default_rng(5)
+    B, ld, k = 64, 100003, 512
+    s = g.standard_normal((B, ld)).astype(np.float32) ** 2
+    lens = [4 * ld - 1 - 4 * b for b in range(B)]
+    got = _topk_gpu(s, k, lens)
+    for b in range(0, B, 9):
+        nb = (lens[b] + 3) // 4
+        assert np.array_equal(got[b], oracle.topk_blocks(s[b, :nb].astype(np.float64), k)), b
 
 
 # ------------------------------------------------------------ merge alone
