@@ -34,11 +34,14 @@
 //                        query rows into one shared buffer when the group
 //                        changes (after the MMAs on the old rows completed)
 //                        and issues the MMAs into one of two accumulators
-//              warps 4-11 epilogue: two warps per TMEM lane quadrant, each
-//                        tcgen05.ld of 32 blocks x 128 columns (half the
-//                        group's rows), per row the head-weighted ReLU sum,
-//                        one coalesced store per (row, 32 blocks), masked to
-//                        the blocks complete within the row's own prefix.
+//              warps 4-19 epilogue: four warps per TMEM lane quadrant, each
+//                        tcgen05.ld of 32 blocks x 64 columns (a quarter of
+//                        the group's rows), per row the head-weighted ReLU
+//                        sum, one coalesced store per (row, 32 blocks),
+//                        masked to the blocks complete within the row's own
+//                        prefix. (With fewer warps the epilogue's TMEM-load
+//                        and arithmetic latencies, not the tensor pipe, set
+//                        the tile time.)
 // Every mbarrier wait is bounded, with the drain of the decode scoring kernel.
 #include <cuda.h>
 
@@ -58,8 +61,9 @@ constexpr int PF_MAX_STAGES = 6;
 constexpr int PF_PROD_WARPS = 3;
 constexpr int PF_MMA_WARP = PF_PROD_WARPS;
 constexpr int PF_EPI0 = PF_PROD_WARPS + 1;
-constexpr int PF_EPI_WARPS = 8;  // two per TMEM lane quadrant, each half the columns
-constexpr int PF_EPI_COLS = PF_N / 2;
+constexpr int PF_EPI_WARPS = 16;  // four per TMEM lane quadrant, each a quarter of the columns
+constexpr int PF_EPI_PARTS = PF_EPI_WARPS / 4;
+constexpr int PF_EPI_COLS = PF_N / PF_EPI_PARTS;
 constexpr int PF_THREADS = 32 * (PF_PROD_WARPS + 1 + PF_EPI_WARPS);
 constexpr int PL_THREADS = 1024;
 
@@ -229,7 +233,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
   extern __shared__ unsigned char smem_raw[];
   __shared__ PfCtrl ctl;
   __shared__ float w_s[PF_EPI_WARPS][PF_EPI_COLS];  // per epilogue warp: its rows' head weights
-  __shared__ int nf_s[PF_EPI_WARPS][QG / 2];        // and their complete blocks
+  __shared__ int nf_s[PF_EPI_WARPS][QG / PF_EPI_PARTS];  // and their complete blocks
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = a.stages;
 
@@ -397,8 +401,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     // ------------------------------------------------------------ epilogue
     const int e = warp - PF_EPI0;
     const int q4 = warp & 3;             // TMEM lane quadrant this warp may access
-    const int half = e >> 2;             // columns [half * 128, half * 128 + 128)
-    constexpr int QH = QG / 2;           // group rows per half
+    const int half = e >> 2;             // columns [half * 64, half * 64 + 64)
+    constexpr int QH = QG / PF_EPI_PARTS;  // group rows per warp
     int acc = 0, g = g_first, cur_g = -1, row0 = 0;
     uint32_t aph = 0;
     int done = 0;
@@ -426,19 +430,18 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                              (uint32_t)(acc * PF_N + half * PF_EPI_COLS);
       float part = 0.f;
 #pragma unroll
-      for (int c0 = 0; c0 < PF_EPI_COLS; c0 += 64) {
-        uint32_t r0[32], r1[32];
+      for (int c0 = 0; c0 < PF_EPI_COLS; c0 += 32) {
+        uint32_t r0[32];
         tc_ld32_nowait(taddr + c0, r0);
-        tc_ld32_nowait(taddr + c0 + 32, r1);
         tc_wait_ld();
-        if (c0 + 64 == PF_EPI_COLS) {  // every column read: the accumulator may be overwritten
+        if (c0 + 32 == PF_EPI_COLS) {  // every column read: the accumulator may be overwritten
           tc_fence_before();
           mbar_arrive(tempty0 + 8 * acc);
         }
 #pragma unroll
-        for (int u = 0; u < 64; ++u) {
+        for (int u = 0; u < 32; ++u) {
           const int col = c0 + u;
-          const float v = __uint_as_float(u < 32 ? r0[u] : r1[u - 32]);
+          const float v = __uint_as_float(r0[u]);
           part = fmaf(w_s[e][col], fmaxf(v, 0.f), part);
           if (col % HI == HI - 1) {
             const int qi = col / HI;
