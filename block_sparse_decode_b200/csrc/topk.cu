@@ -318,20 +318,10 @@ __global__ void __launch_bounds__(TR_THREADS, 1) topk_row_kernel(TopkArgs a) {
 #pragma unroll
     for (int u = 0; u < TR_LOADS; ++u) {
       const int i = i0 + 32 * u + lane;
-      const bool valid = i < s1;
-      const uint32_t key = score_key(v[u]), d = key >> 24;
-      if (valid) k16[i] = (uint16_t)(key >> 16);
-      // the top digits of a warp's keys mostly span a few values: count each
-      // with a ballot instead of 32 same-address atomics
-      const uint32_t dlo = __reduce_min_sync(0xffffffffu, valid ? d : 255u);
-      const uint32_t dhi = __reduce_max_sync(0xffffffffu, valid ? d : 0u);
-      if (dlo <= dhi && dhi - dlo < 4u) {
-        for (uint32_t dd = dlo; dd <= dhi; ++dd) {
-          const unsigned m = __ballot_sync(0xffffffffu, valid && d == dd);
-          if (lane == 0 && m != 0u) atomicAdd(&whist[warp][dd], (unsigned)__popc(m));
-        }
-      } else if (valid) {
-        atomicAdd(&whist[warp][d], 1u);
+      if (i < s1) {
+        const uint32_t key = score_key(v[u]);
+        k16[i] = (uint16_t)(key >> 16);
+        atomicAdd(&whist[warp][key >> 24], 1u);
       }
     }
   }
@@ -345,9 +335,13 @@ __global__ void __launch_bounds__(TR_THREADS, 1) topk_row_kernel(TopkArgs a) {
   if (!done) {  // second digit: bits 23..16
     for (int i = lane; i < 256; i += 32) whist[warp][i] = 0u;
     __syncwarp();
-    for (int i = s0 + lane; i < s1; i += 32) {
-      const uint32_t h = k16[i];
-      if ((h >> 8) == d1) atomicAdd(&whist[warp][h & 255u], 1u);
+    // two keys per lane per round (s0 is even; a read past s1 stays inside
+    // the shared buffer and is ignored)
+    for (int i = s0 + 2 * lane; i < s1; i += 64) {
+      const uint32_t x = *reinterpret_cast<const uint32_t *>(k16 + i);
+      const uint32_t h0 = x & 0xFFFFu, h1 = x >> 16;
+      if ((h0 >> 8) == d1) atomicAdd(&whist[warp][h0 & 255u], 1u);
+      if (i + 1 < s1 && (h1 >> 8) == d1) atomicAdd(&whist[warp][h1 & 255u], 1u);
     }
     __syncthreads();
     tr_pick(whist, wtot, pick, need);
@@ -365,16 +359,19 @@ __global__ void __launch_bounds__(TR_THREADS, 1) topk_row_kernel(TopkArgs a) {
     for (int i = tid; i < nw; i += TR_THREADS) cbit[i] = 0u;
     if (tid == 0) ncand = 0;
     __syncthreads();
-    for (int base = s0; base < s1; base += 32) {
-      const int i = base + lane;
-      const bool c = i < s1 && (((uint32_t)k16[i] << 16) & mu) >= pm;
-      const unsigned m = __ballot_sync(0xffffffffu, c);
-      if (m != 0u) {
+    for (int base = s0; base < s1; base += 64) {  // two keys per lane per round
+      const int i = base + 2 * lane;
+      const uint32_t x = i < s1 ? *reinterpret_cast<const uint32_t *>(k16 + i) : 0u;
+      const bool c0 = i < s1 && ((x << 16) & mu) >= pm;
+      const bool c1 = i + 1 < s1 && ((x & 0xFFFF0000u) & mu) >= pm;
+      const unsigned m0 = __ballot_sync(0xffffffffu, c0), m1 = __ballot_sync(0xffffffffu, c1);
+      if ((m0 | m1) != 0u) {
         int off = 0;
-        if (lane == 0) off = atomicAdd(&ncand, __popc(m));
+        if (lane == 0) off = atomicAdd(&ncand, __popc(m0) + __popc(m1));
         off = __shfl_sync(0xffffffffu, off, 0);
-        const int p = off + __popc(m & lower);
-        if (c && p < TR_GATHER) gidx[p] = i;
+        const int p0 = off + __popc(m0 & lower), p1 = off + __popc(m0) + __popc(m1 & lower);
+        if (c0 && p0 < TR_GATHER) gidx[p0] = i;
+        if (c1 && p1 < TR_GATHER) gidx[p1] = i + 1;
       }
     }
     __syncthreads();

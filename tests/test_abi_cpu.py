@@ -52,6 +52,30 @@ def test_version_and_workspace_sizes(L):
             B * (ncb + R - 1) * 32 * 129 * 4 + B * R * 8, (B, k, R)
 
 
+def test_prefill_workspace_sizes(L):
+    # plan scratch: 16-byte header, each row's sequence, the groups' tile
+    # prefix and their {sequence, first row, rows, blocks} (16 bytes), for at
+    # most S + ceil(Nq / QG) groups of QG = 256 / Hi rows
+    def r16(x):
+        return (x + 15) // 16 * 16
+    for Hi, di in ((16, 128), (4, 64), (8, 128), (32, 64)):
+        d = qsa.QsaDims(32, 4, 128, Hi, di, 64, 0.088)
+        QG = 256 // Hi
+        for S, Nq in ((8, 256), (2, 73), (1, 1), (3, 130)):
+            gmax = S + (Nq + QG - 1) // QG
+            plan = 16 + r16(4 * Nq) + r16(4 * (gmax + 1)) + 16 * gmax
+            assert qsa.qsa_prefill_index_score_workspace_size(d, S, Nq) == plan, (Hi, S, Nq)
+            for k, R in ((512, 4), (64, 1)):
+                total = (plan + 255) // 256 * 256 + \
+                    qsa.qsa_sparse_decode_workspace_size(d, Nq, k, R)
+                assert qsa.qsa_sparse_prefill_workspace_size(d, S, Nq, k, R) == total
+    # indexer heads that do not tile the 256-column MMA are not supported
+    assert qsa.qsa_prefill_index_score_workspace_size(qsa.QsaDims(32, 4, 128, 12, 128, 64,
+                                                                  0.1), 1, 8) == 0
+    assert qsa.qsa_sparse_prefill_workspace_size(qsa.QsaDims(32, 4, 128, 16, 128, 48, 0.1),
+                                                 1, 8, 64, 1) == 0
+
+
 def _status(fn, *args):
     return fn(*args)
 
