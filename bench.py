@@ -274,9 +274,20 @@ def run_ours(args, rank, world, local_rank):
                                        buf.lse_part.view(R, B * Qn, dims.Hq), buf.out, buf.lse),
     }
 
-    def step():
-        for fn in calls.values():
-            fn()
+    if Qn == 1:
+        # the user's one-call step (append, score, top-k, decode with the
+        # merge fused into its last kernel)
+        step_buf = qsa.StepBuffers(scores=buf.scores, sel=buf.sel, o_part=buf.o_part,
+                                   lse_part=buf.lse_part, out=buf.out, lse=buf.lse, ws=buf.ws)
+        step_app = (si["tok_seq"], si["tok_pos"], si["k_new"], si["v_new"], si["kidx_new"])
+
+        def step():
+            qsa.decode_step(dims, cache, si["seq_lens"], si["q"], si["q_idx"], si["w"], k, R,
+                            step_buf, append=step_app)
+    else:
+        def step():
+            for fn in calls.values():
+                fn()
 
     with torch.cuda.stream(stream):
         for _ in range(3):  # eager warm-up (module load, attributes)
@@ -441,7 +452,10 @@ def run_ours(args, rank, world, local_rank):
     nhg = (dims.Hkv + 3) // 4
     ntmax = (k + 3) // 4 + R - 1
     ncb = max(1, min(296 // (B * nhg), ntmax), -(-ntmax // 256))
-    launches = 4 + ((Qn + 1) // 2) * (2 if ncb > 1 else 1)
+    if Qn == 1:  # append, score, top-k, decode, then the combine (merging) or the merge
+        launches = 5
+    else:
+        launches = 4 + ((Qn + 1) // 2) * (2 if ncb > 1 else 1)
     res = {
         "metric": METRIC,
         "value": job_rate(world, B, ms_per_step),
@@ -462,7 +476,10 @@ def run_ours(args, rank, world, local_rank):
                                   if Qn > 1 else ""),
                    "batch": B, "context": max(wl.seq_lens), "k": k, "R": R, "queries": Qn,
                    "l2": "flushed before every timed step (512 MiB write, then 512 MiB read)",
-                   "step": "CUDA graph of append+score+topk+decode+merge",
+                   "step": ("CUDA graph of one qsa_decode_step call (append, score, top-k, "
+                            "decode with the merge fused into its combine kernel)"
+                            if Qn == 1 else
+                            "CUDA graph of append+score+topk+decode (per query pair)+merge"),
                    "parallelism": f"replicas x{world}"},
         "attended_tokens_per_s": job_rate(world, attended, ms_per_step),
         "query_tokens_per_s": job_rate(world, B * Qn, ms_per_step),

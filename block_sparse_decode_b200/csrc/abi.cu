@@ -352,11 +352,37 @@ qsa_status qsa_decode_step(const qsa_dims *dims, const qsa_cache *cache, int32_t
     st = qsa_index_score(dims, cache, B, seq_lens, q_idx, w, scores, ld_scores, stream);
   if (st == QSA_OK)
     st = qsa_topk_select(B, seq_lens, scores, ld_scores, k, sel, nullptr, 0, stream);
-  if (st == QSA_OK)
-    st = qsa_sparse_decode(dims, cache, B, seq_lens, q, sel, k, R, o_part, lse_part, ws, ws_bytes,
-                           stream);
-  if (st == QSA_OK && dims != nullptr)
-    st = qsa_merge(R, B, dims->Hq, dims->D, o_part, lse_part, out, out_is_bf16, lse_out, stream);
+  if (st == QSA_OK) {
+    // qsa_sparse_decode and qsa_merge with the merge fused into the decode's
+    // combine kernel (same arithmetic as qsa_merge); both calls' checks apply
+    try {
+      QSA_TRY(check_dims(dims));
+      QSA_TRY(check_cache(cache, true, false));
+      if (B < 0 || B > 65535) return fail(QSA_ERR_INVALID_ARG, "B=%d outside [0, 65535]", B);
+      if (B > cache->num_seqs)
+        return fail(QSA_ERR_INVALID_ARG, "B=%d exceeds block_table rows %d", B, cache->num_seqs);
+      if (k < 1 || k > 4096) return fail(QSA_ERR_UNSUPPORTED, "k=%d outside [1, 4096]", k);
+      if (R < 1 || R > 64) return fail(QSA_ERR_UNSUPPORTED, "R=%d outside [1, 64]", R);
+      if (B == 0) return ok();
+      if (seq_lens == nullptr || q == nullptr || sel == nullptr || o_part == nullptr ||
+          lse_part == nullptr || ws == nullptr || out == nullptr)
+        return fail(QSA_ERR_INVALID_ARG, "an argument array is NULL");
+      if (!aligned16(q) || !aligned16(o_part) || !aligned16(ws) ||
+          (reinterpret_cast<uintptr_t>(out) & 7u) != 0)
+        return fail(QSA_ERR_INVALID_ARG, "q / o_part / ws not 16-byte or out not 8-byte aligned");
+      const size_t need = decode_ws_bytes(*dims, B, 1, k, R);
+      if (ws_bytes < need)
+        return fail(QSA_ERR_INVALID_ARG, "workspace %zu bytes < %zu needed", ws_bytes, need);
+      QSA_ERRWORD(err);
+      st = cuda_status(launch_sparse_decode(*dims, *cache, B, 1, seq_lens, q, sel, k, R, o_part,
+                                            lse_part, ws, err,
+                                            reinterpret_cast<cudaStream_t>(stream), nullptr, 0,
+                                            out, out_is_bf16, lse_out),
+                       "qsa_decode_step decode + merge launch");
+    } catch (...) {
+      return fail(QSA_ERR_CUDA, "qsa_decode_step: internal exception");
+    }
+  }
   return st;
 }
 

@@ -61,11 +61,15 @@ cudaError_t launch_topk(int B, const int32_t *seq_lens, const float *scores, int
 size_t decode_ws_bytes(const qsa_dims &d, int B, int Qn, int k, int R);
 // row_start != nullptr: B prefill rows of S chunks (sequence s holds rows
 // [row_start[s], row_start[s+1]), seq_lens[s] counts its chunk), Qn = 1.
+// m_out != nullptr (Qn = 1): the R partials are also merged into m_out
+// [B, Hq, D] (bf16 if m_bf16) and m_lse [B, Hq], by the combine kernel's last
+// CTA per row group (or the merge kernel when no sequence is split).
 cudaError_t launch_sparse_decode(const qsa_dims &d, const qsa_cache &c, int B, int Qn,
                                  const int32_t *seq_lens, const void *q, const int32_t *sel,
                                  int k, int R, float *o_part, float *lse_part, void *ws,
                                  unsigned *err, cudaStream_t st,
-                                 const int32_t *row_start = nullptr, int S = 0);
+                                 const int32_t *row_start = nullptr, int S = 0,
+                                 void *m_out = nullptr, int m_bf16 = 0, float *m_lse = nullptr);
 
 cudaError_t launch_select_owned(const int32_t *sel, int B, int k, int P, int W, int r,
                                 int32_t *out, cudaStream_t st);

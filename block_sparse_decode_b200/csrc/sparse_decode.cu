@@ -41,6 +41,7 @@
 // (each selected token's K and V rows read once).
 #include "common.cuh"
 #include "launch.h"
+#include "merge_row.cuh"
 
 namespace qsa {
 namespace {
@@ -73,6 +74,13 @@ struct DecodeArgs {
   float *o_part, *lse_part;  // [R, B, Qn, Hq, D], [R, B, Qn, Hq]
   float *rec_o, *rec_lse;    // [B, rb, QN, Hq, D], [B, rb, QN, Hq]: shared-slice partials
   int2 *span;                // [B, R]: contributors (c_lo, c_hi) of a shared slice
+  // fused merge (decode step, one query): the combine CTA that completes a
+  // row group's R slices merges them into m_out / m_lse; mcnt counts the
+  // arrivals per (sequence, row group). m_out == nullptr: no fused merge.
+  int *mcnt;                 // [B, ceil(Hq / DV_CB_ROWS)]
+  void *m_out;
+  int m_bf16;
+  float *m_lse;
   int B, Hq, Hkv, G, P, max_pages, num_pages, k, k_pad, R, ncb, rb;
   int Qn, q0, qn;            // queries per sequence; first query and size of this group
   int ring_bytes;            // DV_WARPS * ST * DV_STAGE
@@ -444,6 +452,10 @@ __global__ void __launch_bounds__(DV_WARPS * 32, DV_CTAS_PER_SM) sparse_decode_k
       if (s_ct[r] != 0) contributors(r, sp.x, sp.y);
       a.span[(size_t)b * a.R + r] = sp;
     }
+    if (a.m_out != nullptr) {  // the fused merge's arrival counters of this sequence
+      const int ng = (a.Hq + DV_CB_ROWS - 1) / DV_CB_ROWS;
+      for (int g2 = tid; g2 < ng; g2 += blockDim.x) a.mcnt[(size_t)b * ng + g2] = 0;
+    }
   }
   // slices that own no selected block: O_r = 0, LSE_r = -inf (CTA 0 writes them)
   if (has_head && c == 0) {
@@ -570,52 +582,70 @@ __global__ void __launch_bounds__(DV_CB_ROWS * 32) decode_combine_kernel(DecodeA
   // row = (query qq of the group, head h)
   const int q = blockIdx.x * DV_CB_ROWS + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   const int2 sp = a.span[(size_t)b * a.R + r];
-  if (sp.y <= sp.x || q >= a.qn * a.Hq) return;  // written by the decode kernel itself
-  const int n = sp.y - sp.x + 1;
-  const size_t stride = (size_t)a.qn * a.Hq;                         // between records
-  const size_t row0 = ((size_t)b * a.rb + sp.x + r) * stride + q;    // record i at row0 + i*stride
-  float M = -INFINITY;
-  for (int i0 = 0; i0 < n; i0 += 32) {
-    const float l = i0 + lane < n ? __ldcg(a.rec_lse + row0 + (size_t)(i0 + lane) * stride)
-                                  : -INFINITY;
-    M = fmaxf(M, l);
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  float acc[4] = {0.f, 0.f, 0.f, 0.f}, wsum = 0.f;
-  if (M != -INFINITY) {
+  // a slice inside one CTA's range was written by the decode kernel itself
+  if (sp.y > sp.x && q < a.qn * a.Hq) {
+    const int n = sp.y - sp.x + 1;
+    const size_t stride = (size_t)a.qn * a.Hq;                         // between records
+    const size_t row0 = ((size_t)b * a.rb + sp.x + r) * stride + q;    // record i at row0 + i*stride
+    float M = -INFINITY;
     for (int i0 = 0; i0 < n; i0 += 32) {
       const float l = i0 + lane < n ? __ldcg(a.rec_lse + row0 + (size_t)(i0 + lane) * stride)
                                     : -INFINITY;
-      const float wl = l == -INFINITY ? 0.f : __expf(l - M);  // weight of record i0 + lane
-      const int m = min(32, n - i0);
-      for (int u0 = 0; u0 < m; u0 += DV_CB_BATCH) {
-        float4 v[DV_CB_BATCH];
+      M = fmaxf(M, l);
+    }
 #pragma unroll
-        for (int u = 0; u < DV_CB_BATCH; ++u) {
-          const size_t rr = row0 + (size_t)(i0 + min(u0 + u, m - 1)) * stride;
-          v[u] = __ldcg(reinterpret_cast<const float4 *>(a.rec_o + rr * DV_D) + lane);
-        }
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float acc[4] = {0.f, 0.f, 0.f, 0.f}, wsum = 0.f;
+    if (M != -INFINITY) {
+      for (int i0 = 0; i0 < n; i0 += 32) {
+        const float l = i0 + lane < n ? __ldcg(a.rec_lse + row0 + (size_t)(i0 + lane) * stride)
+                                      : -INFINITY;
+        const float wl = l == -INFINITY ? 0.f : __expf(l - M);  // weight of record i0 + lane
+        const int m = min(32, n - i0);
+        for (int u0 = 0; u0 < m; u0 += DV_CB_BATCH) {
+          float4 v[DV_CB_BATCH];
 #pragma unroll
-        for (int u = 0; u < DV_CB_BATCH; ++u) {
-          const float w = __shfl_sync(0xffffffffu, wl, (u0 + u) & 31);
-          if (u0 + u < m && w != 0.f) {  // a record of a query that saw nothing holds zeros
-            wsum += w;
-            acc[0] += w * v[u].x;
-            acc[1] += w * v[u].y;
-            acc[2] += w * v[u].z;
-            acc[3] += w * v[u].w;
+          for (int u = 0; u < DV_CB_BATCH; ++u) {
+            const size_t rr = row0 + (size_t)(i0 + min(u0 + u, m - 1)) * stride;
+            v[u] = __ldcg(reinterpret_cast<const float4 *>(a.rec_o + rr * DV_D) + lane);
+          }
+#pragma unroll
+          for (int u = 0; u < DV_CB_BATCH; ++u) {
+            const float w = __shfl_sync(0xffffffffu, wl, (u0 + u) & 31);
+            if (u0 + u < m && w != 0.f) {  // a record of a query that saw nothing holds zeros
+              wsum += w;
+              acc[0] += w * v[u].x;
+              acc[1] += w * v[u].y;
+              acc[2] += w * v[u].z;
+              acc[3] += w * v[u].w;
+            }
           }
         }
       }
     }
+    const int qq = q / a.Hq, h = q % a.Hq;
+    const size_t orow = (((size_t)r * a.B + b) * a.Qn + a.q0 + qq) * a.Hq + h;
+    const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+    reinterpret_cast<float4 *>(a.o_part + orow * DV_D)[lane] =
+        make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+    if (lane == 0) a.lse_part[orow] = wsum > 0.f ? M + logf(wsum) : -INFINITY;
   }
-  const int qq = q / a.Hq, h = q % a.Hq;
-  const size_t orow = (((size_t)r * a.B + b) * a.Qn + a.q0 + qq) * a.Hq + h;
-  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-  reinterpret_cast<float4 *>(a.o_part + orow * DV_D)[lane] =
-      make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
-  if (lane == 0) a.lse_part[orow] = wsum > 0.f ? M + logf(wsum) : -INFINITY;
+  if (a.m_out == nullptr) return;
+  // fused merge (one query per sequence): the CTA whose arrival completes the
+  // row group's R slices merges them (its own rows, one warp per head)
+  __shared__ int s_last;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();  // this CTA's partials before its arrival
+    int *cnt = a.mcnt + (size_t)b * gridDim.x + blockIdx.x;
+    s_last = atomicAdd(cnt, 1) == a.R - 1;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();  // every other slice's partials are visible now
+  if (q < a.Hq)
+    merge_row(a.R, a.B * a.Hq, DV_D, a.o_part, a.lse_part, b * a.Hq + q, a.m_out, a.m_bf16,
+              a.m_lse);
 }
 
 struct DecodePlan {
@@ -653,7 +683,11 @@ cudaError_t launch_st(const DecodeArgs &a, const DecodePlan &p, int B, cudaStrea
   if (e != cudaSuccess) return e;
   e = launch_pdl(sparse_decode_kernel<ST, QN>, dim3(p.ncb, p.nhg, B), DV_WARPS * 32, p.smem, st,
                  a);
-  if (e != cudaSuccess || p.ncb == 1) return e;  // one CTA per sequence: nothing to combine
+  if (e != cudaSuccess) return e;
+  if (p.ncb == 1)  // one CTA per sequence: nothing to combine
+    return a.m_out == nullptr ? e
+                              : launch_merge(a.R, B, a.Hq, DV_D, a.o_part, a.lse_part, a.m_out,
+                                             a.m_bf16, a.m_lse, st);
   return launch_pdl(decode_combine_kernel,
                     dim3((QN * a.Hq + DV_CB_ROWS - 1) / DV_CB_ROWS, a.R, B), DV_CB_ROWS * 32, 0,
                     st, a);
@@ -673,14 +707,16 @@ cudaError_t launch_qn(const DecodeArgs &a, const DecodePlan &p, int B, cudaStrea
 size_t decode_ws_bytes(const qsa_dims &d, int B, int Qn, int k, int R) {
   const DecodePlan p = plan_decode(d, B, k, R);
   const size_t rows = (size_t)B * p.rb * (Qn < DV_QGROUP ? Qn : DV_QGROUP) * d.Hq;
-  return rows * (DV_D + 1) * sizeof(float) + (size_t)B * R * sizeof(int2);
+  const size_t groups = (size_t)(d.Hq + DV_CB_ROWS - 1) / DV_CB_ROWS;
+  return rows * (DV_D + 1) * sizeof(float) + (size_t)B * R * sizeof(int2) +
+         (size_t)B * groups * sizeof(int);
 }
 
 cudaError_t launch_sparse_decode(const qsa_dims &d, const qsa_cache &c, int B, int Qn,
                                  const int32_t *seq_lens, const void *q, const int32_t *sel,
                                  int k, int R, float *o_part, float *lse_part, void *ws,
                                  unsigned *err, cudaStream_t st, const int32_t *row_start,
-                                 int S) {
+                                 int S, void *m_out, int m_bf16, float *m_lse) {
   if (B == 0) return cudaSuccess;
   const DecodePlan p = plan_decode(d, B, k, R);
   DecodeArgs a;
@@ -692,6 +728,9 @@ cudaError_t launch_sparse_decode(const qsa_dims &d, const qsa_cache &c, int B, i
   a.sel = sel;
   a.row_start = row_start;
   a.S = S;
+  a.m_out = Qn == 1 ? m_out : nullptr;
+  a.m_bf16 = m_bf16;
+  a.m_lse = m_lse;
   a.o_part = o_part;
   a.lse_part = lse_part;
   a.B = B;
@@ -718,6 +757,7 @@ cudaError_t launch_sparse_decode(const qsa_dims &d, const qsa_cache &c, int B, i
     a.rec_o = static_cast<float *>(ws);
     a.rec_lse = a.rec_o + rows * DV_D;
     a.span = reinterpret_cast<int2 *>(a.rec_lse + rows);
+    a.mcnt = reinterpret_cast<int *>(a.span + (size_t)B * R);
     const cudaError_t e = a.qn == 2 ? launch_qn<2>(a, p, B, st) : launch_qn<1>(a, p, B, st);
     if (e != cudaSuccess) return e;
   }

@@ -164,10 +164,11 @@ qsa_status qsa_topk_select(int32_t B, const int32_t *seq_lens,
                            qsa_stream_t stream);
 
 /* Scratch bytes qsa_sparse_decode needs for B sequences, top-k k, R slices.
- * The scratch holds the partial results of slices that several CTAs share
- * and the list of those slices; it needs no initialisation and every call
- * writes what it later reads (calls sharing one scratch buffer must be
- * ordered on the GPU). */
+ * The scratch holds the partial results of slices that several CTAs share,
+ * the list of those slices and (for qsa_decode_step's fused merge) one
+ * arrival counter per sequence and group of 8 query heads; it needs no
+ * initialisation and every call writes what it later reads (calls sharing
+ * one scratch buffer must be ordered on the GPU). */
 size_t qsa_sparse_decode_workspace_size(const qsa_dims *dims, int32_t B,
                                         int32_t k, int32_t R);
 
@@ -270,12 +271,15 @@ qsa_status qsa_merge(int32_t R, int32_t B, int32_t Hq, int32_t D,
  * N == 0), then qsa_index_score, qsa_topk_select (no workspace),
  * qsa_sparse_decode and qsa_merge, enqueued in that order on `stream`, with
  * the arguments documented at each of those calls (the merge writes `out`
- * [B, Hq, D] and `lse_out` [B, Hq] from o_part / lse_part). The page orders
- * the steps (section "What the pull request actually changes"); the single
- * call is an interface convenience of this library that saves the caller
- * four calls. The calls' own argument checks apply; the first failing call
- * stops the sequence and its status is returned (calls before it stay
- * enqueued). */
+ * [B, Hq, D] and `lse_out` [B, Hq] from o_part / lse_part, which also hold
+ * the R partials afterwards). Here the merge runs inside the decode's last
+ * kernel (the CTA that completes a group of rows merges them, with the
+ * arithmetic of qsa_merge, so the results are the same bits), which saves a
+ * launch. The page orders the steps (section "What the pull request
+ * actually changes"); the single call is an interface convenience of this
+ * library that saves the caller four calls. The calls' own argument checks
+ * apply; the first failing call stops the sequence and its status is
+ * returned (calls before it stay enqueued). */
 qsa_status qsa_decode_step(const qsa_dims *dims, const qsa_cache *cache,
                            int32_t N, const int32_t *tok_seq,
                            const int32_t *tok_pos, const void *k_new,

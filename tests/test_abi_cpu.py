@@ -45,11 +45,12 @@ def test_version_and_workspace_sizes(L):
     # records of shared slices: 296 CTA slots / B sequences CTAs per sequence
     # (at most one per tile, at least ceil((k/4 + R - 1) / 256) for the page
     # table), keyed by CTA + slice, each 32 heads x (128 + 1) floats; plus one
-    # (c_lo, c_hi) pair per (sequence, slice)
+    # (c_lo, c_hi) pair per (sequence, slice) and one arrival counter per
+    # (sequence, group of 8 query heads) for the decode step's fused merge
     for B, k, R, ncb in ((8, 512, 4, 37), (512, 512, 4, 1), (512, 4096, 4, 5),
                          (2, 512, 2, 129), (1, 1, 1, 1)):
         assert qsa.qsa_sparse_decode_workspace_size(d, B, k, R) == \
-            B * (ncb + R - 1) * 32 * 129 * 4 + B * R * 8, (B, k, R)
+            B * (ncb + R - 1) * 32 * 129 * 4 + B * R * 8 + B * 4 * 4, (B, k, R)
 
 
 def test_prefill_workspace_sizes(L):

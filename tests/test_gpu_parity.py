@@ -415,6 +415,29 @@ def test_steady128x64k_append_steps():
         assert np.array_equal(run.side_rows(b, L), oracle.side_cache(bits(X), L)), b
 
 
+@pytest.mark.parametrize("lens,R", [
+    ([30001, 5000, 77, 12345, 2048], 4),   # sequences split over CTAs: fused into the combine
+    ([3000] * 300, 2),                     # one CTA per sequence: the merge kernel
+])
+def test_decode_step_fused_merge_equals_qsa_merge(lens, R):
+    wl = make_custom(DIMS_FULL, lens, k=512, R=R, seed=len(lens) + R, device=DEV)
+    run = GpuRun(wl)
+    for out_dtype in (torch.bfloat16, torch.float32):
+        run.buf.out = torch.full((wl.B, run.dims.Hq, run.dims.D), float("nan"), device=DEV,
+                                 dtype=out_dtype)
+        run.step()
+        out2 = torch.full_like(run.buf.out, float("nan"))
+        lse2 = torch.full_like(run.buf.lse, float("nan"))
+        qsa.qsa_merge(run.buf.o_part, run.buf.lse_part, out2, lse2)
+        assert qsa.qsa_check_device_errors() == 0
+        assert torch.equal(run.buf.out.view(torch.int16 if out_dtype == torch.bfloat16
+                                            else torch.int32),
+                           out2.view(torch.int16 if out_dtype == torch.bfloat16 else torch.int32))
+        assert torch.equal(run.buf.lse.view(torch.int32), lse2.view(torch.int32))
+    for b in (0, 2, wl.B - 1):
+        _check_seq(run, b)
+
+
 # ------------------------------------------------------------ multi-query decode
 
 @pytest.mark.parametrize("Qn,R", [(1, 4), (2, 1), (2, 4), (3, 8), (5, 2)])
