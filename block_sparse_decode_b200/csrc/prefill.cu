@@ -78,8 +78,7 @@ struct PfArgs {
   int4 *ginfo;       // [Gmax] {sequence, first row, rows, complete blocks of the last row}
   float *scores;
   int S, Nq, Gmax, QG, ld, P, rpp, max_pages, num_pages, Hi, stages;
-  int box;  // rows per page piece: min(P/4, 128)
-  int ept;  // page pieces per tile: 128 / box
+  int box;  // rows per page piece: min(P/4, 128); a tile holds 128 / box pieces
   unsigned *err;
 };
 
@@ -581,7 +580,6 @@ cudaError_t launch_prefill_index_score(const qsa_dims &d, const qsa_cache &c, in
   a.P = d.P;
   a.rpp = d.P / 4;
   a.box = std::min(a.rpp, PF_M);
-  a.ept = PF_M / a.box;
   a.max_pages = c.max_pages_per_seq;
   a.num_pages = c.num_pages;
   a.Hi = d.Hi;

@@ -25,7 +25,7 @@ def token_index(wl, upto=None):
     return seq, pos
 
 
-class GpuRun:
+class CudaRun:
     """The cache of a workload on the GPU plus the buffers of one decode step."""
 
     def __init__(self, wl, k=None, R=None, prefill=None, poison=True):

@@ -18,7 +18,7 @@ import oracle
 from block_sparse_decode_b200 import qsa
 from synth import make_custom, make_workload, step_queries
 from synth.workloads import DIMS_FULL, Dims
-from tests.gpu_harness import GpuRun, oracle_sequence, score_tolerance, token_index
+from tests.gpu_harness import CudaRun, oracle_sequence, score_tolerance, token_index
 from tests.helpers import bf16_same, bits, check_attention, check_selection
 
 pytestmark = pytest.mark.gpu
@@ -58,7 +58,7 @@ def _check_seq(run, b, L=None, q=None, q_idx=None, w=None, full=True):
 @pytest.mark.parametrize("R", [2, 1, 3, 8])
 def test_tiny_preset_end_to_end(R):
     wl = make_workload("tiny", device=DEV)
-    run = GpuRun(wl, R=R)
+    run = CudaRun(wl, R=R)
     run.step()
     for b in range(wl.B):
         _check_seq(run, b)
@@ -69,7 +69,7 @@ def test_tiny_preset_end_to_end(R):
 def test_ragged_paged_full_heads(R):
     lens = [1, 2, 3, 4, 5, 63, 64, 65, 2047, 2048, 2049, 2051, 4099, 9001, 20000]
     wl = make_custom(DIMS_FULL, lens, k=512, R=R, seed=101, device=DEV, paged=True)
-    run = GpuRun(wl)
+    run = CudaRun(wl)
     run.step()
     for b in range(wl.B):
         _check_seq(run, b)
@@ -84,7 +84,7 @@ def test_ragged_paged_full_heads(R):
 def test_other_dims(dims, lens, k):
     for R in (1, 3):
         wl = make_custom(dims, lens, k=k, R=R, seed=102, device=DEV, paged=True)
-        run = GpuRun(wl)
+        run = CudaRun(wl)
         run.step()
         for b in range(wl.B):
             _check_seq(run, b)
@@ -94,7 +94,7 @@ def test_clustered_selection_leaves_empty_slices():
     # needles + k small: the selection sits in a few slices, most slices empty
     d = DIMS_FULL
     wl = make_custom(d, [8192, 3000], k=4, R=16, seed=103, device=DEV, needles=4)
-    run = GpuRun(wl)
+    run = CudaRun(wl)
     run.step()
     for b in range(wl.B):
         _check_seq(run, b)
@@ -233,7 +233,7 @@ def test_append_incremental_equals_bulk_side_cache():
     d = DIMS_FULL
     lens = [515, 64, 7]
     wl = make_custom(d, lens, k=8, R=1, seed=105, device=DEV, paged=True)
-    run = GpuRun(wl, prefill=[0] * 3)  # nothing written in bulk
+    run = CudaRun(wl, prefill=[0] * 3)  # nothing written in bulk
     for t in range(max(lens)):
         live = [b for b in range(3) if t < lens[b]]
         rows = torch.tensor([wl.tok_off[b] + t for b in live], device=DEV)
@@ -251,7 +251,7 @@ def test_append_incremental_equals_bulk_side_cache():
 
 def test_bad_page_ids_are_flagged_not_faulted():
     wl = make_custom(DIMS_FULL, [3000, 900], k=64, R=2, seed=106, device=DEV)
-    run = GpuRun(wl)
+    run = CudaRun(wl)
     bad = run.cache.block_table.clone()
     run.cache.block_table[0, 3] = wl.num_pages + 1000   # out-of-range page id
     run.cache.block_table[1, 1] = -5
@@ -265,7 +265,7 @@ def test_bad_page_ids_are_flagged_not_faulted():
 
 def test_seq_len_beyond_score_row_is_flagged():
     wl = make_custom(DIMS_FULL, [3000, 900], k=64, R=1, seed=107, device=DEV)
-    run = GpuRun(wl)
+    run = CudaRun(wl)
     sc = torch.zeros((2, 100), dtype=torch.float32, device=DEV)  # ld too short for seq 0
     qsa.qsa_index_score(run.dims, run.cache, run.seq_lens, wl.q_idx, wl.w, sc)
     with pytest.raises(qsa.QsaError) as ei:
@@ -275,7 +275,7 @@ def test_seq_len_beyond_score_row_is_flagged():
 
 def test_invalid_arguments_rejected_on_host():
     wl = make_custom(DIMS_FULL, [100], k=8, R=1, seed=108, device=DEV)
-    run = GpuRun(wl)
+    run = CudaRun(wl)
     with pytest.raises(qsa.QsaError) as ei:
         qsa.qsa_sparse_decode(run.dims, run.cache, run.seq_lens, wl.q, run.buf.sel, 8, 65,
                               run.buf.o_part, run.buf.lse_part, run.buf.ws)
@@ -296,7 +296,7 @@ def test_decode_shapes_back_to_back():
     # calls of different B, k and R in a row (different CTA splits and slice
     # layouts) sharing one scratch buffer, each checked against the oracle
     wl = make_custom(DIMS_FULL, [9000, 3001, 17, 40000], k=512, R=4, seed=109, device=DEV)
-    run = GpuRun(wl)
+    run = CudaRun(wl)
     run.step()
     sel = run.buf.sel
     ws = torch.empty(max(qsa.qsa_sparse_decode_workspace_size(run.dims, B, k, R)
@@ -348,7 +348,7 @@ def _sampled(wl, n):
 
 def test_b32x32k_full_size():
     wl = make_workload("b32x32k", device=DEV)
-    run = GpuRun(wl)
+    run = CudaRun(wl)
     run.step()
     for b in _sampled(wl, 3):
         _check_seq(run, b)
@@ -358,7 +358,7 @@ def test_b32x32k_full_size():
 
 def test_b8x256k_split_equals_unsplit():
     wl = make_workload("b8x256k", device=DEV)
-    run = GpuRun(wl)
+    run = CudaRun(wl)
     run.step()
     for b in _sampled(wl, 2):
         _check_seq(run, b)
@@ -378,7 +378,7 @@ def test_b8x256k_split_equals_unsplit():
 @pytest.mark.parametrize("R", [1, 2, 4, 8])
 def test_ragged64_full_size(R):
     wl = make_workload("ragged64", device=DEV)
-    run = GpuRun(wl, R=R)
+    run = CudaRun(wl, R=R)
     run.step()
     lens = np.array(wl.seq_lens)
     pick = {int(lens.argmin()), int(lens.argmax())}
@@ -395,7 +395,7 @@ def test_steady128x64k_append_steps():
     wl = make_workload("steady128x64k", device=DEV)
     spec_prefill, steps = wl.extra["prefill"], wl.extra["steps"]
     for k in (256, 512, 1024):
-        run = GpuRun(wl, k=k, prefill=[spec_prefill] * wl.B)
+        run = CudaRun(wl, k=k, prefill=[spec_prefill] * wl.B)
         for t in range(steps):
             lens = [spec_prefill + t + 1] * wl.B
             q, q_idx, w = step_queries(wl, t)
@@ -421,7 +421,7 @@ def test_steady128x64k_append_steps():
 ])
 def test_decode_step_fused_merge_equals_qsa_merge(lens, R):
     wl = make_custom(DIMS_FULL, lens, k=512, R=R, seed=len(lens) + R, device=DEV)
-    run = GpuRun(wl)
+    run = CudaRun(wl)
     for out_dtype in (torch.bfloat16, torch.float32):
         run.buf.out = torch.full((wl.B, run.dims.Hq, run.dims.D), float("nan"), device=DEV,
                                  dtype=out_dtype)
@@ -447,7 +447,7 @@ def test_multi_query_decode_matches_oracle(Qn, R):
     # Qn leave the first queries with nothing to see (zeros, LSE = -inf).
     lens = [9001, 2050, 3, 40003, 1026, 13]
     wl = make_custom(DIMS_FULL, lens, k=256, R=R, seed=300 + 10 * Qn + R, device=DEV)
-    run = GpuRun(wl)
+    run = CudaRun(wl)
     run.step()  # cache complete, selection of every sequence in run.buf.sel
     d = run.dims
     g = torch.Generator(device=DEV).manual_seed(Qn)
@@ -486,7 +486,7 @@ def test_context_parallel_ranks_merge_to_full_attention(W):
     # attention over the whole selection
     lens = [30001, 5000, 77, 12345, 2048]
     wl = make_custom(DIMS_FULL, lens, k=512, R=1, seed=400 + W, device=DEV)
-    run = GpuRun(wl)
+    run = CudaRun(wl)
     run.step()
     d, B = run.dims, wl.B
     sel = run.buf.sel

@@ -17,7 +17,7 @@ import oracle
 from block_sparse_decode_b200 import qsa
 from synth import make_custom, prefill_queries
 from synth.workloads import DIMS_FULL, DIMS_TINY, Dims
-from tests.gpu_harness import GpuRun
+from tests.gpu_harness import CudaRun
 from tests.helpers import bits, check_attention, check_selection
 
 pytestmark = pytest.mark.gpu
@@ -69,7 +69,7 @@ def _check_rows(wl, chunks, rows_to_check, row_start, q, q_idx, w, buf, k, R):
 ])
 def test_sparse_prefill_matches_oracle(dims, lens, chunks, k, R):
     wl = make_custom(dims, lens, k=k, R=R, seed=500 + sum(chunks), device=DEV)
-    run = GpuRun(wl, prefill=lens)  # every token, chunks included, appended
+    run = CudaRun(wl, prefill=lens)  # every token, chunks included, appended
     d = run.dims
     row_start, q, q_idx, w = prefill_queries(wl, chunks)
     Nq = int(row_start[-1])
@@ -84,7 +84,7 @@ def test_sparse_prefill_matches_oracle(dims, lens, chunks, k, R):
 def test_prefill_calls_one_by_one_equal_the_single_call():
     lens, chunks, k, R = [3001, 999], [40, 33], 128, 3
     wl = make_custom(DIMS_FULL, lens, k=k, R=R, seed=77, device=DEV)
-    run = GpuRun(wl, prefill=lens)
+    run = CudaRun(wl, prefill=lens)
     d = run.dims
     row_start, q, q_idx, w = prefill_queries(wl, chunks)
     Nq, S, ld = int(row_start[-1]), wl.B, qsa.ld_for(lens)
@@ -118,7 +118,7 @@ def test_prefill_last_rows_equal_the_decode_step():
     # same bytes in, the decode kernels' scores, selection and output out
     lens, chunks, k, R = [20000, 4097, 333], [17, 3, 5], 512, 4
     wl = make_custom(DIMS_FULL, lens, k=k, R=R, seed=12, device=DEV)
-    run = GpuRun(wl, prefill=lens)
+    run = CudaRun(wl, prefill=lens)
     d = run.dims
     row_start, q, q_idx, w = prefill_queries(wl, chunks)
     Nq = int(row_start[-1])
@@ -144,7 +144,7 @@ def test_prefill_last_rows_equal_the_decode_step():
 def test_prefill_bad_layout_is_flagged_and_rows_left_empty():
     lens = [300, 200]
     wl = make_custom(DIMS_FULL, lens, k=64, R=1, seed=3, device=DEV)
-    run = GpuRun(wl, prefill=lens)
+    run = CudaRun(wl, prefill=lens)
     d = run.dims
     _, q, q_idx, w = prefill_queries(wl, [10, 5])
     # sequence 1's chunk claims 250 rows, more than its 200 tokens
@@ -173,7 +173,7 @@ def test_prefill_rejects_unsupported_and_bad_arguments():
     lens = [64]
     wl = make_custom(Dims(Hq=8, Hkv=2, D=128, Hi=12, di=64, P=64, scale=0.1), lens, k=8, R=1,
                      seed=1, device=DEV)
-    run = GpuRun(wl, prefill=lens)
+    run = CudaRun(wl, prefill=lens)
     row_start, q, q_idx, w = prefill_queries(wl, [4])
     scores = torch.empty((4, run.ld), device=DEV)
     row_len = torch.empty(4, dtype=torch.int32, device=DEV)
@@ -184,7 +184,7 @@ def test_prefill_rejects_unsupported_and_bad_arguments():
     assert e.value.status == qsa.QSA_ERR_UNSUPPORTED
     # a workspace below the stated size is refused on the host
     wl2 = make_custom(DIMS_FULL, [100], k=8, R=1, seed=2, device=DEV)
-    run2 = GpuRun(wl2, prefill=[100])
+    run2 = CudaRun(wl2, prefill=[100])
     row_start, q, q_idx, w = prefill_queries(wl2, [4])
     need = qsa.qsa_prefill_index_score_workspace_size(run2.dims, 1, 4)
     small = torch.empty(need - 16, dtype=torch.uint8, device=DEV)
@@ -201,7 +201,7 @@ def test_prefill_256k_chunks_sampled_rows():
     # selection and output against the oracle
     lens, chunks, k, R = [262144, 262144], [128, 128], 512, 4
     wl = make_custom(DIMS_FULL, lens, k=k, R=R, seed=2026, device=DEV, mixture=True)
-    run = GpuRun(wl, prefill=lens)
+    run = CudaRun(wl, prefill=lens)
     d = run.dims
     row_start, q, q_idx, w = prefill_queries(wl, chunks)
     Nq = int(row_start[-1])

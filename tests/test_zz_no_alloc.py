@@ -18,7 +18,7 @@ import torch
 from block_sparse_decode_b200 import qsa
 from synth import make_custom
 from synth.workloads import DIMS_FULL
-from tests.gpu_harness import GpuRun
+from tests.gpu_harness import CudaRun
 from tests.helpers import check_attention
 
 pytestmark = pytest.mark.gpu
@@ -27,7 +27,7 @@ pytestmark = pytest.mark.gpu
 def test_static_scratch_decode_matches_workspace_decode():
     lens = [5000, 20001, 3, 2051, 40000, 777]
     wl = make_custom(DIMS_FULL, lens, k=512, R=4, seed=201, device="cuda", paged=True)
-    run = GpuRun(wl)
+    run = CudaRun(wl)
     run.step()  # cache complete, selection in run.buf.sel
     need = qsa.qsa_sparse_decode_workspace_size(run.dims, wl.B, wl.k, wl.R)
     assert 0 < need <= (32 << 20)
@@ -54,7 +54,7 @@ def test_static_scratch_serves_the_largest_k_and_R():
     assert 0 < need <= (32 << 20)
     wl = make_custom(DIMS_FULL, [20000, 16390], k=4096, R=64, seed=202, device="cuda",
                      paged=True)
-    run = GpuRun(wl)
+    run = CudaRun(wl)
     run.step()
     ref_o = run.buf.o_part.clone()
     ref_l = run.buf.lse_part.clone()
