@@ -576,3 +576,19 @@ def test_prefill_rows_ignore_later_tokens():
         assert np.array_equal(got[i]["O"], base[i]["O"])
         if i + 1 < T:   # a later row sees the change
             assert not np.array_equal(got[T - 1]["O"], base[T - 1]["O"])
+
+
+def test_prefill_rows_split_merge_equals_unsplit():
+    # each row's R partials merged equal its one-slice result (fp64 rounding)
+    L, T = 97, 7
+    K, V, X, q, qi, w = _prefill_case(L, T, seed=31)
+    one = oracle.prefill_sequence(bits(X), bits(K), bits(V), bits(q), bits(qi), w.numpy(), L, T,
+                                  k=9, R=1, scale=0.3)
+    for R in (2, 3, 8):
+        rows = oracle.prefill_sequence(bits(X), bits(K), bits(V), bits(q), bits(qi), w.numpy(), L,
+                                       T, k=9, R=R, scale=0.3)
+        for a, b in zip(rows, one):
+            assert np.array_equal(a["sel"], b["sel"])
+            Om, Lm = oracle.merge_partials(a["O_part"], a["LSE_part"])
+            assert np.abs(Om - b["O"]).max() <= 1e-12
+            assert np.abs(Lm - b["LSE"]).max() <= 1e-12
