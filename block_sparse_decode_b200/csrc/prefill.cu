@@ -413,7 +413,11 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         const int nr = gi.z - half * QH;
         for (int i = lane; i < PF_EPI_COLS; i += 32) {
           const int qi = i / HI, h = i % HI;
-          w_s[e][i] = qi < nr ? __ldg(a.w + (size_t)(row0 + qi) * HI + h) : 0.f;
+          const float wv = qi < nr ? __ldg(a.w + (size_t)(row0 + qi) * HI + h) : 0.f;
+          if constexpr (HI <= 16)  // (row 2p, row 2p + 1) pairs, head by head
+            w_s[e][((qi >> 1) * HI + h) * 2 + (qi & 1)] = wv;
+          else
+            w_s[e][i] = wv;
         }
         for (int i = lane; i < QH; i += 32) nf_s[e][i] = i < nr ? a.row_len[row0 + i] >> 2 : 0;
         __syncwarp();
@@ -437,15 +441,43 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
           tc_fence_before();
           mbar_arrive(tempty0 + 8 * acc);
         }
+        if constexpr (HI <= 16) {
+          // the chunk holds 32 / HI whole rows: two rows advance together in
+          // one paired fp32 FMA, each in head order from 0 (the same bits
+          // as one FMA per column)
+          constexpr int QC = 32 / HI;
 #pragma unroll
-        for (int u = 0; u < 32; ++u) {
-          const int col = c0 + u;
-          const float v = __uint_as_float(r0[u]);
-          part = fmaf(w_s[e][col], fmaxf(v, 0.f), part);
-          if (col % HI == HI - 1) {
-            const int qi = col / HI;
-            if (j < nf_s[e][qi]) a.scores[(size_t)(row0 + qi) * a.ld + j] = part;
-            part = 0.f;
+          for (int pr = 0; pr < QC / 2; ++pr) {
+            const int qa = c0 / HI + 2 * pr;
+            unsigned long long s2;
+            asm("mov.b64 %0, {%1, %1};" : "=l"(s2) : "f"(0.f));
+#pragma unroll
+            for (int h = 0; h < HI; ++h) {
+              const float va = fmaxf(__uint_as_float(r0[2 * pr * HI + h]), 0.f);
+              const float vb = fmaxf(__uint_as_float(r0[(2 * pr + 1) * HI + h]), 0.f);
+              const float2 w2 =
+                  *reinterpret_cast<const float2 *>(&w_s[e][((qa >> 1) * HI + h) * 2]);
+              unsigned long long v2, ww;
+              asm("mov.b64 %0, {%1, %2};" : "=l"(v2) : "f"(va), "f"(vb));
+              asm("mov.b64 %0, {%1, %2};" : "=l"(ww) : "f"(w2.x), "f"(w2.y));
+              asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(s2) : "l"(ww), "l"(v2));
+            }
+            float pa, pb;
+            asm("mov.b64 {%0, %1}, %2;" : "=f"(pa), "=f"(pb) : "l"(s2));
+            if (j < nf_s[e][qa]) a.scores[(size_t)(row0 + qa) * a.ld + j] = pa;
+            if (j < nf_s[e][qa + 1]) a.scores[(size_t)(row0 + qa + 1) * a.ld + j] = pb;
+          }
+        } else {
+#pragma unroll
+          for (int u = 0; u < 32; ++u) {
+            const int col = c0 + u;
+            const float v = __uint_as_float(r0[u]);
+            part = fmaf(w_s[e][col], fmaxf(v, 0.f), part);
+            if (col % HI == HI - 1) {
+              const int qi = col / HI;
+              if (j < nf_s[e][qi]) a.scores[(size_t)(row0 + qi) * a.ld + j] = part;
+              part = 0.f;
+            }
           }
         }
       }
