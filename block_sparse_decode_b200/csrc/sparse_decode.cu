@@ -35,7 +35,14 @@
 // ordered). (6) A second, small kernel, launched as a programmatic dependent
 // of the first, combines the partials of each shared slice once all streaming
 // is done (every load of a row batched, so it costs a couple of L2 round
-// trips); no atomics, fences or counters are needed.
+// trips). Inside the one-call decode step it also merges the R slices: each
+// of its CTAs counts its arrival per (sequence, group of heads) after a
+// fence, and the one that completes the group merges it (merge_row.cuh, the
+// arithmetic of qsa_merge).
+//
+// The same kernels serve sparse prefill rows (row_start != nullptr): a row is
+// a query of a chunk; it takes its sequence's block-table row and its own
+// causal length, and is otherwise a sequence of one query.
 //
 // Roofline: HBM-bound; algorithmic bytes = selected tokens * Hkv * D * 2 * 2
 // (each selected token's K and V rows read once).
