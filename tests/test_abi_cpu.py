@@ -113,3 +113,23 @@ def test_host_side_argument_checks(L):
     unaligned = qsa._Cache(17, 16, 16, 16, 16, 1, 1, 1)
     assert L.qsa_append(ctypes.byref(ok), ctypes.byref(unaligned), 1, 16, 16, 16, 16, 16,
                         None) == qsa.QSA_ERR_INVALID_ARG
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    # no fallback: without libqsa.so every call raises instead of computing
+    # anything on the host
+    import subprocess
+    import sys
+    code = (
+        "import sys; sys.path.insert(0, %r)\n"
+        "from block_sparse_decode_b200 import qsa\n"
+        "qsa.LIB_PATH = %r\n"
+        "try:\n"
+        "    qsa.qsa_version()\n"
+        "except ImportError as e:\n"
+        "    print('raised', 'missing' in str(e))\n"
+    ) % (os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+         str(tmp_path / "libqsa.so"))
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stderr
+    assert r.stdout.strip() == "raised True"
