@@ -33,14 +33,21 @@ __device__ __forceinline__ void merge_row(int R, int rows, int D, const float *o
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
   const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-  for (int d0 = lane * 4; d0 < D; d0 += 128) {
+  // every lane runs the same number of passes over the head dims (the weight
+  // shuffles below need the whole warp); a lane past D loads and stores nothing
+  const int passes = (D + 127) / 128;
+  for (int it = 0; it < passes; ++it) {
+    const int d0 = it * 128 + lane * 4;
+    const bool live = d0 < D;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int r0 = 0; r0 < R; r0 += MERGE_BATCH) {
       float4 v[MERGE_BATCH];
 #pragma unroll
       for (int u = 0; u < MERGE_BATCH; ++u) {
         const int r = min(r0 + u, R - 1);
-        v[u] = __ldcg(reinterpret_cast<const float4 *>(o_part + ((size_t)r * rows + row) * D + d0));
+        v[u] = live ? __ldcg(reinterpret_cast<const float4 *>(o_part + ((size_t)r * rows + row) * D +
+                                                               d0))
+                    : make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll
       for (int u = 0; u < MERGE_BATCH; ++u) {
@@ -58,6 +65,7 @@ __device__ __forceinline__ void merge_row(int R, int rows, int D, const float *o
     acc.y *= inv;
     acc.z *= inv;
     acc.w *= inv;
+    if (!live) continue;
     if (out_is_bf16) {
       uint2 pk = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
       *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(out) + (size_t)row * D + d0) = pk;

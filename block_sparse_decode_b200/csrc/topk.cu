@@ -2,9 +2,9 @@
 // block index asc), written in ascending block order and padded with -1.
 //
 // Page "Qwen 4 QSA gets decode context parallelism" (orcarouter.ai), section
-// "What the pull request actually changes": the indexer "keeps the best 512
-// blocks, roughly 2,048 token positions". The lower-index tie-break and the
-// ascending output order are this library's reading.
+// "What the pull request actually changes": the indexer retains the top 512
+// micro-blocks of a sequence (near 2,048 tokens). The lower-index tie-break
+// and the ascending output order are this library's reading.
 //
 // Design: one thread-block cluster of 8 CTAs per sequence. Each CTA holds a
 // contiguous eighth of the sequence's scores in shared memory as

@@ -4,14 +4,14 @@
  * The library computes one decode step of Qwen Sparse Attention (QSA) as
  * described on the page "Qwen 4 QSA gets decode context parallelism: inside
  * vLLM's draft PR for Qwen3.8-Flash-Next" (orcarouter.ai), section "What the
- * pull request actually changes": a lightweight indexer compresses keys
- * into micro-blocks at ratio 4, scores the blocks and keeps the best 512
- * (about 2,048 token positions); the final softmax and value aggregation run
- * on the uncompressed K and V. The decode-context-parallel split read of the
- * same section (each slice of the main KV cache read on its own, the
- * selector replicated, partial results combined afterwards; also "Questions
- * worth answering directly", DCP vs TP) is done inside one GPU as an R-way
- * split with a log-sum-exp merge.
+ * pull request actually changes": a small indexer shrinks the keys four to
+ * one into micro-blocks, ranks the blocks and retains the top 512 of them
+ * (near 2,048 tokens); exact attention (softmax, then the weighted sum of V)
+ * uses the full-precision K and V of the retained blocks only. The
+ * decode-context-parallel split read of the same section (each part of the
+ * main KV cache read on its own, the selector replicated, partial results
+ * combined afterwards; also "Questions worth answering directly", DCP vs TP)
+ * is done inside one GPU as an R-way split with a log-sum-exp merge.
  *
  * The page gives no formulas; this library fixes these readings:
  *   micro-block key   kc = bf16_rne(fp32 sum of its n keys in token order / n)
@@ -151,7 +151,7 @@ qsa_status qsa_index_score(const qsa_dims *dims, const qsa_cache *cache,
 size_t qsa_topk_workspace_size(int32_t B, int32_t ld_scores, int32_t k);
 
 /* Per-sequence top-k blocks (page section "What the pull request actually
- * changes": "keeps the best 512 blocks").
+ * changes": the indexer retains the top 512 blocks).
  *   scores  fp32 [B, ld_scores] (first nb_b = ceil(seq_lens[b]/4) entries
  *           used; NaN scores are not supported)
  *   sel     int32 [B, k]: the k_b = min(k, nb_b) best blocks by (score
@@ -242,7 +242,7 @@ qsa_status qsa_sparse_decode_static(const qsa_dims *dims, const qsa_cache *cache
                                     qsa_stream_t stream);
 
 /* Decode context parallelism (page section "What the pull request actually
- * changes": each rank reads only its slice of the main KV cache, the
+ * changes": a rank reads just its own part of the main KV cache, the
  * selector stays replicated; "Questions worth answering directly": partial
  * attention results are merged afterwards). This library's reading of a
  * rank's slice: page p of every sequence is held by rank p mod W (balanced,

@@ -9,10 +9,10 @@ It is a plain, slow restatement of what the decode step computes, written
 from the page "Qwen 4 QSA gets decode context parallelism: inside vLLM's
 draft PR for Qwen3.8-Flash-Next" (orcarouter.ai):
 
-* section "What the pull request actually changes", QSA paragraph: an
-  indexer compresses keys into micro-blocks at ratio 4, scores the blocks and
-  keeps the best 512 (about 2,048 tokens); the final softmax and value
-  aggregation run on the uncompressed K and V;
+* section "What the pull request actually changes", QSA paragraph: a small
+  indexer shrinks the keys four to one into micro-blocks, ranks the blocks
+  and retains the top 512 (near 2,048 tokens); exact attention (softmax and
+  the weighted sum of V) then uses the full-precision K and V of those blocks;
 * same section, first bullet and the DCP paragraph: each rank reads only its
   slice of the main KV cache, the selector stays replicated, and the partial
   attention results are combined after the split read (also the answer on

@@ -178,10 +178,15 @@ def test_topk_many_rows_long_score_rows_use_clusters():
 
 # ------------------------------------------------------------ merge alone
 
-@pytest.mark.parametrize("R,out_bf16", [(1, True), (2, False), (5, True), (64, False)])
-def test_merge_matches_oracle(R, out_bf16):
-    g = np.random.default_rng(R)
-    B, Hq, D = 3, 32, 128
+@pytest.mark.parametrize("R,out_bf16,D", [(1, True, 128), (2, False, 128), (5, True, 128),
+                                          (64, False, 128),
+                                          # head dims that are not a multiple of 128: some
+                                          # lanes of the row's warp own no dims in a pass
+                                          (3, True, 64), (9, False, 192), (2, False, 4),
+                                          (33, True, 260)])
+def test_merge_matches_oracle(R, out_bf16, D):
+    g = np.random.default_rng(R * 1000 + D)
+    B, Hq = 3, 32
     O = g.standard_normal((R, B, Hq, D)).astype(np.float32)
     LSE = (3 * g.standard_normal((R, B, Hq))).astype(np.float32)
     LSE[R // 2, 1, :5] = -np.inf

@@ -51,10 +51,8 @@ def _check_rows(wl, chunks, rows_to_check, row_start, q, q_idx, w, buf, k, R):
         check_selection(sel[r], ref["sel"], ref["scores"], k, what=f"row {r}")
         check_attention(o_part[:, r], lse_part[:, r], ref["O_part"], ref["LSE_part"],
                         what=f"row {r} partials")
-        # bf16 output: the bar plus the output's own rounding
-        o_ref, l_ref = ref["O"], ref["LSE"]
-        assert np.abs(out[r] - o_ref).max() <= 1e-2 + np.abs(o_ref).max() * 2.0 ** -8, r
-        assert np.abs(lse[r] - l_ref).max() <= 1e-3, r
+        # the merged bf16 output is held to the same bar as every other output
+        check_attention(out[r], lse[r], ref["O"], ref["LSE"], what=f"row {r} merged")
 
 
 @pytest.mark.parametrize("dims,lens,chunks,k,R", [

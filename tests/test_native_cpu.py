@@ -1,7 +1,7 @@
 """Host-only native checks (no GPU): the tcgen05 descriptor bit packing used
 by the scoring kernel equals CUTLASS/CuTe's bitfield definitions."""
 
-import glob
+import importlib.util
 import os
 import shutil
 import subprocess
@@ -12,11 +12,18 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def _cutlass_include():
-    for pat in ("/opt/prime-rl/.venv/lib/python3*/site-packages/flashinfer/data/cutlass/include",
-                "/opt/prime-rl/.venv/lib/python3*/site-packages/tilelang/3rdparty/cutlass/include"):
-        for d in glob.glob(pat):
-            if os.path.exists(os.path.join(d, "cute", "arch", "mma_sm100_desc.hpp")):
-                return d
+    """CUTLASS/CuTe headers: $CUTLASS_INCLUDE, else a copy vendored inside an
+    installed Python package (found through the import system, not a path)."""
+    cands = [os.environ.get("CUTLASS_INCLUDE", "")]
+    for pkg, sub in (("flashinfer", ("data", "cutlass", "include")),
+                     ("tilelang", ("3rdparty", "cutlass", "include"))):
+        spec = importlib.util.find_spec(pkg)
+        if spec is not None and spec.submodule_search_locations:
+            for loc in spec.submodule_search_locations:
+                cands.append(os.path.join(loc, *sub))
+    for d in cands:
+        if d and os.path.exists(os.path.join(d, "cute", "arch", "mma_sm100_desc.hpp")):
+            return d
     return None
 
 

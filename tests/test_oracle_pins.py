@@ -466,6 +466,31 @@ def test_owned_blocks_partition_the_selection(W, P):
         assert np.all(((4 * live) // P) % W == r)      # by its page
 
 
+def test_owned_blocks_hand():
+    for case in golden("owned_blocks_hand.json")["cases"]:
+        sel = np.asarray(case["sel"], dtype=np.int64)
+        for r in range(case["W"]):
+            got = oracle.owned_blocks(sel, case["P"], case["W"], r)
+            assert got.tolist() == case["owned"][r], (case["derivation"], r)
+
+
+def test_owned_blocks_fixture_catches_plausible_mistakes():
+    # the hand fixture would reject an owner rule that ranks by block index,
+    # or that forgets the 4 tokens per block when finding the page
+    wrong_rules = [lambda j, P, W: j % W,
+                   lambda j, P, W: (j // P) % W,
+                   lambda j, P, W: ((4 * j) // P) % (W + 1)]
+    for rule in wrong_rules:
+        caught = False
+        for case in golden("owned_blocks_hand.json")["cases"]:
+            P, W = case["P"], case["W"]
+            for r in range(W):
+                own = [j for j in case["sel"] if j >= 0 and rule(j, P, W) == r]
+                if own + [-1] * (len(case["sel"]) - len(own)) != case["owned"][r]:
+                    caught = True
+        assert caught
+
+
 def test_context_parallel_merge_equals_single_rank_attention():
     # each rank attends over its own pages' share of the one selection; the
     # LSE-weighted merge of the W partials is the attention over all of it
