@@ -55,6 +55,9 @@ def parse():
     ap.add_argument("--R", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the other workloads (b32x32k, steady128x64k k-sweep, "
+                         "ragged64 R-sweep) timed after the headline step")
     ap.add_argument("--dcp-world", type=int, default=0,
                     help="also time, on this GPU, rank 0's share of a decode-context-parallel "
                          "step over this many ranks (page p on rank p mod W)")
@@ -184,6 +187,191 @@ def algorithmic_bytes(seq_lens, dims, k):
     return side, kv
 
 
+def kernel_nodes(graph) -> int | None:
+    """Kernel nodes of a captured CUDA graph (None if the graph is not kept)."""
+    try:
+        import cuda.bindings.runtime as rt
+        raw = graph.raw_cuda_graph()
+        err, _, n = rt.cudaGraphGetNodes(raw, 0)
+        err, nodes, n = rt.cudaGraphGetNodes(raw, n)
+        if int(err) != 0:
+            return None
+        kern = 0
+        for nd in nodes:
+            e, t = rt.cudaGraphNodeGetType(nd)
+            if int(e) == 0 and t == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel:
+                kern += 1
+        return kern
+    except Exception:
+        return None
+
+
+class GraphTimer:
+    """CUDA graphs of library calls, replayed after an L2 flush and timed with
+    CUDA events on the launching stream."""
+
+    def __init__(self, dev, stream):
+        self.dev, self.stream = dev, stream
+        # write a buffer larger than L2, then read another one: the timed
+        # launch starts with a cold L2 that holds no dirty lines (otherwise the
+        # flush's own write-backs would be billed to the first kernels)
+        self.flush_w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        self.flush_r = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+        self.flush_o = torch.empty((), dtype=torch.float32, device=dev)
+        self.e0 = torch.cuda.Event(enable_timing=True)
+        self.e1 = torch.cuda.Event(enable_timing=True)
+
+    def capture(self, fn):
+        try:
+            g = torch.cuda.CUDAGraph(keep_graph=True)
+        except TypeError:
+            g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=self.stream):
+            fn()
+        return g
+
+    def flush(self):
+        self.flush_w.zero_()
+        torch.sum(self.flush_r, dim=0, out=self.flush_o)
+
+    def timed(self, g) -> float:
+        with torch.cuda.stream(self.stream):
+            self.flush()
+            self.e0.record()
+            g.replay()
+            self.e1.record()
+        self.e1.synchronize()
+        return self.e0.elapsed_time(self.e1)
+
+    def mean_ms(self, g, n: int, warm: int = 3) -> float:
+        for _ in range(warm):
+            self.timed(g)
+        return statistics.mean(self.timed(g) for _ in range(n))
+
+
+def prepare_batch(qsa, dims_spec, lens, k, R, seed, dev, spec, name, Qn=1):
+    """Draw a workload, fill its paged cache with every token but the step's
+    Qn newest (one bulk qsa_append) and allocate the step's buffers. Returns
+    (wl, dims, cache, step inputs, buffers)."""
+    from synth import make_custom
+    wl = make_custom(dims_spec, lens, k=k, R=R, seed=seed, device=dev, paged=spec["paged"],
+                     needles=spec["needles"], mixture=spec["mixture"], name=name)
+    dims = qsa.QsaDims.of(wl.dims)
+    B = wl.B
+    cache = qsa.alloc_cache(dims, wl.num_pages, wl.block_table, device=dev)
+    T = sum(wl.cap_lens)
+    tok_seq = torch.empty(T, dtype=torch.int32, device=dev)
+    tok_pos = torch.empty(T, dtype=torch.int32, device=dev)
+    for b, L in enumerate(wl.cap_lens):
+        o = wl.tok_off[b]
+        tok_seq[o:o + L] = b
+        tok_pos[o:o + L] = torch.arange(L, dtype=torch.int32, device=dev)
+        tok_seq[o + wl.seq_lens[b] - Qn:o + L] = -1
+    qsa.qsa_append(dims, cache, tok_seq, tok_pos, wl.k_tok, wl.v_tok, wl.kidx_tok)
+    del tok_seq, tok_pos
+    rows = torch.tensor([wl.tok_off[b] + L - Qn + j for b, L in enumerate(wl.seq_lens)
+                         for j in range(Qn)], device=dev)
+    if Qn == 1:
+        q_step = wl.q.contiguous()
+    else:  # one decode query per new token
+        gq = torch.Generator(device=dev).manual_seed(seed + 17)
+        q_step = torch.randn((B, Qn, wl.dims.Hq, wl.dims.D), generator=gq,
+                             device=dev).to(torch.bfloat16)
+    step_in = dict(
+        tok_seq=torch.arange(B, dtype=torch.int32, device=dev).repeat_interleave(Qn),
+        tok_pos=torch.tensor([L - Qn + j for L in wl.seq_lens for j in range(Qn)],
+                             dtype=torch.int32, device=dev),
+        k_new=wl.k_tok[rows].contiguous(), v_new=wl.v_tok[rows].contiguous(),
+        kidx_new=wl.kidx_tok[rows].contiguous(),
+        seq_lens=torch.tensor(wl.seq_lens, dtype=torch.int32, device=dev),
+        q=q_step, q_idx=wl.q_idx.contiguous(), w=wl.w.contiguous())
+    buf = qsa.alloc_step(dims, B, qsa.ld_for(wl.seq_lens), k, R, device=dev)
+    return wl, dims, cache, step_in, buf
+
+
+def time_batch(qsa, timer, dims, cache, si, buf, k, R, n_rep):
+    """The one-call step and the calls of the step, each in its own graph;
+    also index score + sparse decode back to back in one graph. Returns
+    ({name: mean us}, kernel nodes of the step graph)."""
+    app = (si["tok_seq"], si["tok_pos"], si["k_new"], si["v_new"], si["kidx_new"])
+    step_buf = qsa.StepBuffers(scores=buf.scores, sel=buf.sel, o_part=buf.o_part,
+                               lse_part=buf.lse_part, out=buf.out, lse=buf.lse, ws=buf.ws)
+
+    def step():
+        qsa.decode_step(dims, cache, si["seq_lens"], si["q"], si["q_idx"], si["w"], k, R,
+                        step_buf, append=app)
+
+    def score():
+        qsa.qsa_index_score(dims, cache, si["seq_lens"], si["q_idx"], si["w"], buf.scores)
+
+    def decode():
+        qsa.qsa_sparse_decode(dims, cache, si["seq_lens"], si["q"], buf.sel, k, R, buf.o_part,
+                              buf.lse_part, buf.ws)
+
+    calls = {"step": step, "index_score": score,
+             "topk_select": lambda: qsa.qsa_topk_select(si["seq_lens"], buf.scores, k, buf.sel),
+             "sparse_decode": decode,
+             "score_then_decode": lambda: (score(), decode())}
+    with torch.cuda.stream(timer.stream):
+        for _ in range(2):
+            step()
+    torch.cuda.synchronize(timer.dev)
+    qsa.qsa_check_device_errors()
+    graphs = {n: timer.capture(fn) for n, fn in calls.items()}
+    nodes = kernel_nodes(graphs["step"])
+    us = {n: 1e3 * timer.mean_ms(g, n_rep) for n, g in graphs.items()}
+    qsa.qsa_check_device_errors()
+    for g in graphs.values():
+        g.reset()
+    return us, nodes
+
+
+def config_line(name, lens, dims, k, R, us, peak):
+    side_b, kv_b = algorithmic_bytes(lens, dims, k)
+    pair = us["index_score"] + us["sparse_decode"]
+    return {
+        "workload": name, "batch": len(lens), "k": k, "R": R,
+        "step_us": us["step"], "seqs_per_s": len(lens) / (us["step"] * 1e-6),
+        "attended_tokens_per_s": sum(min(4 * k, L) for L in lens) / (us["step"] * 1e-6),
+        "kernels_us": {n: us[n] for n in ("index_score", "topk_select", "sparse_decode")},
+        "bytes": {"side_cache": side_b, "selected_kv": kv_b},
+        "index_score_frac": side_b / (us["index_score"] * 1e-6) / 1e9 / peak,
+        "sparse_decode_frac": kv_b / (us["sparse_decode"] * 1e-6) / 1e9 / peak,
+        "score_plus_decode_frac": (side_b + kv_b) / (pair * 1e-6) / 1e9 / peak,
+        "score_then_decode_one_graph_us": us["score_then_decode"],
+        "score_then_decode_one_graph_frac":
+            (side_b + kv_b) / (us["score_then_decode"] * 1e-6) / 1e9 / peak,
+        "step_frac": (side_b + kv_b) / (us["step"] * 1e-6) / 1e9 / peak,
+    }
+
+
+def time_configs(args, qsa, timer, dev, peak):
+    """The other workloads of the scope, each at its full size: b32x32k,
+    steady128x64k (one step at L = 65,537, k in {256, 512, 1024}) and ragged64
+    (R in {1, 2, 4, 8}); same graphs, flush and events as the headline."""
+    from synth import preset_spec, seed_for
+    out = {}
+    n_rep = max(10, min(args.steps, 50))
+    plan = [("b32x32k", None, [(512, 1)]),
+            ("steady128x64k", [65537] * 128, [(256, 4), (512, 4), (1024, 4)]),
+            ("ragged64", None, [(512, 1), (512, 2), (512, 4), (512, 8)])]
+    for name, lens, kr in plan:
+        spec = preset_spec(name)
+        lens = lens or list(spec["seq_lens"])
+        k0, R0 = kr[0]
+        wl, dims, cache, si, buf = prepare_batch(qsa, spec["dims"], lens, k0, R0,
+                                                 seed_for(name), dev, spec, name)
+        del wl.k_tok, wl.v_tok, wl.kidx_tok
+        for k, R in kr:
+            buf = qsa.alloc_step(dims, len(lens), qsa.ld_for(lens), k, R, device=dev)
+            us, _ = time_batch(qsa, timer, dims, cache, si, buf, k, R, n_rep)
+            out[f"{name}_k{k}_R{R}"] = config_line(name, lens, dims, k, R, us, peak)
+            del buf
+        del wl, cache, si
+        torch.cuda.empty_cache()
+    return out
+
+
 # ------------------------------------------------------------ our arm
 
 def run_ours(args, rank, world, local_rank):
@@ -296,13 +484,20 @@ def run_ours(args, rank, world, local_rank):
     qsa.qsa_check_device_errors()
 
     def capture(fn):
-        g = torch.cuda.CUDAGraph()
+        try:  # keep the graph so that its kernel nodes can be counted
+            g = torch.cuda.CUDAGraph(keep_graph=True)
+        except TypeError:
+            g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
             fn()
         return g
 
     graph = capture(step)
+    step_kernels = kernel_nodes(graph)
     kgraphs = {n: capture(fn) for n, fn in calls.items()}
+    if Qn == 1:  # the two HBM-bound calls back to back, one launch of the pair
+        kgraphs["score_then_decode"] = capture(lambda: (calls["index_score"](),
+                                                        calls["sparse_decode"]()))
     # L2 flush: write a buffer larger than L2, then read another one, so the
     # timed step starts with a cold L2 that holds no dirty lines (otherwise
     # the flush's own write-backs would be billed to the first kernels)
@@ -391,6 +586,15 @@ def run_ours(args, rank, world, local_rank):
         prefill_res = time_prefill(args, qsa, wl, dims, cache, si["seq_lens"], k, R, ld, dev,
                                    capture, timed)
 
+    # the other workloads of the scope (their own caches; the headline's
+    # buffers stay allocated, every config frees its own)
+    configs = None
+    if not args.no_configs and Qn == 1 and world == 1 and not args.batch:
+        timer = GraphTimer(dev, stream)
+        peak_c, _ = load_peaks()
+        configs = time_configs(args, qsa, timer, dev, peak_c)
+        del timer
+
     # e2e: host buffers in pinned memory, copies inside the timed region,
     # calls made eagerly through the binding (the user's API)
     e2e = None
@@ -447,15 +651,9 @@ def run_ours(args, rank, world, local_rank):
     achieved = side_b / (score_ms / 1e3) / 1e9
     traffic = profile_traffic("index_score.cu", "index_score_b8x256k.md")
     attended = Qn * sum(min(4 * k, L) for L in wl.seq_lens)
-    # kernels per step: append, score, top-k, merge, and per group of two
-    # queries the decode plus (when sequences are split over CTAs) its combine
-    nhg = (dims.Hkv + 3) // 4
-    ntmax = (k + 3) // 4 + R - 1
-    ncb = max(1, min(296 // (B * nhg), ntmax), -(-ntmax // 256))
-    if Qn == 1:  # append, score, top-k, decode, then the combine (merging) or the merge
-        launches = 5
-    else:
-        launches = 4 + ((Qn + 1) // 2) * (2 if ncb > 1 else 1)
+    # kernels per step: the kernel nodes of the captured step graph (every
+    # node is one of the library's kernels: the step is library calls only)
+    launches = step_kernels if step_kernels is not None else 0
     res = {
         "metric": METRIC,
         "value": job_rate(world, B, ms_per_step),
@@ -496,9 +694,18 @@ def run_ours(args, rank, world, local_rank):
             "bytes": side_b + kv_b,
             "us": 1e3 * (score_ms + dec_ms),
             "gbs": (side_b + kv_b) / ((score_ms + dec_ms) / 1e3) / 1e9,
-            "frac": (side_b + kv_b) / ((score_ms + dec_ms) / 1e3) / 1e9 / peak},
+            "frac": (side_b + kv_b) / ((score_ms + dec_ms) / 1e3) / 1e9 / peak,
+            "timing": "sum of the two calls, each alone in its own graph",
+            **({"one_graph_us": 1e3 * kern_ms["score_then_decode"],
+                "one_graph_frac": (side_b + kv_b) / (kern_ms["score_then_decode"] / 1e3)
+                / 1e9 / peak,
+                "one_graph_timing": "the two calls back to back in one graph (the decode "
+                                    "reads the step's selection)"}
+               if "score_then_decode" in kern_ms else {})},
+        "sparse_decode_frac": kv_b / (dec_ms / 1e3) / 1e9 / peak,
         "step_roofline_frac": (side_b + kv_b) / (ms_per_step / 1e3) / 1e9 / peak,
         "gpu_launches": launches * args.steps,
+        "kernels_per_step": launches,
         "clocks": clk.summary(),
         "e2e": e2e,
     }
@@ -506,6 +713,8 @@ def run_ours(args, rank, world, local_rank):
         res["dcp_emulated"] = dcp_res
     if prefill_res is not None:
         res["prefill"] = prefill_res
+    if configs is not None:
+        res["configs"] = configs
     graph.reset()
     for g in kgraphs.values():
         g.reset()
@@ -554,7 +763,17 @@ def time_prefill(args, qsa, wl, dims, cache, seq_lens, k, R, ld, dev, capture, t
         g.reset()
     lens = [L - T + i + 1 for L in wl.seq_lens for i in range(T)]
     flops = 2.0 * dims.Hi * dims.di * sum(ell // 4 for ell in lens)
-    kv = sum(min(4 * k, ell) for ell in lens) * dims.Hkv * dims.D * 2 * 2
+    kv_rows = sum(min(4 * k, ell) for ell in lens) * dims.Hkv * dims.D * 2 * 2
+    # the rows of a sequence share most of their selected blocks: the bytes
+    # that must come from HBM are the K/V of the union of its rows' selections
+    sel = pb.sel.cpu().numpy()
+    rs = row_start.cpu().tolist()
+    union_tokens = 0
+    for s_, L in enumerate(wl.seq_lens):
+        blocks = np.unique(sel[rs[s_]:rs[s_ + 1]])
+        blocks = blocks[blocks >= 0].astype(np.int64)
+        union_tokens += int(np.minimum(4, L - 4 * blocks).sum())
+    kv = union_tokens * dims.Hkv * dims.D * 2 * 2
     tpk, tpk_src = load_tensor_peak()
     hbm, hbm_src = load_peaks()
     s_tf = flops / (us["prefill_index_score"] * 1e-6) / 1e12
@@ -576,8 +795,9 @@ def time_prefill(args, qsa, wl, dims, cache, seq_lens, k, R, ld, dev, capture, t
             "prefill_sparse_decode": {"bound": "hbm", "achieved": d_gb, "peak": hbm,
                                       "unit": "GB/s", "frac": d_gb / hbm,
                                       "peak_source": hbm_src, "algorithmic_bytes": kv,
-                                      "note": "rows of a sequence share selected blocks "
-                                              "through L2, so frac can exceed 1"},
+                                      "bytes_definition": "K/V of the union of each "
+                                                          "sequence's rows' selected blocks",
+                                      "bytes_per_row_sum": kv_rows},
         },
     }
 

@@ -204,9 +204,6 @@ qsa_status qsa_index_score(const qsa_dims *dims, const qsa_cache *cache, int32_t
     if (B > 0 && (seq_lens == nullptr || q_idx == nullptr || w == nullptr || scores == nullptr))
       return fail(QSA_ERR_INVALID_ARG, "an argument array is NULL");
     if (B > 0 && !aligned16(q_idx)) return fail(QSA_ERR_INVALID_ARG, "q_idx not 16-byte aligned");
-    if (!index_score_supported(*dims))
-      return fail(QSA_ERR_UNSUPPORTED,
-                  "qsa_index_score needs the page size P to be a power of two in [32, 1024]");
     QSA_ERRWORD(err);
     return cuda_status(launch_index_score(*dims, *cache, B, seq_lens, q_idx, w, scores, ld_scores,
                                           err, reinterpret_cast<cudaStream_t>(stream)),
@@ -280,12 +277,12 @@ qsa_status qsa_sparse_decode_mq(const qsa_dims *dims, const qsa_cache *cache, in
     if (R < 1 || R > 64) return fail(QSA_ERR_UNSUPPORTED, "R=%d outside [1, 64]", R);
     if (B == 0) return ok();
     if (seq_lens == nullptr || q == nullptr || sel == nullptr || o_part == nullptr ||
-        lse_part == nullptr || ws == nullptr)
+        lse_part == nullptr)
       return fail(QSA_ERR_INVALID_ARG, "an argument array is NULL");
     if (!aligned16(q) || !aligned16(o_part) || !aligned16(ws))
       return fail(QSA_ERR_INVALID_ARG, "q / o_part / ws not 16-byte aligned");
     const size_t need = decode_ws_bytes(*dims, B, Qn, k, R);
-    if (ws_bytes < need)
+    if (need > 0 && (ws == nullptr || ws_bytes < need))
       return fail(QSA_ERR_INVALID_ARG, "workspace %zu bytes < %zu needed", ws_bytes, need);
     QSA_ERRWORD(err);
     return cuda_status(launch_sparse_decode(*dims, *cache, B, Qn, seq_lens, q, sel, k, R, o_part,
@@ -365,13 +362,13 @@ qsa_status qsa_decode_step(const qsa_dims *dims, const qsa_cache *cache, int32_t
       if (R < 1 || R > 64) return fail(QSA_ERR_UNSUPPORTED, "R=%d outside [1, 64]", R);
       if (B == 0) return ok();
       if (seq_lens == nullptr || q == nullptr || sel == nullptr || o_part == nullptr ||
-          lse_part == nullptr || ws == nullptr || out == nullptr)
+          lse_part == nullptr || out == nullptr)
         return fail(QSA_ERR_INVALID_ARG, "an argument array is NULL");
       if (!aligned16(q) || !aligned16(o_part) || !aligned16(ws) ||
           (reinterpret_cast<uintptr_t>(out) & 7u) != 0)
         return fail(QSA_ERR_INVALID_ARG, "q / o_part / ws not 16-byte or out not 8-byte aligned");
       const size_t need = decode_ws_bytes(*dims, B, 1, k, R);
-      if (ws_bytes < need)
+      if (need > 0 && (ws == nullptr || ws_bytes < need))
         return fail(QSA_ERR_INVALID_ARG, "workspace %zu bytes < %zu needed", ws_bytes, need);
       QSA_ERRWORD(err);
       st = cuda_status(launch_sparse_decode(*dims, *cache, B, 1, seq_lens, q, sel, k, R, o_part,
@@ -407,7 +404,7 @@ qsa_status qsa_prefill_index_score(const qsa_dims *dims, const qsa_cache *cache,
     if (!prefill_supported(*dims))
       return fail(QSA_ERR_UNSUPPORTED,
                   "qsa_prefill_index_score needs Hi in {4, 8, 16, 32} and the page size P a "
-                  "power of two in [32, 1024]");
+                  "multiple of 32");
     if (S == 0 || Nq == 0) return ok();
     if (seq_lens == nullptr || row_start == nullptr || q_idx == nullptr || w == nullptr ||
         scores == nullptr || row_len == nullptr || ws == nullptr)
@@ -443,12 +440,12 @@ qsa_status qsa_prefill_sparse_decode(const qsa_dims *dims, const qsa_cache *cach
     if (R < 1 || R > 64) return fail(QSA_ERR_UNSUPPORTED, "R=%d outside [1, 64]", R);
     if (S == 0 || Nq == 0) return ok();
     if (seq_lens == nullptr || row_start == nullptr || q == nullptr || sel == nullptr ||
-        o_part == nullptr || lse_part == nullptr || ws == nullptr)
+        o_part == nullptr || lse_part == nullptr)
       return fail(QSA_ERR_INVALID_ARG, "an argument array is NULL");
     if (!aligned16(q) || !aligned16(o_part) || !aligned16(ws))
       return fail(QSA_ERR_INVALID_ARG, "q / o_part / ws not 16-byte aligned");
     const size_t need = decode_ws_bytes(*dims, Nq, 1, k, R);
-    if (ws_bytes < need)
+    if (need > 0 && (ws == nullptr || ws_bytes < need))
       return fail(QSA_ERR_INVALID_ARG, "workspace %zu bytes < %zu needed", ws_bytes, need);
     QSA_ERRWORD(err);
     return cuda_status(launch_sparse_decode(*dims, *cache, Nq, 1, seq_lens, q, sel, k, R, o_part,

@@ -38,9 +38,12 @@
 // Every mbarrier wait is bounded: on timeout the kernel sets the TIMEOUT bit,
 // stops all roles, drains what it issued (bounded) and frees TMEM.
 //
-// Supported: P a power of two in [32, 1024] (a page piece is a multiple of 8
-// rows, so every box starts on a 1 KiB swizzle atom, and pieces tile the 128
-// rows exactly), di in {64, 128}, Hi <= 32.
+// Page pieces: a tile's rows are cut into pieces of gcd(P/4, 128) rows, so a
+// piece never spans two pages and pieces tile the 128 rows exactly; with P a
+// multiple of 32 a piece is a multiple of 8 rows and every box starts on a
+// 1 KiB swizzle atom. Supported: P a multiple of 32 in [32, 1024], di in
+// {64, 128}, Hi <= 32; other page sizes (P a multiple of 4) are scored by the
+// warp-level MMA kernel of index_score_warp.cu.
 // Roofline: HBM-bound; algorithmic bytes = nb * di * 2 per sequence.
 #include <cuda.h>
 
@@ -71,7 +74,7 @@ struct TcArgs {
   const int32_t *block_table, *seq_lens;
   float *scores;
   int B, ld, P, rpp, max_pages, num_pages, Hi, stages;
-  int box;  // tile rows per page piece: min(P/4, 128)
+  int box;  // tile rows per page piece: gcd(P/4, 128)
   int ept;  // page pieces per tile: 128 / box
   int tpc;  // tiles per half of the shared page table
   unsigned *err;
@@ -204,9 +207,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     for (int til = warp - wfirst; til < ntiles; til += nwarps) {
       int b, j0;
       tile_start(chunk * a.tpc + til, b, j0);
-      const int col0 = j0 / a.rpp, nfull = lens[b] >> 2;
+      const int nfull = lens[b] >> 2;
       for (int k = lane; k < a.ept; k += 32) {
-        const int col = col0 + k;
+        const int col = (j0 + k * a.box) / a.rpp;  // a piece never spans two pages
         const bool live = (j0 + k * a.box) < nfull && col < a.max_pages;
         if ((j0 + k * a.box) < nfull && col >= a.max_pages) raise_err(a.err, ERR_BT);
         asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(
@@ -486,15 +489,28 @@ cudaError_t launch_tc_t(const qsa_cache &c, TcArgs a, cudaStream_t st) {
 
 }  // namespace
 
+int piece_rows(int rpp) {
+  int x = rpp, y = TC_M;  // gcd(rows per page, rows per tile)
+  while (y != 0) {
+    const int t = x % y;
+    x = y;
+    y = t;
+  }
+  return x;
+}
+
 bool index_score_supported(const qsa_dims &d) {
-  const bool pow2 = d.P >= 32 && d.P <= 1024 && (d.P & (d.P - 1)) == 0;
-  return pow2 && (d.di == 64 || d.di == 128) && d.Hi <= 32;
+  // a page piece of gcd(P/4, 128) rows must start on a 1 KiB swizzle atom
+  const bool pages = d.P >= 32 && d.P <= 1024 && d.P % 32 == 0;
+  return pages && (d.di == 64 || d.di == 128) && d.Hi <= 32;
 }
 
 cudaError_t launch_index_score(const qsa_dims &d, const qsa_cache &c, int B,
                                const int32_t *seq_lens, const void *q_idx, const float *w,
                                float *scores, int ld, unsigned *err, cudaStream_t st) {
   if (B == 0) return cudaSuccess;
+  if (!index_score_supported(d))  // page pieces off the swizzle atoms: warp-level MMA path
+    return launch_index_score_warp(d, c, B, seq_lens, q_idx, w, scores, ld, err, st);
   TcArgs a;
   a.kidx_pool = static_cast<const __nv_bfloat16 *>(c.kidx_pool);
   a.q_idx = static_cast<const __nv_bfloat16 *>(q_idx);
@@ -506,7 +522,7 @@ cudaError_t launch_index_score(const qsa_dims &d, const qsa_cache &c, int B,
   a.ld = ld;
   a.P = d.P;
   a.rpp = d.P / 4;
-  a.box = std::min(a.rpp, TC_M);
+  a.box = piece_rows(a.rpp);
   a.ept = TC_M / a.box;
   a.tpc = (TBL / 2) / a.ept;
   a.max_pages = c.max_pages_per_seq;

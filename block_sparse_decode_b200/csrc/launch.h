@@ -43,6 +43,10 @@ cudaError_t launch_append(const qsa_dims &d, const qsa_cache &c, int N, const in
                           const void *kidx_new, unsigned *err, cudaStream_t st);
 
 bool index_score_supported(const qsa_dims &d);  // page sizes the TMA gather can address
+// Scores through warp-level MMAs for any page size P (a multiple of 4).
+cudaError_t launch_index_score_warp(const qsa_dims &d, const qsa_cache &c, int B,
+                                    const int32_t *seq_lens, const void *q_idx, const float *w,
+                                    float *scores, int ld, unsigned *err, cudaStream_t st);
 cudaError_t launch_index_score(const qsa_dims &d, const qsa_cache &c, int B,
                                const int32_t *seq_lens, const void *q_idx, const float *w,
                                float *scores, int ld, unsigned *err, cudaStream_t st);

@@ -2,10 +2,10 @@
 // context-parallel group holds.
 //
 // Page "Qwen 4 QSA gets decode context parallelism" (orcarouter.ai), section
-// "What the pull request actually changes": with DCP each rank reads only its
-// slice of the main KV cache while the selector stays replicated, and the
-// partial attention results are merged afterwards ("Questions worth answering
-// directly"). This library's reading of the slice: page p of every sequence
+// "What the pull request actually changes": under DCP a rank reads just its
+// own part of the main KV cache, the selector is kept whole on every rank,
+// and the partial attention results are merged at the end ("Questions worth
+// answering directly"). This library's reading of the slice: page p of every sequence
 // is held by rank p mod W, so each rank keeps about 1/W of every sequence and
 // the split does not move as a sequence grows. Every rank scores and selects
 // on the replicated side cache; this kernel keeps the selected blocks whose

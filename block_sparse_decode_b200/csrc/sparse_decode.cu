@@ -2,10 +2,10 @@
 // R context slices that each give a partial output and its log-sum-exp.
 //
 // Page "Qwen 4 QSA gets decode context parallelism" (orcarouter.ai), section
-// "What the pull request actually changes": the final softmax and value
-// aggregation run on the uncompressed K and V of the kept blocks; under DCP
-// each rank reads only its slice of the main KV cache while the selector
-// stays replicated, and the attention results are combined afterwards. Here
+// "What the pull request actually changes": softmax attention over the kept
+// blocks uses their full-precision K and V; under DCP a rank reads just its
+// own part of the main KV cache, the selector is the same on every rank, and
+// the attention results are merged after the split read. Here
 // the slices are the block ranges [floor(r*nb/R), floor((r+1)*nb/R)) of one
 // GPU and the one selection serves all of them.
 //
@@ -91,6 +91,7 @@ struct DecodeArgs {
   int B, Hq, Hkv, G, P, max_pages, num_pages, k, k_pad, R, ncb, rb;
   int Qn, q0, qn;            // queries per sequence; first query and size of this group
   int ring_bytes;            // DV_WARPS * ST * DV_STAGE
+  int bt_smem;               // the block-table row (max_pages entries) is staged in the ring
   float scale_log2;
   unsigned *err;
 };
@@ -273,12 +274,26 @@ __global__ void __launch_bounds__(DV_WARPS * 32, DV_CTAS_PER_SM) sparse_decode_k
   int32_t *s_blk = s_row + DV_TBL_BLOCKS;         // its block index (-1: none)
   uint8_t *s_nv = reinterpret_cast<uint8_t *>(s_blk + DV_TBL_BLOCKS);  // its valid tokens
 
-  // (1) L_b, the block-table row into L2, the query; then, once the top-k
-  // kernel before this one has finished, the selection row
+  // (1) the block-table row (into shared memory when it fits the ring, which
+  // is idle until streaming starts; else into L2), L_b and the query: all
+  // inputs, so they are read before the wait on the top-k kernel; then the
+  // selection row
+  int32_t *s_bt = reinterpret_cast<int32_t *>(smem);
+  auto copy_bt_row = [&](int row) {
+    const int32_t *btr = a.block_table + (size_t)row * a.max_pages;
+    int i0 = 0;
+    if ((reinterpret_cast<uintptr_t>(btr) & 15u) == 0) {  // 16-byte pieces, then the tail
+      const int n4 = a.max_pages >> 2;
+      for (int i = tid; i < n4; i += blockDim.x) cp_async16(smem_u32(s_bt + 4 * i), btr + 4 * i, 16);
+      i0 = 4 * n4;
+    }
+    for (int i = i0 + tid; i < a.max_pages; i += blockDim.x) cp_async4(smem_u32(s_bt + i), btr + i);
+  };
   int bs = b;  // block-table row
   {
     int L;
     if (a.row_start == nullptr) {
+      if (a.bt_smem) copy_bt_row(b);
       L = a.seq_lens[b];
     } else {  // prefill row: the chunk holding it (every thread; S is small)
       int lo = 0, hi = a.S - 1;
@@ -297,12 +312,15 @@ __global__ void __launch_bounds__(DV_WARPS * 32, DV_CTAS_PER_SM) sparse_decode_k
       }
     }
     if (tid == 0) s_L = L;
-    // the CTAs of a sequence pull its block-table row into L2 together, so
-    // the page lookups after the slice search hit L2
-    const char *bt_row = reinterpret_cast<const char *>(a.block_table + (size_t)bs * a.max_pages);
-    const int lines = (a.max_pages * 4 + 127) >> 7;
-    for (int i = c + CL * tid; i < lines; i += CL * (int)blockDim.x)
-      asm volatile("prefetch.global.L2 [%0];\n" ::"l"(bt_row + ((size_t)i << 7)));
+    if (a.row_start != nullptr && a.bt_smem) copy_bt_row(bs);
+    if (!a.bt_smem) {
+      // the CTAs of a sequence pull its block-table row into L2 together, so
+      // the page lookups after the slice search hit L2
+      const char *bt_row = reinterpret_cast<const char *>(a.block_table + (size_t)bs * a.max_pages);
+      const int lines = (a.max_pages * 4 + 127) >> 7;
+      for (int i = c + CL * tid; i < lines; i += CL * (int)blockDim.x)
+        asm volatile("prefetch.global.L2 [%0];\n" ::"l"(bt_row + ((size_t)i << 7)));
+    }
   }
   // query fragments (B operand of S^T = K Q^T): query a.q0 + qq, head g*G + lane/4
   const int gq = lane >> 2, tq = lane & 3;
@@ -321,7 +339,13 @@ __global__ void __launch_bounds__(DV_WARPS * 32, DV_CTAS_PER_SM) sparse_decode_k
   pdl_wait();
   {
     const int32_t *srow = a.sel + (size_t)b * a.k;
-    for (int i = tid; i < a.k; i += blockDim.x) cp_async4(smem_u32(s_sel + i), srow + i);
+    int i0 = 0;
+    if ((reinterpret_cast<uintptr_t>(srow) & 15u) == 0) {  // 16-byte pieces, then the tail
+      const int n4 = a.k >> 2;
+      for (int i = tid; i < n4; i += blockDim.x) cp_async16(smem_u32(s_sel + 4 * i), srow + 4 * i, 16);
+      i0 = 4 * n4;
+    }
+    for (int i = i0 + tid; i < a.k; i += blockDim.x) cp_async4(smem_u32(s_sel + i), srow + i);
     cp_async_commit();
   }
   cp_async_wait<0>();
@@ -424,7 +448,10 @@ __global__ void __launch_bounds__(DV_WARPS * 32, DV_CTAS_PER_SM) sparse_decode_k
       }
     }
 #pragma unroll
-    for (int u = 0; u < 4; ++u) pg[u] = idx[u] >= 0 ? __ldg(a.block_table + idx[u]) : -1;
+    for (int u = 0; u < 4; ++u)
+      pg[u] = idx[u] < 0 ? -1
+              : a.bt_smem ? s_bt[idx[u] - (long long)bs * a.max_pages]
+                          : __ldg(a.block_table + idx[u]);
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int slot = base + tid + u * (int)blockDim.x;
@@ -754,6 +781,7 @@ cudaError_t launch_sparse_decode(const qsa_dims &d, const qsa_cache &c, int B, i
   a.rb = p.rb;
   a.Qn = Qn;
   a.ring_bytes = DV_WARPS * p.stages * DV_STAGE;
+  a.bt_smem = (size_t)c.max_pages_per_seq * 4 <= (size_t)a.ring_bytes ? 1 : 0;
   a.scale_log2 = d.scale * LOG2E;
   a.err = err;
   // query groups of up to DV_QGROUP, each one pass over the selected K/V

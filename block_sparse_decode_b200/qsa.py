@@ -116,6 +116,11 @@ def _stream(stream) -> int:
     return int(stream)
 
 
+def _nbytes(t: torch.Tensor | None) -> int:
+    """Size in bytes of an optional scratch tensor (0 for None)."""
+    return 0 if t is None else t.numel() * t.element_size()
+
+
 def _ptr(t: torch.Tensor | None, dtype=None, name="tensor") -> int | None:
     if t is None:
         return None
@@ -247,7 +252,7 @@ def qsa_sparse_decode(dims: QsaDims, cache: QsaCache, seq_lens, q, sel, k: int, 
                                    _ptr(q, torch.bfloat16, "q"), _ptr(sel, torch.int32, "sel"),
                                    int(k), int(R), _ptr(o_part, torch.float32, "o_part"),
                                    _ptr(lse_part, torch.float32, "lse_part"),
-                                   _ptr(ws, None, "ws"), ws.numel() * ws.element_size(),
+                                   _ptr(ws, None, "ws"), _nbytes(ws),
                                    _stream(stream)))
 
 
@@ -264,7 +269,7 @@ def qsa_sparse_decode_mq(dims: QsaDims, cache: QsaCache, seq_lens, q, sel, k: in
                                       _ptr(q, torch.bfloat16, "q"), _ptr(sel, torch.int32, "sel"),
                                       int(k), int(R), _ptr(o_part, torch.float32, "o_part"),
                                       _ptr(lse_part, torch.float32, "lse_part"),
-                                      _ptr(ws, None, "ws"), ws.numel() * ws.element_size(),
+                                      _ptr(ws, None, "ws"), _nbytes(ws),
                                       _stream(stream)))
 
 
@@ -363,7 +368,7 @@ def decode_step(dims: QsaDims, cache: QsaCache, seq_lens, q, q_idx, w, k: int, R
         _ptr(buf.scores, torch.float32, "scores"), int(buf.scores.shape[1]),
         _ptr(buf.sel, torch.int32, "sel"), _ptr(buf.o_part, torch.float32, "o_part"),
         _ptr(buf.lse_part, torch.float32, "lse_part"), _ptr(buf.ws, None, "ws"),
-        buf.ws.numel() * buf.ws.element_size(), _ptr(buf.out, None, "out"),
+        _nbytes(buf.ws), _ptr(buf.out, None, "out"),
         1 if buf.out.dtype == torch.bfloat16 else 0, _ptr(buf.lse, torch.float32, "lse"),
         _stream(stream)))
 
@@ -389,7 +394,7 @@ def qsa_prefill_index_score(dims: QsaDims, cache: QsaCache, seq_lens, row_start,
         _ptr(q_idx, torch.bfloat16, "q_idx"), _ptr(w, torch.float32, "w"),
         _ptr(scores, torch.float32, "scores"), int(scores.shape[1]),
         _ptr(row_len, torch.int32, "row_len"), _ptr(ws, None, "ws"),
-        ws.numel() * ws.element_size(), _stream(stream)))
+        _nbytes(ws), _stream(stream)))
 
 
 def qsa_prefill_sparse_decode(dims: QsaDims, cache: QsaCache, seq_lens, row_start, q, sel,
@@ -401,7 +406,7 @@ def qsa_prefill_sparse_decode(dims: QsaDims, cache: QsaCache, seq_lens, row_star
         _ptr(seq_lens, torch.int32, "seq_lens"), _ptr(row_start, torch.int32, "row_start"), Nq,
         _ptr(q, torch.bfloat16, "q"), _ptr(sel, torch.int32, "sel"), int(k), int(R),
         _ptr(o_part, torch.float32, "o_part"), _ptr(lse_part, torch.float32, "lse_part"),
-        _ptr(ws, None, "ws"), ws.numel() * ws.element_size(), _stream(stream)))
+        _ptr(ws, None, "ws"), _nbytes(ws), _stream(stream)))
 
 
 def qsa_sparse_prefill_workspace_size(dims: QsaDims, S: int, Nq: int, k: int, R: int) -> int:
@@ -450,6 +455,6 @@ def sparse_prefill(dims: QsaDims, cache: QsaCache, seq_lens, row_start, q, q_idx
         int(buf.scores.shape[1]), _ptr(buf.row_len, torch.int32, "row_len"),
         _ptr(buf.sel, torch.int32, "sel"), _ptr(buf.o_part, torch.float32, "o_part"),
         _ptr(buf.lse_part, torch.float32, "lse_part"), _ptr(buf.ws, None, "ws"),
-        buf.ws.numel() * buf.ws.element_size(), _ptr(buf.out, None, "out"),
+        _nbytes(buf.ws), _ptr(buf.out, None, "out"),
         1 if buf.out.dtype == torch.bfloat16 else 0, _ptr(buf.lse, torch.float32, "lse"),
         _stream(stream)))

@@ -73,8 +73,8 @@ typedef struct CUstream_st *qsa_stream_t;
  *   Hi  indexer heads                     supported: 1..32
  *   di  indexer key width                 supported: 64, 128
  *   P   tokens per cache page             supported: multiple of 4, 4..1024
- *                                         (qsa_index_score: power of two,
- *                                         32..1024)
+ *                                         (qsa_prefill_index_score: multiple
+ *                                         of 32)
  *   G = Hq/Hkv                            supported: 1..8
  *   scale  softmax scale applied to q.K (e.g. 1/sqrt(D)). */
 typedef struct qsa_dims {
@@ -139,9 +139,10 @@ qsa_status qsa_append(const qsa_dims *dims, const qsa_cache *cache, int32_t N,
  *             sequence sets QSA_ERR_BOUNDS and is skipped). Entries
  *             j >= nb_b are not written.
  * Complete blocks read the side pool; the trailing partial block's key is
- * built from its L mod 4 tokens in kidx_pool by the same rule. Needs P a
- * power of two in [32, 1024] (else QSA_ERR_UNSUPPORTED) and q_idx 16-byte
- * aligned. */
+ * built from its L mod 4 tokens in kidx_pool by the same rule. Any page size
+ * P (a multiple of 4) is scored: P a multiple of 32 by the TMA + tcgen05
+ * kernel, other page sizes by a warp-level MMA kernel that gathers the
+ * side-cache rows one by one. Needs q_idx 16-byte aligned. */
 qsa_status qsa_index_score(const qsa_dims *dims, const qsa_cache *cache,
                            int32_t B, const int32_t *seq_lens,
                            const void *q_idx, const float *w, float *scores,

@@ -90,8 +90,6 @@ def test_host_side_argument_checks(L):
         D(32, 4, 128, 33, 128, 64, 0.1),   # Hi > 32
         D(32, 2, 128, 16, 128, 64, 0.1),   # G = 16 > 8
         D(32, 4, 128, 16, 128, 62, 0.1),   # P % 4
-        D(32, 4, 128, 16, 128, 16, 0.1),   # scoring needs P a power of two >= 32
-        D(32, 4, 128, 16, 128, 96, 0.1),   # ... and a power of two
     ]
     c = qsa._Cache(16, 16, 16, 16, 16, 1, 1, 1)
     for d in bad:

@@ -80,6 +80,14 @@ def test_ragged_paged_full_heads(R):
     (Dims(Hq=12, Hkv=2, D=128, Hi=24, di=128, P=128, scale=0.09), [4096, 515, 6000], 100),
     (Dims(Hq=2, Hkv=1, D=128, Hi=1, di=128, P=1024, scale=0.2), [33, 2570], 7),
     (Dims(Hq=16, Hkv=2, D=128, Hi=32, di=64, P=64, scale=0.088), [1500, 2600], 1),
+    # page sizes that are not powers of two: P = 96 (a multiple of 32, the
+    # tensor-core kernel with 8-row page pieces), P = 16 and 48 (the
+    # warp-level kernel that gathers side-cache rows one by one), and P = 4
+    # (one micro-block per page)
+    (Dims(Hq=32, Hkv=4, D=128, Hi=16, di=128, P=96, scale=0.088), [9001, 300, 40003], 512),
+    (Dims(Hq=32, Hkv=4, D=128, Hi=16, di=128, P=16, scale=0.088), [9001, 301, 2], 512),
+    (Dims(Hq=8, Hkv=2, D=128, Hi=5, di=64, P=48, scale=0.11), [4099, 1500, 7], 64),
+    (Dims(Hq=8, Hkv=8, D=128, Hi=32, di=128, P=4, scale=0.1), [517, 2049], 100),
 ])
 def test_other_dims(dims, lens, k):
     for R in (1, 3):
@@ -116,7 +124,7 @@ def _topk_gpu(scores_np, k, lens=None):
 
 @pytest.mark.parametrize("rows", [6, 66])  # clusters per row; one CTA per row
 @pytest.mark.parametrize("case", ["random", "ties", "allzero", "negzero", "negative", "few",
-                                  "heavy"])
+                                  "heavy", "bucket900", "bucket1100"])
 def test_topk_exact(case, rows):
     g = np.random.default_rng(sum(map(ord, case)))
     # one CTA per row takes rows of at most 65,536 blocks
@@ -134,9 +142,22 @@ def test_topk_exact(case, rows):
         s = g.standard_normal((B, ld)).astype(np.float32)
     elif case == "few":
         s = g.standard_normal((B, ld)).astype(np.float32)
-    else:  # heavy tail with a block of exact ties at the threshold
+    elif case == "heavy":  # heavy tail with a block of exact ties at the threshold
         s = np.exp(3 * g.standard_normal((B, ld))).astype(np.float32)
         s[:, 1000:3000] = np.float32(np.sort(s[0])[-400])
+    else:
+        # 400 clear winners, then n keys in [1, 1 + 2^-7): one bucket of the
+        # upper 16 key bits holding the k-th key, their low bits drawn from
+        # 300 values (many exact duplicates, ranked by index), the rest far
+        # below. n = 900 is resolved as one tie list in the cluster kernel,
+        # n = 1100 takes its two further digit passes.
+        n = int(case[len("bucket"):])
+        s = (0.25 * g.random((B, ld))).astype(np.float32)
+        for b in range(B):
+            pos = g.permutation(ld)
+            s[b, pos[:400]] = (2.0 + g.random(400)).astype(np.float32)
+            low = g.integers(0, 300, n).astype(np.uint32)
+            s[b, pos[400:400 + n]] = (np.uint32(0x3F800000) + low).view(np.float32)
     lens = [4 * ld - 3, 4 * ld, 2049, 2048, 4 * 513, 1]
     if case == "few":
         lens = [5, 4 * 511 + 1, 4 * 512, 4 * 512 + 1, 4 * 65536, 4 * 70001]
@@ -291,10 +312,11 @@ def test_invalid_arguments_rejected_on_host():
                               o_mis.view_as(run.buf.o_part), run.buf.lse_part, run.buf.ws)
     assert ei.value.status == qsa.QSA_ERR_INVALID_ARG
     small_ws = torch.empty(16, dtype=torch.uint8, device=DEV)
-    with pytest.raises(qsa.QsaError) as ei:
-        qsa.qsa_sparse_decode(run.dims, run.cache, run.seq_lens, wl.q, run.buf.sel, 8, 1,
-                              run.buf.o_part, run.buf.lse_part, small_ws)
-    assert ei.value.status == qsa.QSA_ERR_INVALID_ARG
+    for ws in (small_ws, None):
+        with pytest.raises(qsa.QsaError) as ei:
+            qsa.qsa_sparse_decode(run.dims, run.cache, run.seq_lens, wl.q, run.buf.sel, 8, 1,
+                                  run.buf.o_part, run.buf.lse_part, ws)
+        assert ei.value.status == qsa.QSA_ERR_INVALID_ARG
 
 
 def test_decode_shapes_back_to_back():
