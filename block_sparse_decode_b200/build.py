@@ -1,6 +1,6 @@
 """Build libqsa.so (all CUDA sources under csrc/) for sm_100a, in-tree.
 
-    python -m block_sparse_decode_b200.build [--force] [--verbose]
+    python -m block_sparse_decode_b200.build [--force] [--verbose] [--nvtx]
 
 Each .cu file is compiled to an object under _build/ (in parallel), then
 linked into block_sparse_decode_b200/libqsa.so with a static CUDA runtime.
@@ -83,5 +83,7 @@ if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true")
+    ap.add_argument("--nvtx", action="store_true",
+                    help="name every C-ABI call as an NVTX range (profiler timelines)")
     a = ap.parse_args()
-    print(build(force=a.force, verbose=a.verbose))
+    print(build(force=a.force or a.nvtx, verbose=a.verbose, extra=("-DQSA_NVTX",) if a.nvtx else ()))

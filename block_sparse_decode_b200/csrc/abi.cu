@@ -11,6 +11,23 @@
 
 #define QSA_VERSION_NUM 100  // 0.1.0
 
+// Tracing: built with -DQSA_NVTX (python -m block_sparse_decode_b200.build
+// --nvtx), every C-ABI call is an NVTX range named after it, so a profiler
+// timeline shows which launches each call enqueued. NVTX v3 is header-only:
+// without a tool attached a range costs a branch.
+#ifdef QSA_NVTX
+#include <nvtx3/nvToolsExt.h>
+namespace {
+struct NvtxRange {
+  explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
+}  // namespace
+#define QSA_RANGE(name) NvtxRange qsa_nvtx_range_(name)
+#else
+#define QSA_RANGE(name) ((void)0)
+#endif
+
 namespace qsa {
 
 // One error word per device (module-scope device variable, no allocation).
@@ -173,6 +190,7 @@ const char *qsa_last_error(void) { return t_last_error.c_str(); }
 qsa_status qsa_append(const qsa_dims *dims, const qsa_cache *cache, int32_t N,
                       const int32_t *tok_seq, const int32_t *tok_pos, const void *k_new,
                       const void *v_new, const void *kidx_new, qsa_stream_t stream) {
+  QSA_RANGE("qsa_append");
   try {
     QSA_TRY(check_dims(dims));
     QSA_TRY(check_cache(cache, true, true));
@@ -194,6 +212,7 @@ qsa_status qsa_append(const qsa_dims *dims, const qsa_cache *cache, int32_t N,
 qsa_status qsa_index_score(const qsa_dims *dims, const qsa_cache *cache, int32_t B,
                            const int32_t *seq_lens, const void *q_idx, const float *w,
                            float *scores, int32_t ld_scores, qsa_stream_t stream) {
+  QSA_RANGE("qsa_index_score");
   try {
     QSA_TRY(check_dims(dims));
     QSA_TRY(check_cache(cache, false, true));
@@ -223,6 +242,7 @@ size_t qsa_topk_workspace_size(int32_t B, int32_t ld_scores, int32_t k) {
 qsa_status qsa_topk_select(int32_t B, const int32_t *seq_lens, const float *scores,
                            int32_t ld_scores, int32_t k, int32_t *sel, void *ws, size_t ws_bytes,
                            qsa_stream_t stream) {
+  QSA_RANGE("qsa_topk_select");
   (void)ws;
   (void)ws_bytes;
   try {
@@ -257,6 +277,7 @@ qsa_status qsa_sparse_decode(const qsa_dims *dims, const qsa_cache *cache, int32
                              const int32_t *seq_lens, const void *q, const int32_t *sel,
                              int32_t k, int32_t R, float *o_part, float *lse_part, void *ws,
                              size_t ws_bytes, qsa_stream_t stream) {
+  QSA_RANGE("qsa_sparse_decode");
   return qsa_sparse_decode_mq(dims, cache, B, 1, seq_lens, q, sel, k, R, o_part, lse_part, ws,
                               ws_bytes, stream);
 }
@@ -266,6 +287,7 @@ qsa_status qsa_sparse_decode_mq(const qsa_dims *dims, const qsa_cache *cache, in
                                 const int32_t *sel, int32_t k, int32_t R, float *o_part,
                                 float *lse_part, void *ws, size_t ws_bytes,
                                 qsa_stream_t stream) {
+  QSA_RANGE("qsa_sparse_decode_mq");
   try {
     QSA_TRY(check_dims(dims));
     QSA_TRY(check_cache(cache, true, false));
@@ -296,6 +318,7 @@ qsa_status qsa_sparse_decode_mq(const qsa_dims *dims, const qsa_cache *cache, in
 
 qsa_status qsa_select_owned(int32_t B, const int32_t *sel, int32_t k, int32_t P, int32_t W,
                             int32_t r, int32_t *sel_out, qsa_stream_t stream) {
+  QSA_RANGE("qsa_select_owned");
   try {
     if (B < 0 || B > 65535) return fail(QSA_ERR_INVALID_ARG, "B=%d outside [0, 65535]", B);
     if (k < 1 || k > 4096) return fail(QSA_ERR_UNSUPPORTED, "k=%d outside [1, 4096]", k);
@@ -316,6 +339,7 @@ qsa_status qsa_select_owned(int32_t B, const int32_t *sel, int32_t k, int32_t P,
 qsa_status qsa_merge(int32_t R, int32_t B, int32_t Hq, int32_t D, const float *o_part,
                      const float *lse_part, void *out, int32_t out_is_bf16, float *lse_out,
                      qsa_stream_t stream) {
+  QSA_RANGE("qsa_merge");
   try {
     if (R < 1 || R > 64) return fail(QSA_ERR_UNSUPPORTED, "R=%d outside [1, 64]", R);
     if (B < 0 || Hq <= 0 || D <= 0 || D % 4 != 0)
@@ -342,6 +366,7 @@ qsa_status qsa_decode_step(const qsa_dims *dims, const qsa_cache *cache, int32_t
                            int32_t *sel, float *o_part, float *lse_part, void *ws,
                            size_t ws_bytes, void *out, int32_t out_is_bf16, float *lse_out,
                            qsa_stream_t stream) {
+  QSA_RANGE("qsa_decode_step");
   qsa_status st = QSA_OK;
   if (N != 0)
     st = qsa_append(dims, cache, N, tok_seq, tok_pos, k_new, v_new, kidx_new, stream);
@@ -393,6 +418,7 @@ qsa_status qsa_prefill_index_score(const qsa_dims *dims, const qsa_cache *cache,
                                    const void *q_idx, const float *w, float *scores,
                                    int32_t ld_scores, int32_t *row_len, void *ws,
                                    size_t ws_bytes, qsa_stream_t stream) {
+  QSA_RANGE("qsa_prefill_index_score");
   try {
     QSA_TRY(check_dims(dims));
     QSA_TRY(check_cache(cache, false, true));
@@ -429,6 +455,7 @@ qsa_status qsa_prefill_sparse_decode(const qsa_dims *dims, const qsa_cache *cach
                                      int32_t Nq, const void *q, const int32_t *sel, int32_t k,
                                      int32_t R, float *o_part, float *lse_part, void *ws,
                                      size_t ws_bytes, qsa_stream_t stream) {
+  QSA_RANGE("qsa_prefill_sparse_decode");
   try {
     QSA_TRY(check_dims(dims));
     QSA_TRY(check_cache(cache, true, false));
@@ -476,6 +503,7 @@ qsa_status qsa_sparse_prefill(const qsa_dims *dims, const qsa_cache *cache, int3
                               int32_t *sel, float *o_part, float *lse_part, void *ws,
                               size_t ws_bytes, void *out, int32_t out_is_bf16, float *lse_out,
                               qsa_stream_t stream) {
+  QSA_RANGE("qsa_sparse_prefill");
   if (dims == nullptr) return fail(QSA_ERR_INVALID_ARG, "dims is NULL");
   if (S < 0 || Nq < 0) return fail(QSA_ERR_INVALID_ARG, "S or Nq negative");
   if (S == 0 || Nq == 0) return ok();
@@ -498,6 +526,7 @@ qsa_status qsa_sparse_prefill(const qsa_dims *dims, const qsa_cache *cache, int3
 }
 
 qsa_status qsa_check_device_errors(qsa_stream_t stream, int32_t *flags) {
+  QSA_RANGE("qsa_check_device_errors");
   try {
     if (flags) *flags = 0;
     cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));

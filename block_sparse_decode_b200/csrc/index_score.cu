@@ -48,6 +48,7 @@
 #include <cuda.h>
 
 #include <algorithm>
+#include <cstdlib>
 #include <mutex>
 
 #include "common.cuh"
@@ -77,6 +78,8 @@ struct TcArgs {
   int box;  // tile rows per page piece: gcd(P/4, 128)
   int ept;  // page pieces per tile: 128 / box
   int tpc;  // tiles per half of the shared page table
+  uint32_t spin_limit;  // try_wait rounds before a role gives up
+  int stall;            // failure injection: producers issue nothing (debug_stall_score())
   unsigned *err;
 };
 
@@ -260,14 +263,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     // overlaps the other's TMA issue.
     int last_chunk = -1, refilled = 0;
     int ti = warp;
-    for (; ti < my_tiles; ti += TC_PROD_WARPS) {
+    for (; ti < my_tiles && !a.stall; ti += TC_PROD_WARPS) {
       const int chunk = ti / a.tpc, tl = ti - chunk * a.tpc;
       if (chunk != last_chunk) {  // this half of the page table must have landed
         bool ok = true;
         if (lane == 0)
-          ok = chunk == 0 ? mbar_wait(smem_u32(&ctl.tbl0), 0u, abort_flag, a.err)
+          ok = chunk == 0 ? mbar_wait(smem_u32(&ctl.tbl0), 0u, abort_flag, a.err, a.spin_limit)
                           : mbar_wait(smem_u32(&ctl.tbl[chunk & 1]),
-                                      (uint32_t)(((chunk - 1) >> 1) & 1), abort_flag, a.err);
+                                      (uint32_t)(((chunk - 1) >> 1) & 1), abort_flag, a.err,
+                                      a.spin_limit);
         if (!__shfl_sync(0xffffffffu, ok, 0)) break;
         __syncwarp();
         last_chunk = chunk;
@@ -297,7 +301,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       const int s = ti % S;
       const uint32_t ph = (uint32_t)((ti / S) & 1);
       bool ok = true;
-      if (lane == 0) ok = mbar_wait(empty0 + 8 * s, ph ^ 1u, abort_flag, a.err);
+      if (lane == 0) ok = mbar_wait(empty0 + 8 * s, ph ^ 1u, abort_flag, a.err, a.spin_limit);
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       __syncwarp();
       const unsigned live = __ballot_sync(0xffffffffu, page >= 0);
@@ -326,8 +330,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       uint32_t ph = 0, aph = 0;
       int consumed = 0;
       for (int ti = 0; ti < my_tiles; ++ti) {
-        if (!mbar_wait(tempty0 + 8 * acc, aph ^ 1u, abort_flag, a.err)) break;
-        if (!mbar_wait(full0 + 8 * s, ph, abort_flag, a.err)) break;
+        if (!mbar_wait(tempty0 + 8 * acc, aph ^ 1u, abort_flag, a.err, a.spin_limit)) break;
+        if (!mbar_wait(full0 + 8 * s, ph, abort_flag, a.err, a.spin_limit)) break;
         tc_fence_after();
         const uint32_t stage_s = ring_s + (uint32_t)s * STAGE;
         const uint32_t d = tmem + (uint32_t)(acc * 32);
@@ -365,7 +369,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
       for (int h = 0; h < N; ++h) wv[h] = h < a.Hi ? __ldg(a.w + (size_t)b * a.Hi + h) : 0.f;
       bool ok = true;
-      if (lane == 0) ok = mbar_wait(tfull0 + 8 * acc, aph, abort_flag, a.err);
+      if (lane == 0) ok = mbar_wait(tfull0 + 8 * acc, aph, abort_flag, a.err, a.spin_limit);
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       __syncwarp();
       tc_fence_after();
@@ -395,6 +399,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     if (threadIdx.x == 32 * TC_EPI0) ctl.done = done;
   }
 
+  asm volatile("cp.async.wait_all;" ::: "memory");  // page-table copies, even after an abort
   __syncthreads();
   pdl_trigger();
   if (ctl.abort_flag) {
@@ -421,6 +426,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 }
 
 }  // namespace
+
+bool debug_stall_score() {
+  const char *v = std::getenv("QSA_DEBUG_STALL_SCORE");
+  return v != nullptr && v[0] == '1' && v[1] == '\0';
+}
 
 EncodeTiledFn encode_tiled_fn(cudaError_t *status) {
   static std::once_flag once;
@@ -529,6 +539,8 @@ cudaError_t launch_index_score(const qsa_dims &d, const qsa_cache &c, int B,
   a.num_pages = c.num_pages;
   a.Hi = d.Hi;
   a.stages = 2;
+  a.stall = debug_stall_score() ? 1 : 0;
+  a.spin_limit = a.stall ? TC_STALL_LIMIT : TC_SPIN_LIMIT;
   a.err = err;
   if (d.di == 128)
     return d.Hi <= 16 ? launch_tc_t<128, 16>(c, a, st) : launch_tc_t<128, 32>(c, a, st);

@@ -13,6 +13,15 @@ namespace qsa {
 constexpr uint32_t TC_SPIN_LIMIT = 1u << 22;  // try_wait rounds before giving up
 constexpr uint32_t TC_DRAIN_LIMIT = 1u << 20;
 
+// Failure injection for the decode scoring kernel, read at each launch from
+// the environment variable QSA_DEBUG_STALL_SCORE: when it is "1", the
+// producer warps issue no copy (a barrier that nothing completes) and the
+// roles' waits give up after TC_STALL_LIMIT rounds. This exercises the
+// timeout path (the TIMEOUT bit, the drain, the release of TMEM) on a real
+// GPU without faulting or hanging anything; unset, it costs one getenv.
+constexpr uint32_t TC_STALL_LIMIT = 1024;
+bool debug_stall_score();
+
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
 }

@@ -39,3 +39,22 @@ def test_umma_descriptors_match_cute(tmp_path):
                    check=True, capture_output=True)
     r = subprocess.run([str(exe)], capture_output=True, text=True)
     assert r.returncode == 0 and "OK" in r.stdout, r.stdout
+
+
+def test_nvtx_ranges_build(tmp_path):
+    # the tracing build (-DQSA_NVTX) compiles and names the C-ABI calls as
+    # NVTX ranges; the default build has none
+    nvcc = shutil.which("nvcc") or "/usr/local/cuda/bin/nvcc"
+    if not os.path.exists(nvcc):
+        pytest.skip("nvcc not available")
+    src = os.path.join(ROOT, "block_sparse_decode_b200", "csrc", "abi.cu")
+    objs = {}
+    for name, extra in (("plain", []), ("nvtx", ["-DQSA_NVTX"])):
+        obj = tmp_path / f"abi_{name}.o"
+        subprocess.run([nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-std=c++17",
+                        "-Xcompiler", "-fPIC", "-I" + os.path.join(ROOT, "include"), *extra,
+                        "-c", src, "-o", str(obj)], check=True, capture_output=True)
+        objs[name] = subprocess.run(["strings", str(obj)], capture_output=True,
+                                    text=True).stdout
+    assert "qsa_decode_step" in objs["nvtx"] and "nvtx" in objs["nvtx"].lower()
+    assert "nvtx" not in objs["plain"].lower()
