@@ -103,9 +103,18 @@ cudaError_t ensure_dynamic_smem(const void *kernel, size_t bytes) {
 
 int device_sm_count() {
   const int dev = current_device();
-  if (dev < 0 || dev >= kMaxDevices) return 148;
+  if (dev < 0 || dev >= kMaxDevices) return 148;  // no device: a B200's count
   std::lock_guard<std::mutex> lk(g_mu);
-  return g_sm_count[dev] > 0 ? g_sm_count[dev] : 148;
+  if (g_sm_count[dev] <= 0) {
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      (void)cudaGetLastError();
+      sms = 0;
+    }
+    if (sms <= 0) return 148;
+    g_sm_count[dev] = sms;
+  }
+  return g_sm_count[dev];
 }
 
 }  // namespace qsa

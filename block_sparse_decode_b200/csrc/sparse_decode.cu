@@ -62,7 +62,6 @@ constexpr int DV_TBL_BLOCKS = 1024;          // blocks per CTA range (host guara
 constexpr int DV_TBL_TILES = DV_TBL_BLOCKS / 4;
 constexpr int DV_RMAX = 64;
 constexpr int DV_CTAS_PER_SM = 2;
-constexpr int DV_SLOTS = DV_CTAS_PER_SM * 148;  // CTAs in flight on a B200
 constexpr size_t DV_SMEM_LIMIT = 113 * 1024;    // shared memory per CTA so that two fit an SM
 constexpr int DV_CB_ROWS = 8;                   // query-head rows per combine CTA
 constexpr int DV_CB_BATCH = 16;                 // records' outputs loaded together (combine)
@@ -697,10 +696,13 @@ DecodePlan plan_decode(const qsa_dims &d, int B, int k, int R) {
   const size_t fit = (DV_SMEM_LIMIT - static_smem - extra) / ((size_t)DV_WARPS * DV_STAGE);
   p.stages = fit >= 4 ? 4 : (fit >= 3 ? 3 : 2);
   p.smem = (size_t)DV_WARPS * p.stages * DV_STAGE + extra;
-  // CTAs per sequence: enough to keep DV_SLOTS CTAs busy, at most one per
-  // tile, and enough that a CTA's tile range fits its page table
+  // CTAs per sequence: enough to keep DV_CTAS_PER_SM CTAs busy on every SM
+  // of the device (the workspace size follows, so it is sized the same way
+  // for the same device), at most one per tile, and enough that a CTA's tile
+  // range fits its page table
+  const long long slots = (long long)DV_CTAS_PER_SM * device_sm_count();
   const long long ntmax = (k + 3) / 4 + R - 1;
-  long long ncb = DV_SLOTS / ((long long)B * p.nhg);
+  long long ncb = slots / ((long long)B * p.nhg);
   if (ncb > ntmax) ncb = ntmax;
   if (ncb < 1) ncb = 1;
   const long long need = (ntmax + DV_TBL_TILES - 1) / DV_TBL_TILES;
