@@ -66,7 +66,7 @@ constexpr int TC_PROD_WARPS = 3;                          // producers take tile
 constexpr int TC_MMA_WARP = TC_PROD_WARPS;                // warp 3
 constexpr int TC_EPI0 = TC_PROD_WARPS + 1;                // first epilogue warp
 constexpr int TC_THREADS = 32 * (TC_PROD_WARPS + 1 + TC_EPI_WARPS);
-constexpr int TBL = 4096;  // shared page-table entries (two halves)
+constexpr int TBL = 2048;  // shared page-table entries (two halves)
 __device__ const int32_t k_no_page = -1;
 
 struct TcArgs {

@@ -37,3 +37,23 @@ def test_scoring_wait_that_runs_out_is_reported_and_the_context_survives(monkeyp
     run.step(append=False)  # the same context still runs the whole step
     for b in range(wl.B):
         _check_seq(run, b)
+
+
+def test_stalled_scoring_inside_a_decode_step(monkeypatch):
+    """The same failure inside qsa_decode_step (append, then the stalled
+    scoring chained to it): every role gives up, the kernel drains and frees
+    TMEM, the later kernels of the step run on whatever the scores hold (no
+    fault), TIMEOUT is reported, and the next step passes parity."""
+    wl = make_custom(DIMS_FULL, [70001, 9001, 517, 40000], k=512, R=2, seed=405,
+                     device="cuda", paged=True)
+    run = CudaRun(wl)
+    monkeypatch.setenv("QSA_DEBUG_STALL_SCORE", "1")
+    qsa.decode_step(run.dims, run.cache, run.seq_lens, wl.q, wl.q_idx, wl.w, run.k, run.R,
+                    run.buf, append=run.current_tokens())
+    with pytest.raises(qsa.QsaError) as ei:
+        qsa.qsa_check_device_errors()
+    assert ei.value.status == qsa.QSA_ERR_TIMEOUT
+    monkeypatch.delenv("QSA_DEBUG_STALL_SCORE")
+    run.step()
+    for b in range(wl.B):
+        _check_seq(run, b)

@@ -98,6 +98,57 @@ def test_other_dims(dims, lens, k):
             _check_seq(run, b)
 
 
+@pytest.mark.parametrize("P", [32, 64])
+def test_index_score_long_rows_refill_the_page_table(P):
+    """Score rows so long that each scoring CTA's tiles overflow its shared
+    page table (two halves of 1,024 page ids: 64 tiles at P = 32, 128 tiles
+    at P = 64) more than once, so both halves are refilled while the
+    producers run: 4 sequences of 2,600,000 tokens at P = 32 (137 tiles per
+    CTA), of 5,200,000 at P = 64. Scoring reads only the side cache here
+    (every length a multiple of 4: no partial block), filled with random
+    bf16 rows through a shuffled block table; sampled blocks of every
+    sequence (both ends, tile and page boundaries, random ones) are checked
+    against the oracle's score formula within the scores' fp32 bound."""
+    g = torch.Generator(device=DEV).manual_seed(4200 + P)
+    di, Hi, B = 128, 16, 4
+    L = 2_600_000 * (P // 32)
+    dims = qsa.QsaDims(Hq=8, Hkv=1, D=128, Hi=Hi, di=di, P=P, scale=0.088)
+    npp = L // P                                 # pages per sequence
+    num_pages = B * npp
+    perm = torch.randperm(num_pages, generator=g, device=DEV).to(torch.int32)
+    bt = perm.view(B, npp).contiguous()
+    side = torch.randn((num_pages, P // 4, di), generator=g, device=DEV).to(torch.bfloat16)
+    small = torch.zeros((num_pages, 1, 1, 8), dtype=torch.bfloat16, device=DEV)  # never read
+    cache = qsa.QsaCache(k_pool=small, v_pool=small, kidx_pool=small, side_pool=side,
+                         block_table=bt)
+    q_idx = torch.randn((B, Hi, di), generator=g, device=DEV).to(torch.bfloat16)
+    w = torch.rand((B, Hi), generator=g, device=DEV)
+    lens = torch.full((B,), L, dtype=torch.int32, device=DEV)
+    nb = L // 4
+    scores = torch.full((B, nb), float("nan"), device=DEV)
+    qsa.qsa_index_score(dims, cache, lens, q_idx, w, scores)
+    assert qsa.qsa_check_device_errors() == 0
+    assert not torch.isnan(scores).any()
+    rng = np.random.default_rng(P)
+    picks = np.unique(np.concatenate([
+        np.arange(0, 300), np.arange(nb - 300, nb),
+        np.arange(127, nb, 128 * 997), np.arange(128, nb, 128 * 997),
+        np.arange(P // 4 - 1, nb, (P // 4) * 4999), rng.integers(0, nb, 3000)]))
+    rpp = P // 4
+    for b in range(B):
+        j = torch.from_numpy(picks).to(DEV)
+        rows = side[bt[b].long()[j // rpp], j % rpp]                   # [n, di] bf16
+        kc = oracle.bf16_to_f32(bits(rows)).astype(np.float64)
+        qb = bits(q_idx[b])
+        wb = w[b].cpu().numpy()
+        ref = oracle.index_scores(kc, qb, wb)
+        q64 = oracle.bf16_to_f32(qb).astype(np.float64)
+        tol = (np.abs(kc) @ np.abs(q64).T) @ np.abs(wb.astype(np.float64)) * 2.0 ** -12 + 1e-30
+        got = scores[b, j].double().cpu().numpy()
+        err = np.abs(got - ref)
+        assert np.all(err <= tol), (b, int(picks[err.argmax()]), float(err.max()))
+
+
 def test_clustered_selection_leaves_empty_slices():
     # needles + k small: the selection sits in a few slices, most slices empty
     d = DIMS_FULL
