@@ -109,9 +109,9 @@ __device__ __forceinline__ int tc_find_seq(const int *prefix, int B, int t) {
 
 // Score of the trailing partial block of sequence b (whole warp; every lane
 // returns it).
-template <int DI>
+template <int DI, int N>
 __device__ float partial_block_score(const TcArgs &a, int b, int L, bool *ok_out) {
-  return partial_block_score_row<DI>(a.kidx_pool, a.P, a.block_table + (size_t)b * a.max_pages,
+  return partial_block_score_row<DI, N>(a.kidx_pool, a.P, a.block_table + (size_t)b * a.max_pages,
                                      a.max_pages, a.num_pages, L, a.q_idx + (size_t)b * a.Hi * DI,
                                      a.w + (size_t)b * a.Hi, a.Hi, a.err, ok_out);
 }
@@ -390,7 +390,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       if (j < nfull) a.scores[(size_t)b * a.ld + j] = score;
       if (nfull < nb && nfull >= j0 + q * 32 && nfull < j0 + q * 32 + 32) {
         bool ok;
-        const float sp = partial_block_score<DI>(a, b, L, &ok);
+        const float sp = partial_block_score<DI, N>(a, b, L, &ok);
         if (lane == 0 && ok) a.scores[(size_t)b * a.ld + nfull] = sp;
       }
       ++done;

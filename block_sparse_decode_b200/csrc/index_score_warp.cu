@@ -153,7 +153,7 @@ __global__ void __launch_bounds__(SW_WARPS * 32) index_score_warp_kernel(SwArgs 
     }
     if (nfull < nb && nfull >= j0 && nfull < j0 + SW_ROWS) {  // the trailing partial block
       bool ok;
-      const float sp = partial_block_score_row<DI>(a.kidx_pool, a.P, bt, a.max_pages, a.num_pages,
+      const float sp = partial_block_score_row<DI, NT * 8>(a.kidx_pool, a.P, bt, a.max_pages, a.num_pages,
                                                    L, a.q_idx + (size_t)b * a.Hi * DI,
                                                    a.w + (size_t)b * a.Hi, a.Hi, a.err, &ok);
       if (lane == 0 && ok) a.scores[(size_t)b * a.ld + nfull] = sp;

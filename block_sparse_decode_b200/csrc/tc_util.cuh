@@ -145,8 +145,14 @@ __device__ __forceinline__ void tc_wait_ld() {
 // L tokens of the sequence with block-table row bt_row (whole warp; every
 // lane returns it). The key is the bf16-rounded mean of its L mod 4 indexer
 // keys, built exactly as the side cache builds complete blocks; q_rows holds
-// the query's Hi indexer rows of DI elements, w_row its Hi head weights.
-template <int DI>
+// the query's Hi <= HMAX indexer rows of DI elements, w_row its Hi head
+// weights. It runs while the memory system streams at full load, where each
+// dependent round trip costs microseconds, so it makes two: the query rows
+// and weights are asked into L1 first (one 128-byte line per lane), the up to
+// 3 key rows are loaded together once the page id is known, and the per-head
+// loop then reads the query from L1. Same operations in the same order as
+// before, so the score is the same bits.
+template <int DI, int HMAX = 32>
 __device__ float partial_block_score_row(const __nv_bfloat16 *kidx_pool, int P,
                                          const int32_t *bt_row, int max_pages, int num_pages,
                                          int L, const __nv_bfloat16 *q_rows, const float *w_row,
@@ -154,6 +160,12 @@ __device__ float partial_block_score_row(const __nv_bfloat16 *kidx_pool, int P,
   const int lane = threadIdx.x & 31;
   const int nfull = L >> 2, n = L - 4 * nfull, pos = 4 * nfull;
   const int col = pos / P;
+  constexpr int QLINES = HMAX * DI * 2 / 128;  // 128-byte lines of HMAX query rows
+#pragma unroll
+  for (int l = lane; l < QLINES; l += 32)
+    if (l * 128 < Hi * DI * 2)
+      asm volatile("prefetch.global.L1 [%0];" ::"l"(reinterpret_cast<const char *>(q_rows) + l * 128));
+  if (lane == 0) asm volatile("prefetch.global.L1 [%0];" ::"l"(w_row));
   int page = -1;
   if (col < max_pages) page = bt_row[col];
   const bool ok = page >= 0 && page < num_pages;
@@ -164,22 +176,28 @@ __device__ float partial_block_score_row(const __nv_bfloat16 *kidx_pool, int P,
   }
   const uint32_t *x = reinterpret_cast<const uint32_t *>(kidx_pool) +
                       ((size_t)page * P + pos % P) * (DI / 2);
+  uint32_t xv[3][DI / 64];
+#pragma unroll
+  for (int u = 0; u < 3; ++u)
+#pragma unroll
+    for (int i = 0; i < DI / 64; ++i) xv[u][i] = u < n ? x[u * (DI / 2) + lane + 32 * i] : 0u;
   float klo[DI / 64], khi[DI / 64];
 #pragma unroll
   for (int i = 0; i < DI / 64; ++i) {
-    const int e = lane + 32 * i;
-    uint32_t v = x[e];
-    float lo = bf16lo(v), hi = bf16hi(v);
-    for (int u = 1; u < n; ++u) {
-      v = x[u * (DI / 2) + e];
-      lo = __fadd_rn(lo, bf16lo(v));
-      hi = __fadd_rn(hi, bf16hi(v));
+    float lo = bf16lo(xv[0][i]), hi = bf16hi(xv[0][i]);
+#pragma unroll
+    for (int u = 1; u < 3; ++u) {
+      if (u < n) {
+        lo = __fadd_rn(lo, bf16lo(xv[u][i]));
+        hi = __fadd_rn(hi, bf16hi(xv[u][i]));
+      }
     }
     const uint32_t kc = pack_bf16x2(__fdiv_rn(lo, (float)n), __fdiv_rn(hi, (float)n));
     klo[i] = bf16lo(kc);
     khi[i] = bf16hi(kc);
   }
   float score = 0.f;
+#pragma unroll 4
   for (int h = 0; h < Hi; ++h) {
     const uint32_t *qrow = reinterpret_cast<const uint32_t *>(q_rows + (size_t)h * DI);
     float part = 0.f;
