@@ -53,10 +53,13 @@ cudaError_t launch_index_score(const qsa_dims &d, const qsa_cache &c, int B,
 
 constexpr int TOPK_CLUSTER = 8;
 constexpr int TOPK_MAX_KEYS_PER_CTA = 49152;  // 192 KiB of keys per CTA
-// One CTA per sequence instead of a cluster from this many sequences on, for
-// score rows of at most TOPK_ROW_MAX_KEYS blocks (2 bytes each in shared
-// memory). Measured: 8 rows take 13.9 us in clusters and 44.8 us one CTA
-// each; 256 rows 140 us in clusters and 57 us one CTA each.
+// Top-k runs one cluster of 8 or 4 CTAs per sequence, the larger size whose
+// clusters all stay resident; when neither is (e.g. 128 sequences, 256
+// prefill rows), one CTA per sequence from this many sequences on, for score
+// rows of at most TOPK_ROW_MAX_KEYS blocks (2 bytes each in shared memory).
+// Measured: 8 rows take 13.9 us in clusters of 8 and 44.8 us one CTA each;
+// 64 rows of up to 65,536 blocks 28.9 us in clusters of 4 and 30.7 us one
+// CTA each; 256 rows 140 us in clusters of 8 and 57 us one CTA each.
 constexpr int TOPK_ROW_MIN_B = 64;
 constexpr int TOPK_ROW_MAX_KEYS = 65536;
 cudaError_t launch_topk(int B, const int32_t *seq_lens, const float *scores, int ld, int k,

@@ -21,6 +21,8 @@
 // memory and no inter-CTA waits other than cluster barriers.
 #include <cooperative_groups.h>
 
+#include <algorithm>
+
 #include "common.cuh"
 #include "launch.h"
 
@@ -49,6 +51,9 @@ __device__ __forceinline__ uint32_t score_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// CS CTAs per sequence (a cluster of 8 or 4): the host picks the larger one
+// that keeps every cluster of the batch resident at two CTAs per SM.
+template <int CS>
 __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a) {
   cg::cluster_group cluster = cg::this_cluster();
   const int crank = (int)cluster.block_rank();
@@ -68,16 +73,16 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a) {
   pdl_wait();  // the scores come from the kernel before this one
   if (L < 0 || nb > a.ld) {  // uniform over the cluster
     if (crank == 0 && tid == 0) raise_err(a.err, ERR_LEN);
-    for (int i = crank * TK_THREADS + tid; i < a.k; i += TOPK_CLUSTER * TK_THREADS) out[i] = -1;
+    for (int i = crank * TK_THREADS + tid; i < a.k; i += CS * TK_THREADS) out[i] = -1;
     return;
   }
   if (nb <= a.k) {  // every block is kept
-    for (int i = crank * TK_THREADS + tid; i < a.k; i += TOPK_CLUSTER * TK_THREADS)
+    for (int i = crank * TK_THREADS + tid; i < a.k; i += CS * TK_THREADS)
       out[i] = i < nb ? i : -1;
     return;
   }
 
-  const int chunk = (nb + TOPK_CLUSTER - 1) / TOPK_CLUSTER;
+  const int chunk = (nb + CS - 1) / CS;
   const int lo = min(nb, crank * chunk);
   const int n = min(nb, lo + chunk) - lo;
   const float *src = a.scores + (size_t)b * a.ld + lo;
@@ -124,12 +129,12 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a) {
     // sum the 8 histograms; thread t takes digit 255 - t (descending order)
     unsigned c = 0u, cum = 0u;
     if (tid < 256) {
-      unsigned v[TOPK_CLUSTER];
+      unsigned v[CS];
 #pragma unroll
-      for (int r = 0; r < TOPK_CLUSTER; ++r)
+      for (int r = 0; r < CS; ++r)
         v[r] = cluster.map_shared_rank(&hist[buf][0], r)[255 - tid];
 #pragma unroll
-      for (int r = 0; r < TOPK_CLUSTER; ++r) c += v[r];
+      for (int r = 0; r < CS; ++r) c += v[r];
       cum = c;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -178,15 +183,15 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a) {
   cluster.sync();
   {
     // the counts of every lower-ranked CTA, all loads in flight together
-    unsigned rg[TOPK_CLUSTER], re[TOPK_CLUSTER];
+    unsigned rg[CS], re[CS];
 #pragma unroll
-    for (int r = 0; r < TOPK_CLUSTER; ++r) {
+    for (int r = 0; r < CS; ++r) {
       const unsigned *rt = cluster.map_shared_rank(&ctot[0], r < crank ? r : crank);
       rg[r] = rt[0];
       re[r] = rt[1];
     }
 #pragma unroll
-    for (int r = 0; r < TOPK_CLUSTER; ++r) {
+    for (int r = 0; r < CS; ++r) {
       if (r < crank) {
         run_gt += rg[r];
         run_eq += re[r];
@@ -555,31 +560,50 @@ cudaError_t launch_topk(int B, const int32_t *seq_lens, const float *scores, int
                         int32_t *sel, unsigned *err, cudaStream_t st) {
   if (B == 0) return cudaSuccess;
   TopkArgs a{scores, seq_lens, sel, ld, k, err};
-  if (B >= TOPK_ROW_MIN_B && ld <= TOPK_ROW_MAX_KEYS) {
+  // clusters of CS CTAs while the batch's clusters all fit at two CTAs per SM
+  // (largest CS first, each CTA's keys within its shared memory); beyond
+  // that, one CTA per sequence for rows it can hold, else clusters of 8
+  // (clusters of 2 were measured slower than one CTA per row: 25.6 against
+  // 20.5 us for 128 rows of 16,384 blocks)
+  int cs = 0;
+  for (int c = TOPK_CLUSTER; c >= 4 && cs == 0; c >>= 1) {
+    const long long keys_b = (long long)((ld + c - 1) / c) * 4;
+    // CTAs per SM: two by registers (512 threads), fewer if the keys need it
+    // (the kernel's own shared arrays and 1 KiB reserved per CTA besides)
+    const long long per_sm = std::min<long long>(2, (228 * 1024) / (keys_b + 20 * 1024));
+    if (keys_b <= (long long)TOPK_MAX_KEYS_PER_CTA * 4 && per_sm > 0 &&
+        (long long)B * c <= per_sm * device_sm_count())
+      cs = c;
+  }
+  if (cs == 0 && B >= TOPK_ROW_MIN_B && ld <= TOPK_ROW_MAX_KEYS) {
     const size_t smem = tr_k16_bytes(ld) + tr_bit_bytes(ld) + (size_t)TR_GATHER * 8;
     cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void *>(topk_row_kernel), smem);
     if (e != cudaSuccess) return e;
     return launch_pdl(topk_row_kernel, B, TR_THREADS, smem, st, a);
   }
-  const int per_cta = (ld + TOPK_CLUSTER - 1) / TOPK_CLUSTER;
+  if (cs == 0) cs = TOPK_CLUSTER;
+  const void *kern = cs == 8 ? reinterpret_cast<const void *>(topk_kernel<8>)
+                             : reinterpret_cast<const void *>(topk_kernel<4>);
+  const int per_cta = (ld + cs - 1) / cs;
   const size_t smem = (size_t)per_cta * 4;
-  cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void *>(topk_kernel), smem);
+  cudaError_t e = ensure_dynamic_smem(kern, smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(TOPK_CLUSTER, B, 1);
+  cfg.gridDim = dim3(cs, B, 1);
   cfg.blockDim = dim3(TK_THREADS, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = TOPK_CLUSTER;
+  attr[0].val.clusterDim.x = cs;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, topk_kernel, a);
+  return cs == 8 ? cudaLaunchKernelEx(&cfg, topk_kernel<8>, a)
+                 : cudaLaunchKernelEx(&cfg, topk_kernel<4>, a);
 }
 
 }  // namespace qsa

@@ -173,7 +173,8 @@ def _topk_gpu(scores_np, k, lens=None):
     return sel.cpu().numpy()
 
 
-@pytest.mark.parametrize("rows", [6, 66])  # clusters per row; one CTA per row
+# clusters of 8 CTAs per row (6 rows), of 4 (66 rows), one CTA per row (300)
+@pytest.mark.parametrize("rows", [6, 66, 300])
 @pytest.mark.parametrize("case", ["random", "ties", "allzero", "negzero", "negative", "few",
                                   "heavy", "bucket900", "bucket1100"])
 def test_topk_exact(case, rows):
@@ -224,7 +225,7 @@ def test_topk_exact(case, rows):
         assert np.array_equal(got[b], ref), f"{case} b={b} nb={nb}"
 
 
-@pytest.mark.parametrize("rows", [3, 66])
+@pytest.mark.parametrize("rows", [3, 66, 300])  # clusters of 8, 4 CTAs; one CTA per row
 @pytest.mark.parametrize("k", [1, 2, 255, 256, 1024, 4096])
 def test_topk_k_sweep(k, rows):
     g = np.random.default_rng(k)
