@@ -22,6 +22,21 @@ __device__ __forceinline__ void merge_row(int R, int rows, int D, const float *o
                                           const float *lse_part, int row, void *out,
                                           int out_is_bf16, float *lse_out) {
   const int lane = threadIdx.x & 31;
+  const int passes = (D + 127) / 128;
+  // the first batch of partial outputs is requested together with the LSEs
+  // (one round trip instead of two when R <= MERGE_BATCH and D <= 128)
+  float4 v0[MERGE_BATCH];
+  {
+    const int d0 = lane * 4;
+    const bool live = d0 < D;
+#pragma unroll
+    for (int u = 0; u < MERGE_BATCH; ++u) {
+      const int r = min(u, R - 1);
+      v0[u] = live ? __ldcg(reinterpret_cast<const float4 *>(o_part + ((size_t)r * rows + row) * D +
+                                                              d0))
+                   : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
   const float l0 = lane < R ? __ldcg(lse_part + (size_t)lane * rows + row) : -INFINITY;
   const float l1 = lane + 32 < R ? __ldcg(lse_part + (size_t)(lane + 32) * rows + row) : -INFINITY;
   float M = fmaxf(l0, l1);
@@ -35,7 +50,6 @@ __device__ __forceinline__ void merge_row(int R, int rows, int D, const float *o
   const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
   // every lane runs the same number of passes over the head dims (the weight
   // shuffles below need the whole warp); a lane past D loads and stores nothing
-  const int passes = (D + 127) / 128;
   for (int it = 0; it < passes; ++it) {
     const int d0 = it * 128 + lane * 4;
     const bool live = d0 < D;
@@ -45,9 +59,10 @@ __device__ __forceinline__ void merge_row(int R, int rows, int D, const float *o
 #pragma unroll
       for (int u = 0; u < MERGE_BATCH; ++u) {
         const int r = min(r0 + u, R - 1);
-        v[u] = live ? __ldcg(reinterpret_cast<const float4 *>(o_part + ((size_t)r * rows + row) * D +
-                                                               d0))
-                    : make_float4(0.f, 0.f, 0.f, 0.f);
+        v[u] = it == 0 && r0 == 0 ? v0[u]
+               : live ? __ldcg(reinterpret_cast<const float4 *>(o_part + ((size_t)r * rows + row) * D +
+                                                                 d0))
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll
       for (int u = 0; u < MERGE_BATCH; ++u) {

@@ -620,6 +620,14 @@ __global__ void __launch_bounds__(DV_CB_ROWS * 32) decode_combine_kernel(DecodeA
     const int n = sp.y - sp.x + 1;
     const size_t stride = (size_t)a.qn * a.Hq;                         // between records
     const size_t row0 = ((size_t)b * a.rb + sp.x + r) * stride + q;    // record i at row0 + i*stride
+    // the first DV_CB_BATCH records' outputs are requested together with the
+    // LSEs (one round trip instead of two for slices of that many records)
+    float4 v[DV_CB_BATCH];
+#pragma unroll
+    for (int u = 0; u < DV_CB_BATCH; ++u) {
+      const size_t rr = row0 + (size_t)min(u, n - 1) * stride;
+      v[u] = __ldcg(reinterpret_cast<const float4 *>(a.rec_o + rr * DV_D) + lane);
+    }
     float M = -INFINITY;
     for (int i0 = 0; i0 < n; i0 += 32) {
       const float l = i0 + lane < n ? __ldcg(a.rec_lse + row0 + (size_t)(i0 + lane) * stride)
@@ -636,11 +644,12 @@ __global__ void __launch_bounds__(DV_CB_ROWS * 32) decode_combine_kernel(DecodeA
         const float wl = l == -INFINITY ? 0.f : __expf(l - M);  // weight of record i0 + lane
         const int m = min(32, n - i0);
         for (int u0 = 0; u0 < m; u0 += DV_CB_BATCH) {
-          float4 v[DV_CB_BATCH];
+          if (i0 != 0 || u0 != 0) {  // (the first batch is in v already)
 #pragma unroll
-          for (int u = 0; u < DV_CB_BATCH; ++u) {
-            const size_t rr = row0 + (size_t)(i0 + min(u0 + u, m - 1)) * stride;
-            v[u] = __ldcg(reinterpret_cast<const float4 *>(a.rec_o + rr * DV_D) + lane);
+            for (int u = 0; u < DV_CB_BATCH; ++u) {
+              const size_t rr = row0 + (size_t)(i0 + min(u0 + u, m - 1)) * stride;
+              v[u] = __ldcg(reinterpret_cast<const float4 *>(a.rec_o + rr * DV_D) + lane);
+            }
           }
 #pragma unroll
           for (int u = 0; u < DV_CB_BATCH; ++u) {
