@@ -248,12 +248,13 @@ size_t qsa_topk_workspace_size(int32_t B, int32_t ld_scores, int32_t k) {
   return 0;
 }
 
-qsa_status qsa_topk_select(int32_t B, const int32_t *seq_lens, const float *scores,
-                           int32_t ld_scores, int32_t k, int32_t *sel, void *ws, size_t ws_bytes,
-                           qsa_stream_t stream) {
-  QSA_RANGE("qsa_topk_select");
-  (void)ws;
-  (void)ws_bytes;
+namespace {
+
+// qsa_topk_select's checks and launch; starts / R / wrote_starts as in
+// launch_topk (the decode step's slice starts).
+qsa_status topk_checked(int32_t B, const int32_t *seq_lens, const float *scores,
+                        int32_t ld_scores, int32_t k, int32_t *sel, qsa_stream_t stream,
+                        int32_t *starts, int R, bool *wrote_starts) {
   try {
     if (B < 0 || B > 65535) return fail(QSA_ERR_INVALID_ARG, "B=%d outside [0, 65535]", B);
     if (k < 1 || k > 4096) return fail(QSA_ERR_UNSUPPORTED, "k=%d outside [1, 4096]", k);
@@ -264,11 +265,23 @@ qsa_status qsa_topk_select(int32_t B, const int32_t *seq_lens, const float *scor
       return fail(QSA_ERR_INVALID_ARG, "an argument array is NULL");
     QSA_ERRWORD(err);
     return cuda_status(launch_topk(B, seq_lens, scores, ld_scores, k, sel, err,
-                                   reinterpret_cast<cudaStream_t>(stream)),
+                                   reinterpret_cast<cudaStream_t>(stream), starts, R,
+                                   wrote_starts),
                        "qsa_topk_select launch");
   } catch (...) {
     return fail(QSA_ERR_CUDA, "qsa_topk_select: internal exception");
   }
+}
+
+}  // namespace
+
+qsa_status qsa_topk_select(int32_t B, const int32_t *seq_lens, const float *scores,
+                           int32_t ld_scores, int32_t k, int32_t *sel, void *ws, size_t ws_bytes,
+                           qsa_stream_t stream) {
+  QSA_RANGE("qsa_topk_select");
+  (void)ws;
+  (void)ws_bytes;
+  return topk_checked(B, seq_lens, scores, ld_scores, k, sel, stream, nullptr, 0, nullptr);
 }
 
 size_t qsa_sparse_decode_workspace_size(const qsa_dims *dims, int32_t B, int32_t k, int32_t R) {
@@ -381,8 +394,17 @@ qsa_status qsa_decode_step(const qsa_dims *dims, const qsa_cache *cache, int32_t
     st = qsa_append(dims, cache, N, tok_seq, tok_pos, k_new, v_new, kidx_new, stream);
   if (st == QSA_OK)
     st = qsa_index_score(dims, cache, B, seq_lens, q_idx, w, scores, ld_scores, stream);
+  // the top-k kernel also hands the decode kernel each selection's slice
+  // starts, through the end of the workspace (when it is large enough)
+  int32_t *starts = nullptr;
+  bool have_starts = false;
+  if (st == QSA_OK && dims != nullptr && check_dims(dims) == QSA_OK && ws != nullptr &&
+      aligned16(ws) && B > 0 && k >= 1 && k <= 4096 && R >= 1 && R <= 64 &&
+      ws_bytes >= decode_ws_bytes(*dims, B, 1, k, R))
+    starts = reinterpret_cast<int32_t *>(static_cast<char *>(ws) +
+                                         decode_ws_starts_offset(*dims, B, 1, k, R));
   if (st == QSA_OK)
-    st = qsa_topk_select(B, seq_lens, scores, ld_scores, k, sel, nullptr, 0, stream);
+    st = topk_checked(B, seq_lens, scores, ld_scores, k, sel, stream, starts, R, &have_starts);
   if (st == QSA_OK) {
     // qsa_sparse_decode and qsa_merge with the merge fused into the decode's
     // combine kernel (same arithmetic as qsa_merge); both calls' checks apply
@@ -408,7 +430,8 @@ qsa_status qsa_decode_step(const qsa_dims *dims, const qsa_cache *cache, int32_t
       st = cuda_status(launch_sparse_decode(*dims, *cache, B, 1, seq_lens, q, sel, k, R, o_part,
                                             lse_part, ws, err,
                                             reinterpret_cast<cudaStream_t>(stream), nullptr, 0,
-                                            out, out_is_bf16, lse_out),
+                                            out, out_is_bf16, lse_out,
+                                            have_starts ? starts : nullptr),
                        "qsa_decode_step decode + merge launch");
     } catch (...) {
       return fail(QSA_ERR_CUDA, "qsa_decode_step: internal exception");

@@ -62,10 +62,18 @@ constexpr int TOPK_MAX_KEYS_PER_CTA = 49152;  // 192 KiB of keys per CTA
 // CTA each; 256 rows 140 us in clusters of 8 and 57 us one CTA each.
 constexpr int TOPK_ROW_MIN_B = 64;
 constexpr int TOPK_ROW_MAX_KEYS = 65536;
+// starts (may be nullptr): [B, R + 1] slice starts of each selection for the
+// decode step (st[r] = selected blocks below floor(r nb / R)); *wrote_starts
+// tells whether the chosen kernel wrote them (the one-CTA-per-row kernel does
+// not).
 cudaError_t launch_topk(int B, const int32_t *seq_lens, const float *scores, int ld, int k,
-                        int32_t *sel, unsigned *err, cudaStream_t st);
+                        int32_t *sel, unsigned *err, cudaStream_t st, int32_t *starts = nullptr,
+                        int R = 0, bool *wrote_starts = nullptr);
 
 size_t decode_ws_bytes(const qsa_dims &d, int B, int Qn, int k, int R);
+// Offset of the [B, R + 1] int slice starts at the end of that workspace,
+// which the decode step's top-k kernel writes for its decode kernel.
+size_t decode_ws_starts_offset(const qsa_dims &d, int B, int Qn, int k, int R);
 // row_start != nullptr: B prefill rows of S chunks (sequence s holds rows
 // [row_start[s], row_start[s+1]), seq_lens[s] counts its chunk), Qn = 1.
 // m_out != nullptr (Qn = 1): the R partials are also merged into m_out
@@ -76,7 +84,8 @@ cudaError_t launch_sparse_decode(const qsa_dims &d, const qsa_cache &c, int B, i
                                  int k, int R, float *o_part, float *lse_part, void *ws,
                                  unsigned *err, cudaStream_t st,
                                  const int32_t *row_start = nullptr, int S = 0,
-                                 void *m_out = nullptr, int m_bf16 = 0, float *m_lse = nullptr);
+                                 void *m_out = nullptr, int m_bf16 = 0, float *m_lse = nullptr,
+                                 const int32_t *starts = nullptr);
 
 cudaError_t launch_select_owned(const int32_t *sel, int B, int k, int P, int W, int r,
                                 int32_t *out, cudaStream_t st);

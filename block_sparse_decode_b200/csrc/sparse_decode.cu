@@ -72,6 +72,10 @@ constexpr float LN2 = 0.6931471805599453f;
 struct DecodeArgs {
   const __nv_bfloat16 *k_pool, *v_pool, *q;  // q [B, Qn, Hq, D]
   const int32_t *block_table, *seq_lens, *sel;
+  // [B, R + 1] slice starts of each selection from the top-k kernel of a
+  // decode step (st[r] = selected blocks below floor(r nb / R)), nullptr:
+  // found here by binary search
+  const int32_t *starts;
   // prefill rows (nullptr for decode): row b belongs to the sequence s with
   // row_start[s] <= b < row_start[s+1] and sees L_s - T_s + (b - row_start[s]) + 1
   // tokens (T_s its chunk rows), through block-table row s
@@ -122,7 +126,8 @@ __device__ __forceinline__ int slice_of_tile(const int *pre, int R, int v) {
 
 // CTA whose tile range [floor(c*NT/ncb), floor((c+1)*NT/ncb)) holds tile v.
 __device__ __forceinline__ int cta_of_tile(int v, int NT, int ncb) {
-  return (int)(((long long)(v + 1) * ncb + NT - 1) / NT) - 1;
+  // 32-bit: (v + 1) * ncb <= NT * ncb, both below 2^11 by the host's bounds
+  return (int)(((unsigned)(v + 1) * (unsigned)ncb + (unsigned)NT - 1u) / (unsigned)NT) - 1;
 }
 
 // Online-softmax state of one warp: heads 2tq, 2tq+1 of the group (tq = lane
@@ -253,14 +258,15 @@ __device__ __forceinline__ void tile_range(int c, int NT, int ncb, int &v0, int 
     v0 = n = 0;
     return;
   }
-  v0 = (int)(((long long)c * NT) / ncb);
-  n = (int)(((long long)(c + 1) * NT) / ncb) - v0;
+  v0 = (int)(((unsigned)c * (unsigned)NT) / (unsigned)ncb);  // products below 2^22
+  n = (int)(((unsigned)(c + 1) * (unsigned)NT) / (unsigned)ncb) - v0;
 }
 
 template <int ST, int QN>
 __global__ void __launch_bounds__(DV_WARPS * 32, DV_CTAS_PER_SM) sparse_decode_kernel(DecodeArgs a) {
   extern __shared__ __align__(1024) unsigned char smem[];
   __shared__ int s_st[DV_RMAX], s_ct[DV_RMAX], s_pre[DV_RMAX + 1];
+  __shared__ int s_gst[DV_RMAX + 1];  // slice starts given by the top-k kernel
   __shared__ int s_L;
   const int c = blockIdx.x, CL = a.ncb;
   const int hg = blockIdx.y, b = blockIdx.z;
@@ -345,6 +351,9 @@ __global__ void __launch_bounds__(DV_WARPS * 32, DV_CTAS_PER_SM) sparse_decode_k
       i0 = 4 * n4;
     }
     for (int i = i0 + tid; i < a.k; i += blockDim.x) cp_async4(smem_u32(s_sel + i), srow + i);
+    if (a.starts != nullptr)
+      for (int r = tid; r <= a.R; r += blockDim.x)
+        cp_async4(smem_u32(s_gst + r), a.starts + (size_t)b * (a.R + 1) + r);
     cp_async_commit();
   }
   cp_async_wait<0>();
@@ -355,7 +364,7 @@ __global__ void __launch_bounds__(DV_WARPS * 32, DV_CTAS_PER_SM) sparse_decode_k
   const int L = s_L;
   const int nb = L <= 0 ? 0 : (L + 3) >> 2;
   int kb = min(a.k, nb);
-  {
+  if (a.starts == nullptr) {
     // the list ends at its first -1 (a selection may hold fewer than
     // min(k, nb) blocks, e.g. one rank's share): valid ids come first, so the
     // predicate "entry < 0" is monotone over the row
@@ -366,15 +375,54 @@ __global__ void __launch_bounds__(DV_WARPS * 32, DV_CTAS_PER_SM) sparse_decode_k
     }
     kb = lo;
   }
-  if (warp == 0) {
+  if (warp == 0 && a.starts != nullptr) {  // the starts came with the selection
     int st[2], ct[2], nt[2];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int r = lane + 32 * h;
       st[h] = ct[h] = nt[h] = 0;
       if (r < a.R) {
-        const int lo = (int)(((long long)r * nb) / a.R);
-        const int hi = (int)(((long long)(r + 1) * nb) / a.R);
+        // clamped: a corrupt start can only shorten a run, never leave the row
+        st[h] = min(max(s_gst[r], 0), kb);
+        ct[h] = min(max(s_gst[r + 1], st[h]), kb) - st[h];
+        nt[h] = (ct[h] + 3) >> 2;
+      }
+    }
+    int inc0 = nt[0], inc1 = nt[1];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y0 = __shfl_up_sync(0xffffffffu, inc0, o), y1 = __shfl_up_sync(0xffffffffu, inc1, o);
+      if (lane >= o) {
+        inc0 += y0;
+        inc1 += y1;
+      }
+    }
+    inc1 += __shfl_sync(0xffffffffu, inc0, 31);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int r = lane + 32 * h;
+      if (r < a.R) {
+        s_st[r] = st[h];
+        s_ct[r] = ct[h];
+        s_pre[r] = (h ? inc1 : inc0) - nt[h];
+      }
+    }
+    const int total = __shfl_sync(0xffffffffu, inc1, 31);
+    if (lane == 0) {
+      s_pre[a.R] = total;
+      if (L < 0 && c == 0 && hg == 0) raise_err(a.err, ERR_LEN);
+    }
+  } else if (warp == 0) {
+    int st[2], ct[2], nt[2];
+    // floor(r nb / R) = r q + floor(r m / R) with nb = q R + m: 32-bit, no overflow
+    const unsigned qR = (unsigned)nb / (unsigned)a.R, mR = (unsigned)nb - qR * (unsigned)a.R;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int r = lane + 32 * h;
+      st[h] = ct[h] = nt[h] = 0;
+      if (r < a.R) {
+        const int lo = (int)((unsigned)r * qR + ((unsigned)r * mR) / (unsigned)a.R);
+        const int hi = (int)((unsigned)(r + 1) * qR + ((unsigned)(r + 1) * mR) / (unsigned)a.R);
         st[h] = lower_bound(s_sel, kb, lo);
         ct[h] = lower_bound(s_sel, kb, hi) - st[h];
         nt[h] = (ct[h] + 3) >> 2;
@@ -749,19 +797,25 @@ cudaError_t launch_qn(const DecodeArgs &a, const DecodePlan &p, int B, cudaStrea
 
 }  // namespace
 
-size_t decode_ws_bytes(const qsa_dims &d, int B, int Qn, int k, int R) {
+size_t decode_ws_starts_offset(const qsa_dims &d, int B, int Qn, int k, int R) {
   const DecodePlan p = plan_decode(d, B, k, R);
   const size_t rows = (size_t)B * p.rb * (Qn < DV_QGROUP ? Qn : DV_QGROUP) * d.Hq;
   const size_t groups = (size_t)(d.Hq + DV_CB_ROWS - 1) / DV_CB_ROWS;
-  return rows * (DV_D + 1) * sizeof(float) + (size_t)B * R * sizeof(int2) +
-         (size_t)B * groups * sizeof(int);
+  const size_t used = rows * (DV_D + 1) * sizeof(float) + (size_t)B * R * sizeof(int2) +
+                      (size_t)B * groups * sizeof(int);
+  return (used + 15) & ~(size_t)15;
+}
+
+size_t decode_ws_bytes(const qsa_dims &d, int B, int Qn, int k, int R) {
+  return decode_ws_starts_offset(d, B, Qn, k, R) + (size_t)B * (R + 1) * sizeof(int32_t);
 }
 
 cudaError_t launch_sparse_decode(const qsa_dims &d, const qsa_cache &c, int B, int Qn,
                                  const int32_t *seq_lens, const void *q, const int32_t *sel,
                                  int k, int R, float *o_part, float *lse_part, void *ws,
                                  unsigned *err, cudaStream_t st, const int32_t *row_start,
-                                 int S, void *m_out, int m_bf16, float *m_lse) {
+                                 int S, void *m_out, int m_bf16, float *m_lse,
+                                 const int32_t *starts) {
   if (B == 0) return cudaSuccess;
   const DecodePlan p = plan_decode(d, B, k, R);
   DecodeArgs a;
@@ -771,6 +825,7 @@ cudaError_t launch_sparse_decode(const qsa_dims &d, const qsa_cache &c, int B, i
   a.block_table = c.block_table;
   a.seq_lens = seq_lens;
   a.sel = sel;
+  a.starts = row_start == nullptr && Qn == 1 ? starts : nullptr;
   a.row_start = row_start;
   a.S = S;
   a.m_out = Qn == 1 ? m_out : nullptr;

@@ -41,6 +41,11 @@ struct TopkArgs {
   int32_t *sel;
   int ld, k;
   unsigned *err;
+  // decode step only (cluster kernel): for every sequence, the R + 1 slice
+  // starts of the selection, st[r] = number of selected blocks below
+  // floor(r nb / R) (st[R] = all of them), [B, R + 1]; nullptr: none
+  int32_t *starts;
+  int R;
 };
 
 // Order-preserving map of fp32 onto uint32 (larger float -> larger key);
@@ -53,7 +58,7 @@ __device__ __forceinline__ uint32_t score_key(float f) {
 
 // CS CTAs per sequence (a cluster of 8 or 4): the host picks the larger one
 // that keeps every cluster of the batch resident at two CTAs per SM.
-template <int CS>
+template <int CS, bool WS>  // WS: write the decode step's slice starts
 __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a) {
   cg::cluster_group cluster = cg::this_cluster();
   const int crank = (int)cluster.block_rank();
@@ -71,14 +76,19 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a) {
   const int nb = L < 0 ? 0 : (L + 3) >> 2;
   int32_t *out = a.sel + (size_t)b * a.k;
   pdl_wait();  // the scores come from the kernel before this one
+  int32_t *st_row = WS ? a.starts + (size_t)b * (a.R + 1) : nullptr;
   if (L < 0 || nb > a.ld) {  // uniform over the cluster
     if (crank == 0 && tid == 0) raise_err(a.err, ERR_LEN);
     for (int i = crank * TK_THREADS + tid; i < a.k; i += CS * TK_THREADS) out[i] = -1;
+    if (WS && crank == 0)
+      for (int r = tid; r <= a.R; r += TK_THREADS) st_row[r] = 0;
     return;
   }
   if (nb <= a.k) {  // every block is kept
     for (int i = crank * TK_THREADS + tid; i < a.k; i += CS * TK_THREADS)
       out[i] = i < nb ? i : -1;
+    if (WS && crank == 0)  // block j sits at position j
+      for (int r = tid; r <= a.R; r += TK_THREADS) st_row[r] = (int)(((long long)r * nb) / a.R);
     return;
   }
 
@@ -201,6 +211,18 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a) {
   cluster.sync();  // no CTA leaves while another still reads its counts
 
   const unsigned lower = (1u << lane) - 1u;
+  // slice boundaries floor(r nb / R), 0 < r < R, in this warp's segment (the
+  // first one at or past its start): the lane holding that block writes the
+  // number of winners before it
+  int rc = 1, jb = 0x7fffffff;  // next boundary index and its block (none: INT_MAX)
+  if (WS) {
+    while (rc < a.R && (rc * nb) / a.R < lo + s0) ++rc;
+    if (rc < a.R) jb = (rc * nb) / a.R;
+    if (crank == 0 && tid == 0) {
+      st_row[0] = 0;
+      st_row[a.R] = a.k;  // nb > k: exactly k winners
+    }
+  }
   for (int base = s0; base < s1; base += 32) {
     const int i = base + lane;
     const uint32_t key = (i < s1 ? keys[i] : 0u) & mask;
@@ -211,6 +233,12 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a) {
     // positions stay below k by construction; the bound only guards the buffer
     const unsigned pos = is_gt ? gb + min(eb, (unsigned)take_eq) : gb + eb;
     if ((is_gt || (is_eq && eb < (unsigned)take_eq)) && pos < (unsigned)a.k) out[pos] = lo + i;
+    // (warp-uniform; a division only per boundary passed; r * nb < 2^25)
+    while (WS && jb < lo + min(base + 32, s1)) {
+      if (lo + i == jb) st_row[rc] = (int)(gb + min(eb, (unsigned)take_eq));
+      ++rc;
+      jb = rc < a.R ? (rc * nb) / a.R : 0x7fffffff;
+    }
     run_gt += __popc(bg);
     run_eq += __popc(be);
   }
@@ -557,9 +585,11 @@ __global__ void __launch_bounds__(TR_THREADS, 1) topk_row_kernel(TopkArgs a) {
 }  // namespace
 
 cudaError_t launch_topk(int B, const int32_t *seq_lens, const float *scores, int ld, int k,
-                        int32_t *sel, unsigned *err, cudaStream_t st) {
+                        int32_t *sel, unsigned *err, cudaStream_t st, int32_t *starts, int R,
+                        bool *wrote_starts) {
+  if (wrote_starts != nullptr) *wrote_starts = false;
   if (B == 0) return cudaSuccess;
-  TopkArgs a{scores, seq_lens, sel, ld, k, err};
+  TopkArgs a{scores, seq_lens, sel, ld, k, err, nullptr, R};
   // clusters of CS CTAs while the batch's clusters all fit at two CTAs per SM
   // (largest CS first, each CTA's keys within its shared memory); beyond
   // that, one CTA per sequence for rows it can hold, else clusters of 8
@@ -582,8 +612,13 @@ cudaError_t launch_topk(int B, const int32_t *seq_lens, const float *scores, int
     return launch_pdl(topk_row_kernel, B, TR_THREADS, smem, st, a);
   }
   if (cs == 0) cs = TOPK_CLUSTER;
-  const void *kern = cs == 8 ? reinterpret_cast<const void *>(topk_kernel<8>)
-                             : reinterpret_cast<const void *>(topk_kernel<4>);
+  a.starts = starts;  // the cluster kernel writes the slice starts
+  if (wrote_starts != nullptr) *wrote_starts = starts != nullptr;
+  const bool ws = starts != nullptr;
+  const void *kern = cs == 8 ? (ws ? reinterpret_cast<const void *>(topk_kernel<8, true>)
+                                   : reinterpret_cast<const void *>(topk_kernel<8, false>))
+                             : (ws ? reinterpret_cast<const void *>(topk_kernel<4, true>)
+                                   : reinterpret_cast<const void *>(topk_kernel<4, false>));
   const int per_cta = (ld + cs - 1) / cs;
   const size_t smem = (size_t)per_cta * 4;
   cudaError_t e = ensure_dynamic_smem(kern, smem);
@@ -602,8 +637,11 @@ cudaError_t launch_topk(int B, const int32_t *seq_lens, const float *scores, int
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cs == 8 ? cudaLaunchKernelEx(&cfg, topk_kernel<8>, a)
-                 : cudaLaunchKernelEx(&cfg, topk_kernel<4>, a);
+  if (cs == 8)
+    return ws ? cudaLaunchKernelEx(&cfg, topk_kernel<8, true>, a)
+              : cudaLaunchKernelEx(&cfg, topk_kernel<8, false>, a);
+  return ws ? cudaLaunchKernelEx(&cfg, topk_kernel<4, true>, a)
+            : cudaLaunchKernelEx(&cfg, topk_kernel<4, false>, a);
 }
 
 }  // namespace qsa

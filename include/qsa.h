@@ -166,10 +166,11 @@ qsa_status qsa_topk_select(int32_t B, const int32_t *seq_lens,
 
 /* Scratch bytes qsa_sparse_decode needs for B sequences, top-k k, R slices.
  * The scratch holds the partial results of slices that several CTAs share,
- * the list of those slices and (for qsa_decode_step's fused merge) one
- * arrival counter per sequence and group of 8 query heads; it needs no
- * initialisation and every call writes what it later reads (calls sharing
- * one scratch buffer must be ordered on the GPU). */
+ * the list of those slices, (for qsa_decode_step's fused merge) one arrival
+ * counter per sequence and group of 8 query heads and, at the end, the R + 1
+ * slice starts per sequence that qsa_decode_step's top-k hands to its decode;
+ * it needs no initialisation and every call writes what it later reads
+ * (calls sharing one scratch buffer must be ordered on the GPU). */
 size_t qsa_sparse_decode_workspace_size(const qsa_dims *dims, int32_t B,
                                         int32_t k, int32_t R);
 

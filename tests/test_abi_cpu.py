@@ -46,11 +46,14 @@ def test_version_and_workspace_sizes(L):
     # (at most one per tile, at least ceil((k/4 + R - 1) / 256) for the page
     # table), keyed by CTA + slice, each 32 heads x (128 + 1) floats; plus one
     # (c_lo, c_hi) pair per (sequence, slice) and one arrival counter per
-    # (sequence, group of 8 query heads) for the decode step's fused merge
+    # (sequence, group of 8 query heads) for the decode step's fused merge;
+    # then, 16-byte aligned, the R + 1 slice starts per sequence that the
+    # decode step's top-k hands to its decode kernel
     for B, k, R, ncb in ((8, 512, 4, 37), (512, 512, 4, 1), (512, 4096, 4, 5),
                          (2, 512, 2, 129), (1, 1, 1, 1)):
+        used = B * (ncb + R - 1) * 32 * 129 * 4 + B * R * 8 + B * 4 * 4
         assert qsa.qsa_sparse_decode_workspace_size(d, B, k, R) == \
-            B * (ncb + R - 1) * 32 * 129 * 4 + B * R * 8 + B * 4 * 4, (B, k, R)
+            (used + 15) // 16 * 16 + B * (R + 1) * 4, (B, k, R)
 
 
 def test_prefill_workspace_sizes(L):

@@ -517,6 +517,30 @@ def test_decode_step_fused_merge_equals_qsa_merge(lens, R):
         _check_seq(run, b)
 
 
+@pytest.mark.parametrize("lens,R", [
+    ([30001, 5000, 77, 12345, 2048, 262144], 4),  # clusters of 8 per selection
+    ([9000, 2049, 40003, 3] * 10, 3),              # 40 rows: clusters of 4
+    ([700, 3000, 1] * 2, 64),                      # more slices than some rows have blocks
+])
+def test_decode_step_slice_starts_equal_the_decode_kernels_own(lens, R):
+    """Inside qsa_decode_step the top-k kernel hands each selection's slice
+    starts to the decode kernel; a standalone qsa_sparse_decode finds them by
+    binary search in the selection. Same starts mean the same tiles and
+    slices, so the partials must be the same bits."""
+    wl = make_custom(DIMS_FULL, lens, k=512, R=R, seed=len(lens) + 7 * R, device=DEV)
+    run = CudaRun(wl)
+    run.step()
+    o2 = torch.full_like(run.buf.o_part, float("nan"))
+    l2 = torch.full_like(run.buf.lse_part, float("nan"))
+    qsa.qsa_sparse_decode(run.dims, run.cache, run.seq_lens, wl.q, run.buf.sel, run.k, run.R,
+                          o2, l2, run.buf.ws)
+    assert qsa.qsa_check_device_errors() == 0
+    assert torch.equal(run.buf.o_part.view(torch.int32), o2.view(torch.int32))
+    assert torch.equal(run.buf.lse_part.view(torch.int32), l2.view(torch.int32))
+    for b in (0, len(lens) - 1):
+        _check_seq(run, b)
+
+
 # ------------------------------------------------------------ multi-query decode
 
 @pytest.mark.parametrize("Qn,R", [(1, 4), (2, 1), (2, 4), (3, 8), (5, 2)])
