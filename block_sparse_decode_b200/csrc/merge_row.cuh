@@ -15,12 +15,16 @@ namespace qsa {
 
 constexpr int MERGE_BATCH = 8;  // slices whose partial outputs are loaded together
 
-// o_part [R, rows, D] and lse_part [R, rows] fp32 (read through L2: they may
-// come from other CTAs of the running grid); out [rows, D] bf16 or fp32.
-// Lane r holds the weights of slices r and r + 32 (R <= 64).
-__device__ __forceinline__ void merge_row(int R, int rows, int D, const float *o_part,
-                                          const float *lse_part, int row, void *out,
-                                          int out_is_bf16, float *lse_out) {
+// The combine of output row `row` (out [rows, D] bf16 or fp32, lse_out
+// [rows] or nullptr) from R partials that the two loaders fetch:
+// load_o(r, d0) gives dims d0..d0+3 of slice r's partial output (d0 < D, a
+// multiple of 4), load_lse(r) its LSE. The arithmetic does not depend on
+// where the partials live, so every caller gets the same bits from the same
+// values. Lane r holds the weights of slices r and r + 32 (R <= 64).
+template <class LoadO, class LoadL>
+__device__ __forceinline__ void merge_row_with(int R, int D, int row, LoadO load_o,
+                                               LoadL load_lse, void *out, int out_is_bf16,
+                                               float *lse_out) {
   const int lane = threadIdx.x & 31;
   const int passes = (D + 127) / 128;
   // the first batch of partial outputs is requested together with the LSEs
@@ -32,13 +36,11 @@ __device__ __forceinline__ void merge_row(int R, int rows, int D, const float *o
 #pragma unroll
     for (int u = 0; u < MERGE_BATCH; ++u) {
       const int r = min(u, R - 1);
-      v0[u] = live ? __ldcg(reinterpret_cast<const float4 *>(o_part + ((size_t)r * rows + row) * D +
-                                                              d0))
-                   : make_float4(0.f, 0.f, 0.f, 0.f);
+      v0[u] = live ? load_o(r, d0) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
   }
-  const float l0 = lane < R ? __ldcg(lse_part + (size_t)lane * rows + row) : -INFINITY;
-  const float l1 = lane + 32 < R ? __ldcg(lse_part + (size_t)(lane + 32) * rows + row) : -INFINITY;
+  const float l0 = lane < R ? load_lse(lane) : -INFINITY;
+  const float l1 = lane + 32 < R ? load_lse(lane + 32) : -INFINITY;
   float M = fmaxf(l0, l1);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
@@ -59,10 +61,7 @@ __device__ __forceinline__ void merge_row(int R, int rows, int D, const float *o
 #pragma unroll
       for (int u = 0; u < MERGE_BATCH; ++u) {
         const int r = min(r0 + u, R - 1);
-        v[u] = it == 0 && r0 == 0 ? v0[u]
-               : live ? __ldcg(reinterpret_cast<const float4 *>(o_part + ((size_t)r * rows + row) * D +
-                                                                 d0))
-                      : make_float4(0.f, 0.f, 0.f, 0.f);
+        v[u] = it == 0 && r0 == 0 ? v0[u] : live ? load_o(r, d0) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll
       for (int u = 0; u < MERGE_BATCH; ++u) {
@@ -89,6 +88,19 @@ __device__ __forceinline__ void merge_row(int R, int rows, int D, const float *o
     }
   }
   if (lane == 0 && lse_out != nullptr) lse_out[row] = wsum > 0.f ? M + logf(wsum) : -INFINITY;
+}
+
+// o_part [R, rows, D] and lse_part [R, rows] fp32 in global memory (read
+// through L2: they may come from other CTAs of the running grid).
+__device__ __forceinline__ void merge_row(int R, int rows, int D, const float *o_part,
+                                          const float *lse_part, int row, void *out,
+                                          int out_is_bf16, float *lse_out) {
+  merge_row_with(
+      R, D, row,
+      [&](int r, int d0) {
+        return __ldcg(reinterpret_cast<const float4 *>(o_part + ((size_t)r * rows + row) * D + d0));
+      },
+      [&](int r) { return __ldcg(lse_part + (size_t)r * rows + row); }, out, out_is_bf16, lse_out);
 }
 
 }  // namespace qsa

@@ -656,6 +656,10 @@ __global__ void __launch_bounds__(DV_WARPS * 32, DV_CTAS_PER_SM) sparse_decode_k
 // of record i of each group of 32 (its LSE loaded in one round trip per 32
 // records, the max taken across the warp); the outputs are then read
 // DV_CB_BATCH records at a time, their weights broadcast from the lanes.
+// SELF (fused merge with R = 1): the slice is the whole selection, so each
+// warp merges its own row straight from registers (no arrival counting, no
+// re-read of o_part).
+template <bool SELF>
 __global__ void __launch_bounds__(DV_CB_ROWS * 32) decode_combine_kernel(DecodeArgs a) {
   pdl_wait();  // the records come from the decode kernel before this one
   pdl_trigger();  // the merge kernel waits for this whole grid
@@ -716,11 +720,24 @@ __global__ void __launch_bounds__(DV_CB_ROWS * 32) decode_combine_kernel(DecodeA
     const int qq = q / a.Hq, h = q % a.Hq;
     const size_t orow = (((size_t)r * a.B + b) * a.Qn + a.q0 + qq) * a.Hq + h;
     const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-    reinterpret_cast<float4 *>(a.o_part + orow * DV_D)[lane] =
-        make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
-    if (lane == 0) a.lse_part[orow] = wsum > 0.f ? M + logf(wsum) : -INFINITY;
+    const float4 res = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+    const float lse = wsum > 0.f ? M + logf(wsum) : -INFINITY;
+    reinterpret_cast<float4 *>(a.o_part + orow * DV_D)[lane] = res;
+    if (lane == 0) a.lse_part[orow] = lse;
+    // (the loaders hand back the values just stored: the bits of qsa_merge)
+    if (SELF)
+      merge_row_with(1, DV_D, b * a.Hq + q, [&](int, int) { return res; },
+                     [&](int) { return lse; }, a.m_out, a.m_bf16, a.m_lse);
+  } else if (SELF && q < a.Hq) {
+    // a selection inside one decode CTA's range, or empty: the decode kernel
+    // wrote the slice's partial (one query per sequence here)
+    const size_t orow = (size_t)b * a.Hq + q;
+    const float4 v = __ldcg(reinterpret_cast<const float4 *>(a.o_part + orow * DV_D) + lane);
+    const float l = __ldcg(a.lse_part + orow);
+    merge_row_with(1, DV_D, b * a.Hq + q, [&](int, int) { return v; }, [&](int) { return l; },
+                   a.m_out, a.m_bf16, a.m_lse);
   }
-  if (a.m_out == nullptr) return;
+  if (SELF || a.m_out == nullptr) return;
   // fused merge (one query per sequence): the CTA whose arrival completes the
   // row group's R slices merges them (its own rows, one warp per head)
   __shared__ int s_last;
@@ -781,9 +798,10 @@ cudaError_t launch_st(const DecodeArgs &a, const DecodePlan &p, int B, cudaStrea
     return a.m_out == nullptr ? e
                               : launch_merge(a.R, B, a.Hq, DV_D, a.o_part, a.lse_part, a.m_out,
                                              a.m_bf16, a.m_lse, st);
-  return launch_pdl(decode_combine_kernel,
-                    dim3((QN * a.Hq + DV_CB_ROWS - 1) / DV_CB_ROWS, a.R, B), DV_CB_ROWS * 32, 0,
-                    st, a);
+  const dim3 grid((QN * a.Hq + DV_CB_ROWS - 1) / DV_CB_ROWS, a.R, B);
+  if (a.m_out != nullptr && a.R == 1)
+    return launch_pdl(decode_combine_kernel<true>, grid, DV_CB_ROWS * 32, 0, st, a);
+  return launch_pdl(decode_combine_kernel<false>, grid, DV_CB_ROWS * 32, 0, st, a);
 }
 
 template <int QN>

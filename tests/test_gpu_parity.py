@@ -495,7 +495,15 @@ def test_steady128x64k_append_steps():
 
 
 @pytest.mark.parametrize("lens,R", [
-    ([30001, 5000, 77, 12345, 2048], 4),   # sequences split over CTAs: fused into the combine
+    # sequences split over CTAs: the merge is fused into the combine kernel,
+    # by the CTA that completes a row group's R slices ...
+    ([30001, 5000, 77, 12345, 2048], 4),
+    ([30001, 5000, 77, 12345, 2048], 3),
+    ([30001, 5000, 77, 12345, 2048], 16),
+    # ... or, with R = 1, by every combine warp for its own row (a 9-token
+    # sequence whose one tile lies in one decode CTA: its partial comes from
+    # the decode kernel)
+    ([70001, 9001, 9, 517], 1),
     ([3000] * 300, 2),                     # one CTA per sequence: the merge kernel
 ])
 def test_decode_step_fused_merge_equals_qsa_merge(lens, R):
