@@ -65,6 +65,8 @@ constexpr int DV_CTAS_PER_SM = 2;
 constexpr size_t DV_SMEM_LIMIT = 113 * 1024;    // shared memory per CTA so that two fit an SM
 constexpr int DV_CB_ROWS = 8;                   // query-head rows per combine CTA
 constexpr int DV_CB_BATCH = 16;                 // records' outputs loaded together (combine)
+constexpr int DV_CG_WARPS = 8;                  // warps of a combine CTA that also merges (R >= 2)
+constexpr int DV_CB_PER_SM = 2;                 // combine CTAs resident per SM (256 threads, ~104 registers)
 constexpr int DV_QGROUP = 2;                    // queries of a sequence per pass over K/V
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
@@ -651,79 +653,89 @@ __global__ void __launch_bounds__(DV_WARPS * 32, DV_CTAS_PER_SM) sparse_decode_k
   }
 }
 
-// (6) One CTA per (group of DV_CB_ROWS query rows, slice, sequence); warp =
-// one (query, head) row, lane l owns dims 4l..4l+3. Lane i holds the weight
-// of record i of each group of 32 (its LSE loaded in one round trip per 32
+// (6) Merge of one slice's records for one row q = (query of the group,
+// head), by one warp; lane l owns dims 4l..4l+3. Lane i holds the weight of
+// record i of each group of 32 (its LSE loaded in one round trip per 32
 // records, the max taken across the warp); the outputs are then read
 // DV_CB_BATCH records at a time, their weights broadcast from the lanes.
-// SELF (fused merge with R = 1): the slice is the whole selection, so each
-// warp merges its own row straight from registers (no arrival counting, no
-// re-read of o_part).
+// Writes the slice partial to o_part / lse_part and returns it in res / lse;
+// returns false for a slice the decode kernel wrote itself (inside one CTA's
+// range, or empty).
+__device__ __forceinline__ bool combine_slice_row(const DecodeArgs &a, int b, int r, int q,
+                                                  int lane, float4 &res, float &lse) {
+  const int2 sp = a.span[(size_t)b * a.R + r];
+  if (sp.y <= sp.x) return false;
+  const int n = sp.y - sp.x + 1;
+  const size_t stride = (size_t)a.qn * a.Hq;                         // between records
+  const size_t row0 = ((size_t)b * a.rb + sp.x + r) * stride + q;    // record i at row0 + i*stride
+  // the first DV_CB_BATCH records' outputs are requested together with the
+  // LSEs (one round trip instead of two for slices of that many records)
+  float4 v[DV_CB_BATCH];
+#pragma unroll
+  for (int u = 0; u < DV_CB_BATCH; ++u) {
+    const size_t rr = row0 + (size_t)min(u, n - 1) * stride;
+    v[u] = __ldcg(reinterpret_cast<const float4 *>(a.rec_o + rr * DV_D) + lane);
+  }
+  float M = -INFINITY;
+  for (int i0 = 0; i0 < n; i0 += 32) {
+    const float l = i0 + lane < n ? __ldcg(a.rec_lse + row0 + (size_t)(i0 + lane) * stride)
+                                  : -INFINITY;
+    M = fmaxf(M, l);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  float acc[4] = {0.f, 0.f, 0.f, 0.f}, wsum = 0.f;
+  if (M != -INFINITY) {
+    for (int i0 = 0; i0 < n; i0 += 32) {
+      const float l = i0 + lane < n ? __ldcg(a.rec_lse + row0 + (size_t)(i0 + lane) * stride)
+                                    : -INFINITY;
+      const float wl = l == -INFINITY ? 0.f : __expf(l - M);  // weight of record i0 + lane
+      const int m = min(32, n - i0);
+      for (int u0 = 0; u0 < m; u0 += DV_CB_BATCH) {
+        if (i0 != 0 || u0 != 0) {  // (the first batch is in v already)
+#pragma unroll
+          for (int u = 0; u < DV_CB_BATCH; ++u) {
+            const size_t rr = row0 + (size_t)(i0 + min(u0 + u, m - 1)) * stride;
+            v[u] = __ldcg(reinterpret_cast<const float4 *>(a.rec_o + rr * DV_D) + lane);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < DV_CB_BATCH; ++u) {
+          const float w = __shfl_sync(0xffffffffu, wl, (u0 + u) & 31);
+          if (u0 + u < m && w != 0.f) {  // a record of a query that saw nothing holds zeros
+            wsum += w;
+            acc[0] += w * v[u].x;
+            acc[1] += w * v[u].y;
+            acc[2] += w * v[u].z;
+            acc[3] += w * v[u].w;
+          }
+        }
+      }
+    }
+  }
+  const int qq = q / a.Hq, h = q % a.Hq;
+  const size_t orow = (((size_t)r * a.B + b) * a.Qn + a.q0 + qq) * a.Hq + h;
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+  res = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+  lse = wsum > 0.f ? M + logf(wsum) : -INFINITY;
+  reinterpret_cast<float4 *>(a.o_part + orow * DV_D)[lane] = res;
+  if (lane == 0) a.lse_part[orow] = lse;
+  return true;
+}
+
+// One CTA per (group of DV_CB_ROWS query rows, slice, sequence), one warp per
+// row. The fused merge (one query per sequence): with R = 1 (SELF) each warp
+// merges its own row from the registers holding its slice partial; otherwise
+// the CTA whose arrival completes the row group's R slices merges them.
 template <bool SELF>
 __global__ void __launch_bounds__(DV_CB_ROWS * 32) decode_combine_kernel(DecodeArgs a) {
   pdl_wait();  // the records come from the decode kernel before this one
   pdl_trigger();  // the merge kernel waits for this whole grid
   const int b = blockIdx.z, r = blockIdx.y;
-  // row = (query qq of the group, head h)
   const int q = blockIdx.x * DV_CB_ROWS + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-  const int2 sp = a.span[(size_t)b * a.R + r];
-  // a slice inside one CTA's range was written by the decode kernel itself
-  if (sp.y > sp.x && q < a.qn * a.Hq) {
-    const int n = sp.y - sp.x + 1;
-    const size_t stride = (size_t)a.qn * a.Hq;                         // between records
-    const size_t row0 = ((size_t)b * a.rb + sp.x + r) * stride + q;    // record i at row0 + i*stride
-    // the first DV_CB_BATCH records' outputs are requested together with the
-    // LSEs (one round trip instead of two for slices of that many records)
-    float4 v[DV_CB_BATCH];
-#pragma unroll
-    for (int u = 0; u < DV_CB_BATCH; ++u) {
-      const size_t rr = row0 + (size_t)min(u, n - 1) * stride;
-      v[u] = __ldcg(reinterpret_cast<const float4 *>(a.rec_o + rr * DV_D) + lane);
-    }
-    float M = -INFINITY;
-    for (int i0 = 0; i0 < n; i0 += 32) {
-      const float l = i0 + lane < n ? __ldcg(a.rec_lse + row0 + (size_t)(i0 + lane) * stride)
-                                    : -INFINITY;
-      M = fmaxf(M, l);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float acc[4] = {0.f, 0.f, 0.f, 0.f}, wsum = 0.f;
-    if (M != -INFINITY) {
-      for (int i0 = 0; i0 < n; i0 += 32) {
-        const float l = i0 + lane < n ? __ldcg(a.rec_lse + row0 + (size_t)(i0 + lane) * stride)
-                                      : -INFINITY;
-        const float wl = l == -INFINITY ? 0.f : __expf(l - M);  // weight of record i0 + lane
-        const int m = min(32, n - i0);
-        for (int u0 = 0; u0 < m; u0 += DV_CB_BATCH) {
-          if (i0 != 0 || u0 != 0) {  // (the first batch is in v already)
-#pragma unroll
-            for (int u = 0; u < DV_CB_BATCH; ++u) {
-              const size_t rr = row0 + (size_t)(i0 + min(u0 + u, m - 1)) * stride;
-              v[u] = __ldcg(reinterpret_cast<const float4 *>(a.rec_o + rr * DV_D) + lane);
-            }
-          }
-#pragma unroll
-          for (int u = 0; u < DV_CB_BATCH; ++u) {
-            const float w = __shfl_sync(0xffffffffu, wl, (u0 + u) & 31);
-            if (u0 + u < m && w != 0.f) {  // a record of a query that saw nothing holds zeros
-              wsum += w;
-              acc[0] += w * v[u].x;
-              acc[1] += w * v[u].y;
-              acc[2] += w * v[u].z;
-              acc[3] += w * v[u].w;
-            }
-          }
-        }
-      }
-    }
-    const int qq = q / a.Hq, h = q % a.Hq;
-    const size_t orow = (((size_t)r * a.B + b) * a.Qn + a.q0 + qq) * a.Hq + h;
-    const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-    const float4 res = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
-    const float lse = wsum > 0.f ? M + logf(wsum) : -INFINITY;
-    reinterpret_cast<float4 *>(a.o_part + orow * DV_D)[lane] = res;
-    if (lane == 0) a.lse_part[orow] = lse;
+  float4 res;
+  float lse;
+  if (q < a.qn * a.Hq && combine_slice_row(a, b, r, q, lane, res, lse)) {
     // (the loaders hand back the values just stored: the bits of qsa_merge)
     if (SELF)
       merge_row_with(1, DV_D, b * a.Hq + q, [&](int, int) { return res; },
@@ -753,6 +765,41 @@ __global__ void __launch_bounds__(DV_CB_ROWS * 32) decode_combine_kernel(DecodeA
   if (q < a.Hq)
     merge_row(a.R, a.B * a.Hq, DV_D, a.o_part, a.lse_part, b * a.Hq + q, a.m_out, a.m_bf16,
               a.m_lse);
+}
+
+// The fused merge with 2 <= R <= DV_CG_WARPS (one query per sequence) when
+// all its CTAs are resident at once: one CTA per (group of DV_CG_WARPS / R
+// query heads, sequence), one warp per (slice, head). Each warp merges its
+// slice's records for its head (or takes the partial the decode kernel
+// wrote) and keeps the result in shared memory; after one block barrier the
+// warps of slice 0 merge the R slices of their heads: no arrival counting,
+// no re-read of o_part.
+__global__ void __launch_bounds__(DV_CG_WARPS * 32) decode_combine_group_kernel(DecodeArgs a) {
+  pdl_wait();  // the records come from the decode kernel before this one
+  pdl_trigger();
+  extern __shared__ float4 g_o[];  // [R][rows][32] slice partials, then the LSEs [R][rows]
+  const int rows = DV_CG_WARPS / a.R;
+  float *g_l = reinterpret_cast<float *>(g_o + (size_t)a.R * rows * 32);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = warp / rows, i = warp - r * rows;
+  const int b = blockIdx.y, q = blockIdx.x * rows + i;
+  if (r < a.R && q < a.Hq) {
+    float4 res;
+    float lse;
+    if (!combine_slice_row(a, b, r, q, lane, res, lse)) {
+      const size_t orow = ((size_t)r * a.B + b) * a.Hq + q;
+      res = __ldcg(reinterpret_cast<const float4 *>(a.o_part + orow * DV_D) + lane);
+      lse = __ldcg(a.lse_part + orow);
+    }
+    g_o[(r * rows + i) * 32 + lane] = res;
+    if (lane == 0) g_l[r * rows + i] = lse;
+  }
+  __syncthreads();
+  // (the same values as in o_part / lse_part: the bits of qsa_merge)
+  if (r == 0 && q < a.Hq)
+    merge_row_with(
+        a.R, DV_D, b * a.Hq + q, [&](int rr, int d0) { return g_o[(rr * rows + i) * 32 + (d0 >> 2)]; },
+        [&](int rr) { return g_l[rr * rows + i]; }, a.m_out, a.m_bf16, a.m_lse);
 }
 
 struct DecodePlan {
@@ -801,6 +848,19 @@ cudaError_t launch_st(const DecodeArgs &a, const DecodePlan &p, int B, cudaStrea
   const dim3 grid((QN * a.Hq + DV_CB_ROWS - 1) / DV_CB_ROWS, a.R, B);
   if (a.m_out != nullptr && a.R == 1)
     return launch_pdl(decode_combine_kernel<true>, grid, DV_CB_ROWS * 32, 0, st, a);
+  // A CTA holding all R slices of its heads lasts as long as its slowest
+  // slice: it shortens the chain while every combine CTA is resident at once,
+  // but costs time when the CTAs run in several waves (then a slice's CTA
+  // that finishes early makes room for the next)
+  if (a.m_out != nullptr && a.R <= DV_CG_WARPS) {
+    const int rows = DV_CG_WARPS / a.R;
+    const long long ctas = (long long)((a.Hq + rows - 1) / rows) * B;
+    if (ctas <= (long long)DV_CB_PER_SM * device_sm_count()) {
+      const size_t smem = (size_t)a.R * rows * (32 * sizeof(float4) + sizeof(float));
+      return launch_pdl(decode_combine_group_kernel, dim3((a.Hq + rows - 1) / rows, B),
+                        a.R * rows * 32, smem, st, a);
+    }
+  }
   return launch_pdl(decode_combine_kernel<false>, grid, DV_CB_ROWS * 32, 0, st, a);
 }
 

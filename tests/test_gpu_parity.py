@@ -495,15 +495,19 @@ def test_steady128x64k_append_steps():
 
 
 @pytest.mark.parametrize("lens,R", [
-    # sequences split over CTAs: the merge is fused into the combine kernel,
-    # by the CTA that completes a row group's R slices ...
+    # sequences split over CTAs: the merge is fused into the combine; with
+    # 2 <= R <= 8 and few sequences one CTA holds every slice of its heads
+    # and merges them in shared memory (a 9-token sequence, whose one tile
+    # lies in one decode CTA, has its partial from the decode kernel) ...
     ([30001, 5000, 77, 12345, 2048], 4),
-    ([30001, 5000, 77, 12345, 2048], 3),
-    ([30001, 5000, 77, 12345, 2048], 16),
-    # ... or, with R = 1, by every combine warp for its own row (a 9-token
-    # sequence whose one tile lies in one decode CTA: its partial comes from
-    # the decode kernel)
+    ([30001, 5000, 9, 12345, 2048], 3),
+    ([30001, 5000, 77, 12345, 2048], 8),
+    # ... with R = 1 every combine warp merges its own row ...
     ([70001, 9001, 9, 517], 1),
+    # ... and beyond 8 slices, or with more combine CTAs than fit the GPU at
+    # once, the CTA completing a row group's slices merges
+    ([30001, 5000, 77, 12345, 2048], 16),
+    ([30001, 5000, 77, 12345, 2048] * 16, 4),
     ([3000] * 300, 2),                     # one CTA per sequence: the merge kernel
 ])
 def test_decode_step_fused_merge_equals_qsa_merge(lens, R):
