@@ -35,10 +35,13 @@
 // ordered). (6) A second, small kernel, launched as a programmatic dependent
 // of the first, combines the partials of each shared slice once all streaming
 // is done (every load of a row batched, so it costs a couple of L2 round
-// trips). Inside the one-call decode step it also merges the R slices: each
-// of its CTAs counts its arrival per (sequence, group of heads) after a
-// fence, and the one that completes the group merges it (merge_row.cuh, the
-// arithmetic of qsa_merge).
+// trips). Inside the one-call decode step it also merges the R slices
+// (merge_row.cuh, the arithmetic of qsa_merge), in one of three forms: with
+// R = 1 each warp merges its own row from registers; with 2 <= R <= 8 and
+// every combine CTA resident at once, a CTA holds all R slices of its heads
+// (a warp per slice and head) and merges them in shared memory after a
+// block barrier; otherwise each CTA counts its arrival per (sequence, group
+// of heads) after a fence, and the one that completes the group merges it.
 //
 // The same kernels serve sparse prefill rows (row_start != nullptr): a row is
 // a query of a chunk; it takes its sequence's block-table row and its own
