@@ -275,9 +275,8 @@ qsa_status qsa_merge(int32_t R, int32_t B, int32_t Hq, int32_t D,
  * the arguments documented at each of those calls (the merge writes `out`
  * [B, Hq, D] and `lse_out` [B, Hq] from o_part / lse_part, which also hold
  * the R partials afterwards). Here the merge runs inside the decode's last
- * kernel (the CTA that completes a group of rows merges them, with the
- * arithmetic of qsa_merge, so the results are the same bits), which saves a
- * launch. The page orders the steps (section "What the pull request
+ * kernel, with the arithmetic of qsa_merge, so the results are the same
+ * bits; this saves a launch. The page orders the steps (section "What the pull request
  * actually changes"); the single call is an interface convenience of this
  * library that saves the caller four calls. The calls' own argument checks
  * apply; the first failing call stops the sequence and its status is
